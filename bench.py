@@ -1,0 +1,445 @@
+#!/usr/bin/env python
+"""Throughput of the gated delta rule (Gated DeltaNet token mixing) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line.  A step is one gdn_prefill call over the mid-size prefill
+workload (B=2, T=4096, H=16, dk=dv=128, bf16 q/k/v, fp32 g/beta/state, S0=0);
+`value` is whole-job prefill tokens/s with inputs resident in HBM.  The same line
+carries the decode workload (256 sequences x 128 single-token steps, H=32,
+dk=dv=128, bf16 q/k/v, fp32 state ~ N(0, 0.02)) under "decode", the roofline of
+each kernel, the end-to-end figure through the C ABI with host buffers ("e2e"),
+and the CPU oracle timed on this host ("cpu_baseline").
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
+the launching stream; a 256 MB buffer is written between prefill steps (outside
+the events) so no step starts with its inputs in the 126 MB L2.  The decode state
+(537 MB) is larger than L2.  With N > 1 (torchrun) every rank runs its own replica
+of the workload (the layer has no cross-GPU exchange), the job time is the max over
+ranks and `value` counts all ranks' tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_token_b200 import inputs  # noqa: E402
+
+METRIC = "GDN prefill tokens/s and decode tokens/s on 1 B200; % of tensor/HBM roofline"
+PREFILL_W = 1
+DECODE_W = 4
+CHUNK = 64
+
+
+# ----------------------------------------------------------------- algorithmic counts
+def prefill_flops_per_token_head(dk: int, dv: int, C: int = CHUNK) -> int:
+    """The chunked method's contractions at tile shape, per token per value head:
+    [K;Q]K^T (2 C dk), K^T T'^T / V^T T''^T (C dk + C dv), W S and Q S (2 dk dv),
+    (P U) (C dv) and the state update K~^T U (dk dv), times 2 flops per MAC."""
+    return 2 * (C * (3 * dk + 2 * dv) + 3 * dk * dv)
+
+
+def prefill_bytes(w) -> int:
+    """q/k/v/out once in the I/O dtype, g and beta in fp32, S0 and S_final once."""
+    e = torch.tensor([], dtype=w.dtype).element_size()
+    T = w.tokens
+    b = T * (2 * w.H_qk * w.dk + 2 * w.H_v * w.dv) * e + T * w.H_v * 8
+    b += w.num_seqs * w.H_v * w.dk * w.dv * 4 * (2 if w.s0_std else 1)
+    return b
+
+
+def decode_bytes_per_step(w) -> int:
+    e = torch.tensor([], dtype=w.dtype).element_size()
+    N = w.decode_seqs
+    return (N * w.H_v * w.dk * w.dv * 4 * 2 + N * (2 * w.H_qk * w.dk + 2 * w.H_v * w.dv) * e
+            + N * w.H_v * 8)
+
+
+def decode_flops_per_step(w) -> int:
+    # a = S^T k, b = S^T q, S <- alpha S + k u^T: 3 MACs per state element
+    return 2 * 3 * w.decode_seqs * w.H_v * w.dk * w.dv
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def profiled_traffic(kernel_key: str, source_file: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    kernel source as it is now (sha256 of the .cu file recorded in the summary)."""
+    summary = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(summary):
+        return None
+    sha = hashlib.sha256(open(source_file, "rb").read()).hexdigest()[:16]
+    for line in open(summary):
+        parts = line.split()
+        if len(parts) >= 3 and parts[0] == kernel_key and parts[1] == sha:
+            return int(float(parts[2]))
+    return None
+
+
+# -------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append((float(p[1]), float(p[2]), p[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        load = [r for r in rows if r[0] > 0.5 * r[1]] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, x in enumerate(r[2]) if x == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------- our arm
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def time_prefill(gdn, x, w, steps, warmup, stream, flush):
+    B, T = len(w.seq_lens), w.seq_lens[0]
+    view = lambda t: t.view(B, T, *t.shape[1:])
+    args = [view(x[n]) for n in ("q", "k", "v", "g", "beta")]
+    out = torch.empty_like(args[2])
+    S_final = torch.empty(B, w.H_v, w.dk, w.dv, dtype=torch.float32, device=out.device)
+    ws = gdn.prefill_workspace(B, w.tokens, w.H_v, w.dk, w.dv, out.device)
+    call = lambda: gdn.gdn_prefill(*args, None, None, out=out, S_final=S_final, workspace=ws,
+                                   stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush_l2(flush)
+            call()
+    stream.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            flush_l2(flush)
+            a.record(stream)
+            call()
+            b.record(stream)
+    stream.synchronize()
+    times = [a.elapsed_time(b) for a, b in evs]
+    status = gdn.gdn_get_device_error(ws, stream)
+    return times, status
+
+
+def time_prefill_e2e(gdn, w, steps, warmup, stream, device):
+    """Through the public API with HOST buffers: pinned H2D of the step's inputs, the
+    prefill, and D2H of its result (outputs and final state), all inside the events."""
+    B, T = len(w.seq_lens), w.seq_lens[0]
+    xh = inputs.prefill_inputs(w, device="cpu")
+    host = {n: xh[n].view(B, T, *xh[n].shape[1:]).pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    dev = {n: torch.empty_like(t, device=device) for n, t in host.items()}
+    out_h = torch.empty(host["v"].shape, dtype=w.dtype).pin_memory()
+    S_h = torch.empty(B, w.H_v, w.dk, w.dv, dtype=torch.float32).pin_memory()
+    out_d = torch.empty_like(out_h, device=device)
+    S_d = torch.empty_like(S_h, device=device)
+    ws = gdn.prefill_workspace(B, w.tokens, w.H_v, w.dk, w.dv, device)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + S_h.numel() * 4
+
+    def step():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        gdn.gdn_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], None, None,
+                        out=out_d, S_final=S_d, workspace=ws, stream=stream)
+        out_h.copy_(out_d, non_blocking=True)
+        S_h.copy_(S_d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    stream.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            a.record(stream)
+            step()
+            b.record(stream)
+    stream.synchronize()
+    return [a.elapsed_time(b) for a, b in evs], h2d, d2h
+
+
+def time_decode(gdn, w, passes, warmup, stream, device):
+    """`passes` timed passes of all decode steps (each pass: decode_steps launches)."""
+    S = inputs.decode_state(w, device)
+    xs = [inputs.decode_step_inputs(w, s, device) for s in range(w.decode_steps)]
+    outs = [torch.empty_like(x["v"]) for x in xs]
+
+    def one_pass():
+        for x, o in zip(xs, outs):
+            gdn.gdn_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S, out=o, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one_pass()
+    stream.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(passes)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            a.record(stream)
+            one_pass()
+            b.record(stream)
+    stream.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def cpu_baseline_prefill(w, max_tokens=None):
+    """The oracle (float variant, all host cores) on the prefill workload, timed."""
+    import oracle
+    x = inputs.prefill_inputs(w, device="cpu")
+    cu = x["cu_seqlens"]
+    if max_tokens is not None and w.tokens > max_tokens:
+        lens = [min(n, max_tokens // len(w.seq_lens)) for n in w.seq_lens]
+        parts = [slice(int(cu[i]), int(cu[i]) + lens[i]) for i in range(len(lens))]
+        pick = lambda t: torch.cat([t[p] for p in parts])
+        x = {n: pick(x[n]) for n in ("q", "k", "v", "g", "beta")} | {"S0": x["S0"]}
+        cu = inputs.cu_seqlens_of(lens)
+    q, k, v, g, beta = (x[n].float().numpy() for n in ("q", "k", "v", "g", "beta"))
+    S0 = None if x["S0"] is None else x["S0"].numpy()
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, g, beta, S0=S0, cu_seqlens=cu.numpy(), precision="f32",
+                     threads=threads)
+    dt = time.perf_counter() - t0
+    ntok = int(cu[-1])
+    return {"value": ntok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"{ntok} tokens x {w.H_v} heads of {w.name} (sequential fp32 recurrence, "
+                      f"{threads} threads over (sequence, head))"}
+
+
+def cpu_baseline_decode(w, steps=2):
+    import oracle
+    S = inputs.decode_state(w, "cpu").numpy()
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    for s in range(steps):
+        x = inputs.decode_step_inputs(w, s, "cpu")
+        q, k, v, g, beta = (x[n].float().numpy() for n in ("q", "k", "v", "g", "beta"))
+        import numpy as np
+        cu = np.arange(w.decode_seqs + 1, dtype=np.int64)
+        _, S = oracle.recurrent(q, k, v, g, beta, S0=S, cu_seqlens=cu, precision="f32",
+                                threads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": steps * w.decode_seqs / dt, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle", "seconds": dt,
+            "sample": f"{steps} of {w.decode_steps} decode steps x {w.decode_seqs} sequences x "
+                      f"{w.H_v} heads of {w.name}"}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world <= 1:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    rank, world, local = dist_init()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import linear_attention_token_b200 as gdn
+    gdn.lib()                                   # loud failure if libgdn.so is missing
+    peaks = load_peaks()
+    wp, wd = inputs.get(PREFILL_W), inputs.get(DECODE_W)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    x = inputs.prefill_inputs(wp, device=device)
+
+    barrier(world)
+    with ClockSampler(local) as clk:
+        times, status = time_prefill(gdn, x, wp, args.steps, max(args.warmup, 3), stream, flush)
+        barrier(world)
+        dec_passes = max(1, min(args.steps, 5))
+        dtimes = time_decode(gdn, wd, dec_passes, max(1, min(args.warmup, 3)), stream, device)
+        barrier(world)
+    clocks = clk.summary()
+    if status != 0:
+        raise RuntimeError(f"device error after prefill: {gdn.gdn_status_string(status)}")
+
+    ms_prefill = max_over_ranks(sum(times) / len(times), world)
+    ms_decode_pass = max_over_ranks(sum(dtimes) / len(dtimes), world)
+    e2e_times, h2d, d2h = time_prefill_e2e(gdn, wp, max(3, args.steps // 2), 2, stream, device)
+    ms_e2e = max_over_ranks(sum(e2e_times) / len(e2e_times), world)
+
+    tok = wp.tokens
+    flops = prefill_flops_per_token_head(wp.dk, wp.dv) * tok * wp.H_v
+    pf_tflops = flops / (ms_prefill * 1e-3) / 1e12
+    pf_bytes = prefill_bytes(wp)
+    tc_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "prefill_tc.cu")
+    dec_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode.cu")
+    ms_dec_step = ms_decode_pass / wd.decode_steps
+    dec_bytes = decode_bytes_per_step(wd)
+    dec_gbs = dec_bytes / (ms_dec_step * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC,
+        "value": world * tok / (ms_prefill * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_prefill,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; q,k ~ N(0,1) L2-normalised, v ~ N(0,1), g = -softplus(N(0,1)), "
+                "beta = sigmoid(N(0,1)))",
+        "config": {"workload": wp.name, "B": len(wp.seq_lens), "T": wp.seq_lens[0],
+                   "H_qk": wp.H_qk, "H_v": wp.H_v, "dk": wp.dk, "dv": wp.dv, "chunk": CHUNK,
+                   "state": "fp32", "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "l2": "256 MB buffer written between timed prefill steps (outside the events)"},
+        "roofline": {"bound": "tensor", "achieved": pf_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": pf_tflops / peaks["bf16_tflops"],
+                     "traffic": profiled_traffic("prefill", tc_src),
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "flops_per_launch": flops, "algorithmic_bytes_per_launch": pf_bytes,
+                     "hbm_frac": pf_bytes / (ms_prefill * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "decode": {
+            "workload": wd.name, "value": world * wd.decode_seqs / (ms_dec_step * 1e-3),
+            "unit": "tokens/s", "ms_per_step": ms_dec_step, "passes": dec_passes,
+            "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic("decode", dec_src),
+                         "peak_source": f"{peaks['source']} copy bandwidth",
+                         "algorithmic_bytes_per_launch": dec_bytes},
+        },
+        "e2e": {"value": world * tok / (ms_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "gdn_prefill via the C ABI; pinned host inputs copied in and outputs + "
+                        "final state copied out inside the timed region"},
+        "gpu_launches": args.steps + dec_passes * wd.decode_steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(wp)
+        line["decode"]["cpu_baseline"] = cpu_baseline_decode(wd)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, on our arm's workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wp = inputs.get(PREFILL_W)
+    for _ in range(args.warmup):
+        cpu_baseline_prefill(wp, max_tokens=512)
+    runs = [cpu_baseline_prefill(wp) for _ in range(args.steps)]
+    secs = [r["seconds"] for r in runs]
+    ms = 1e3 * sum(secs) / len(secs)
+    v = wp.tokens / (ms * 1e-3)
+    base = dict(runs[0])
+    base["value"] = v
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wp.name, "B": len(wp.seq_lens), "T": wp.seq_lens[0],
+                   "H_qk": wp.H_qk, "H_v": wp.H_v, "dk": wp.dk, "dv": wp.dv},
+        "cpu_baseline": base,
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,123 @@
+/* libgdn — the gated delta rule (Gated DeltaNet token mixing) on one NVIDIA B200.
+ *
+ * Operation ("論文解説: Qwen3.8-Next の設計" (ta-paperlens), section "GDNの中身",
+ * Eq. (1), the ranges stated under it, and the one-token concept code beside it):
+ *
+ *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t                       (read after the update)
+ *
+ * per (sequence, value head), with alpha_t = exp(g_t) (the decay gate, in (0,1)
+ * for g_t < 0) and beta_t the write strength.  S is a dk x dv fp32 matrix, row
+ * index = key dimension, dv contiguous.
+ *
+ * Layouts (all row-major and contiguous; B sequences are folded into tokens):
+ *   q, k       [T_total, H_qk, dk]     dtype (GDN_F32 or GDN_BF16)
+ *   v, out     [T_total, H_v,  dv]     dtype
+ *   g, beta    [T_total, H_v]          fp32
+ *   S0/S_final [num_seqs, H_v, dk, dv] fp32
+ * Value head h reads q/k head h / (H_v / H_qk) (grouped heads; H_v % H_qk == 0).
+ *
+ * Ownership: the caller owns every buffer (device memory unless stated).  No
+ * entry point allocates, frees or synchronises, except gdn_get_device_error,
+ * which synchronises the stream it is given.  Work is enqueued on `stream` and
+ * completes asynchronously.
+ *
+ * Errors: argument checks run on the host before anything is enqueued and return
+ * GDN_ERR_INVALID_ARG or GDN_ERR_UNSUPPORTED with nothing launched.  A failed
+ * launch returns GDN_ERR_CUDA.  A device-side wait that runs out of its bounded
+ * iteration budget records GDN_ERR_TIMEOUT in the workspace; read it with
+ * gdn_get_device_error.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, bad offsets */
+    GDN_ERR_UNSUPPORTED = 2,   /* a valid combination this build has no kernel for       */
+    GDN_ERR_CUDA = 3,          /* a CUDA runtime call or a kernel launch failed          */
+    GDN_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (see the workspace)  */
+} gdn_status;
+
+typedef enum {
+    GDN_F32 = 0,               /* q, k, v, out in fp32 (CUDA-core kernels)             */
+    GDN_BF16 = 1               /* q, k, v, out in bf16 (tensor-core prefill, dk=dv=128) */
+} gdn_dtype;
+
+/* L2-normalise q and k per (token, head) inside the kernel: x / sqrt(sum x^2 + 1e-6). */
+#define GDN_FLAG_QK_L2NORM 1u
+/* Prefill: use the CUDA-core chunked kernel even where the tensor-core one applies. */
+#define GDN_FLAG_FORCE_CUDA_CORE 2u
+
+/* Bytes of device workspace gdn_prefill needs for these sizes (at least 256).
+ * The workspace holds the device error word; it must be zero-filled before its
+ * first use and must stay allocated while work that uses it is in flight. */
+size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t T_total, int32_t H_v, int32_t dk,
+                                  int32_t dv);
+
+/* Chunked prefill over whole sequences: Eq. (1) for every token, all outputs, and
+ * the final state.  Chunks of 64 tokens are re-associated exactly (the WY / UT
+ * form of the rule); results equal the token-by-token recurrence up to rounding.
+ *
+ *   q, k, v, g, beta : inputs in the layouts above (T_total tokens).
+ *   S0               : initial state per sequence, or NULL for zero.
+ *   out              : [T_total, H_v, dv] outputs, written.
+ *   S_final          : final state per sequence, or NULL to skip.  May equal S0.
+ *   cu_seqlens       : DEVICE int32[num_seqs + 1] token offsets (non-decreasing,
+ *                      cu_seqlens[0] = 0, cu_seqlens[num_seqs] = T), or NULL for a
+ *                      dense batch of B sequences of T tokens each.
+ *   num_seqs         : number of sequences when cu_seqlens != NULL (then B must be 1);
+ *                      ignored (taken as B) when cu_seqlens == NULL.
+ *   B, T             : dense batch shape; T_total = B * T.
+ *   H_qk, H_v, dk, dv: heads and head dims; dk, dv in {64, 128}; H_v % H_qk == 0.
+ *   dtype            : element type of q, k, v, out.
+ *   scale            : read-out multiplier (1.0 for the plain rule).
+ *   flags            : GDN_FLAG_* bits.
+ *   workspace        : device scratch of at least gdn_prefill_workspace_size bytes.
+ * Pointers to q, k, v, out, S0, S_final must be 16-byte aligned; g, beta, cu_seqlens
+ * 4-byte aligned.  When there are no tokens (T_total == 0) q, k, v, g, beta, out may be
+ * NULL and only S_final is written (a copy of S0, or zero).  g must be finite (alpha = 0
+ * is reached by a large negative g). */
+gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *S0, void *out, float *S_final,
+                       const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int64_t T,
+                       int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype,
+                       float scale, uint32_t flags, void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/* One decode step: Eq. (1) applied once per (sequence, value head), in place.
+ * The one-token concept code of the same section is this step; its erase term is
+ * taken as in Eq. (1), i.e. u = beta (v - alpha S^T k), S <- alpha S + k u^T,
+ * o = scale * S^T q, each state element read once and written once.
+ *
+ *   q, k    : [N, H_qk, dk] dtype;  v, out : [N, H_v, dv] dtype
+ *   g, beta : [N, H_v] fp32
+ *   S_inout : [N, H_v, dk, dv] fp32, updated in place
+ * dk, dv in {64, 128}; H_v % H_qk == 0; q, k, v, out, S_inout 16-byte aligned.
+ * N == 0 is a no-op (the pointers may then be NULL). */
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, float *S_inout, void *out, int32_t N,
+                           int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype,
+                           float scale, uint32_t flags, cudaStream_t stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded in
+ * `workspace` (GDN_OK if none) and clears it.  GDN_ERR_CUDA if the stream itself
+ * reports an error. */
+gdn_status gdn_get_device_error(void *workspace, cudaStream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char *gdn_status_string(gdn_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,160 @@
+"""ctypes binding of libgdn (include/gdn.h): argument marshalling only.
+
+Every step of the gated delta rule runs in libgdn's CUDA kernels; this module
+passes torch device pointers, sizes and the current CUDA stream through the C ABI
+and turns status codes into exceptions.  There is no fallback: if libgdn.so is
+missing, or a tensor is not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
+GDN_F32, GDN_BF16 = 0, 1
+GDN_FLAG_QK_L2NORM = 1
+GDN_FLAG_FORCE_CUDA_CORE = 2
+
+# every symbol include/gdn.h declares
+EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
+            "gdn_get_device_error", "gdn_status_string")
+
+_lib = None
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {gdn_status_string(status)}")
+
+
+def lib():
+    """The loaded libgdn handle (raises if the library has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libgdn.so not found at {LIB_PATH}; build it with "
+                               "`python -m linear_attention_token_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, U32, F, SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                   ctypes.c_uint32, ctypes.c_float, ctypes.c_size_t)
+        L.gdn_prefill_workspace_size.argtypes = [I32, I64, I32, I32, I32]
+        L.gdn_prefill_workspace_size.restype = SZ
+        L.gdn_prefill.argtypes = [P, P, P, P, P, P, P, P, P, I32, I32, I64, I32, I32, I32, I32,
+                                  ctypes.c_int, F, U32, P, SZ, P]
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, ctypes.c_int,
+                                      F, U32, P]
+        L.gdn_decode_step.restype = ctypes.c_int
+        L.gdn_get_device_error.argtypes = [P, P]
+        L.gdn_get_device_error.restype = ctypes.c_int
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def gdn_status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != GDN_OK:
+        raise GdnError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDN_F32
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; libgdn takes float32 or bfloat16")
+
+
+def _dev(t: Optional[torch.Tensor], name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libgdn has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def gdn_prefill_workspace_size(num_seqs: int, T_total: int, H_v: int, dk: int, dv: int) -> int:
+    return int(lib().gdn_prefill_workspace_size(num_seqs, T_total, H_v, dk, dv))
+
+
+def prefill_workspace(num_seqs: int, T_total: int, H_v: int, dk: int, dv: int,
+                      device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size gdn_prefill needs (torch allocates it)."""
+    n = gdn_prefill_workspace_size(num_seqs, T_total, H_v, dk, dv)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def gdn_prefill(q, k, v, g, beta, S0=None, cu_seqlens=None, *, out=None, S_final=None,
+                scale: float = 1.0, flags: int = 0, workspace=None, want_state: bool = True,
+                stream=None):
+    """Chunked prefill.  q,k [..., T, H_qk, dk]; v [..., T, H_v, dv]; g,beta [..., T, H_v].
+
+    Dense batch: q is [B, T, H_qk, dk] (or [T, H_qk, dk] for B = 1) and cu_seqlens is None.
+    Varlen: q is [T_total, H_qk, dk] and cu_seqlens an int32 CUDA tensor [num_seqs + 1].
+    Returns (out, S_final); S_final is None when want_state is False and none was given.
+    """
+    if cu_seqlens is not None:
+        T_total, H_qk, dk = q.shape[-3:]
+        B, T, N = 1, T_total, cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+    else:
+        if q.dim() == 4:
+            B, T, H_qk, dk = q.shape
+        else:
+            B, (T, H_qk, dk) = 1, q.shape
+        T_total, N = B * T, B
+    H_v, dv = v.shape[-2:]
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    if S_final is None and want_state:
+        S_final = torch.empty(N, H_v, dk, dv, dtype=torch.float32, device=v.device)
+    if workspace is None:
+        workspace = prefill_workspace(N, T_total, H_v, dk, dv, v.device)
+    st = lib().gdn_prefill(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+        _dev(S0, "S0"), _dev(out, "out"), _dev(S_final, "S_final"),
+        _dev(cu_seqlens, "cu_seqlens"), N if cu_seqlens is not None else 0, B, T, H_qk, H_v,
+        dk, dv, _dtype_code(q), float(scale), int(flags), _dev(workspace, "workspace"),
+        workspace.numel(), _stream(stream))
+    _check(st, "gdn_prefill")
+    return out, S_final
+
+
+def gdn_decode_step(q, k, v, g, beta, S_inout, *, out=None, scale: float = 1.0, flags: int = 0,
+                    stream=None):
+    """One decode step in place on S_inout [N, H_v, dk, dv]; q,k [N, H_qk, dk]; v [N, H_v, dv]."""
+    N, H_qk, dk = q.shape
+    H_v, dv = v.shape[-2:]
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    st = lib().gdn_decode_step(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+        _dev(S_inout, "S_inout"), _dev(out, "out"), N, H_qk, H_v, dk, dv, _dtype_code(q),
+        float(scale), int(flags), _stream(stream))
+    _check(st, "gdn_decode_step")
+    return out
+
+
+def gdn_get_device_error(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream; return (and clear) the device error status in the workspace."""
+    return int(lib().gdn_get_device_error(_dev(workspace, "workspace"), _stream(stream)))

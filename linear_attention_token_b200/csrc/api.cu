@@ -1,0 +1,156 @@
+// libgdn C ABI: argument checks, kernel choice, launch on the caller's stream.
+// The operation and the contract of every entry point are stated in include/gdn.h.
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+
+#define GDN_API extern "C" __attribute__((visibility("default")))
+
+namespace gdn {
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float *S, void *out, int N, int H_qk, int H_v,
+                          int dk, int dv, gdn_dtype dtype, float scale, int l2norm,
+                          cudaStream_t stream);
+cudaError_t launch_prefill_cc(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *S0, void *out, float *S_final,
+                              const int32_t *cu, int N, long long T, int H_qk, int H_v, int dk,
+                              int dv, gdn_dtype dtype, float scale, int l2norm,
+                              cudaStream_t stream);
+bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype);
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *S0, void *out, float *S_final,
+                              const int32_t *cu, int N, long long T_dense, long long T_total,
+                              int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
+                              cudaStream_t stream);
+}  // namespace gdn
+
+namespace {
+
+constexpr size_t kWorkspaceBytes = 256;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool head_dim_ok(int32_t d) { return d == 64 || d == 128; }
+
+// `has_tokens` false: there is no token to read or write, so the token buffers may be
+// NULL (an empty tensor has no storage).
+gdn_status common_checks(const void *q, const void *k, const void *v, const float *g,
+                         const float *beta, const void *out, int32_t H_qk, int32_t H_v,
+                         int32_t dk, int32_t dv, gdn_dtype dtype, uint32_t flags,
+                         bool has_tokens)
+{
+    if (has_tokens && (!q || !k || !v || !g || !beta || !out)) return GDN_ERR_INVALID_ARG;
+    if (H_qk <= 0 || H_v <= 0 || H_v % H_qk != 0) return GDN_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (flags & ~(GDN_FLAG_QK_L2NORM | GDN_FLAG_FORCE_CUDA_CORE)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned(g, 4) || !aligned(beta, 4)) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+}  // namespace
+
+GDN_API size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t T_total, int32_t H_v,
+                                          int32_t dk, int32_t dv)
+{
+    (void)num_seqs; (void)T_total; (void)H_v; (void)dk; (void)dv;
+    return kWorkspaceBytes;
+}
+
+GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *S0, void *out, float *S_final,
+                               const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int64_t T,
+                               int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                               gdn_dtype dtype, float scale, uint32_t flags, void *workspace,
+                               size_t workspace_bytes, cudaStream_t stream)
+{
+    if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    const bool has_tokens = (cu_seqlens ? (long long)T : (long long)B * T) > 0;
+    gdn_status st = common_checks(q, k, v, g, beta, out, H_qk, H_v, dk, dv, dtype, flags,
+                                  has_tokens);
+    if (st != GDN_OK) return st;
+    int N;
+    if (cu_seqlens) {
+        if (B != 1 || num_seqs < 0 || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+        N = num_seqs;
+    } else {
+        N = B;
+    }
+    if (N > 0 && H_v > 65535) return GDN_ERR_UNSUPPORTED;
+    if ((S0 && !aligned(S0, 16)) || (S_final && !aligned(S_final, 16))) return GDN_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kWorkspaceBytes || !aligned(workspace, 16))
+        return GDN_ERR_INVALID_ARG;
+    const long long T_total = cu_seqlens ? (long long)T : (long long)B * T;
+    if (N == 0 || T_total == 0) {
+        // nothing to compute; S_final = S0 (or zero) per sequence still has to be written
+        if (S_final && N > 0) {
+            const size_t bytes = (size_t)N * H_v * dk * dv * sizeof(float);
+            cudaError_t e = S0 ? (S0 == S_final ? cudaSuccess
+                                                : cudaMemcpyAsync(S_final, S0, bytes,
+                                                                  cudaMemcpyDeviceToDevice, stream))
+                               : cudaMemsetAsync(S_final, 0, bytes, stream);
+            if (e != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        return GDN_OK;
+    }
+    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    cudaError_t e;
+    if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
+        e = gdn::launch_prefill_tc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                   cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v, scale, l2,
+                                   reinterpret_cast<gdn::DeviceError *>(workspace), stream);
+    } else {
+        e = gdn::launch_prefill_cc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                   cu_seqlens ? 0 : (long long)T, H_qk, H_v, dk, dv, dtype, scale,
+                                   l2, stream);
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                                   const float *beta, float *S_inout, void *out, int32_t N,
+                                   int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv,
+                                   gdn_dtype dtype, float scale, uint32_t flags,
+                                   cudaStream_t stream)
+{
+    if (N < 0) return GDN_ERR_INVALID_ARG;
+    gdn_status st = common_checks(q, k, v, g, beta, out, H_qk, H_v, dk, dv, dtype, flags, N > 0);
+    if (st != GDN_OK) return st;
+    if ((N > 0 && !S_inout) || !aligned(S_inout, 16)) return GDN_ERR_INVALID_ARG;
+    if ((long long)N * H_v > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (N == 0) return GDN_OK;
+    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    cudaError_t e = gdn::launch_decode(q, k, v, g, beta, S_inout, out, N, H_qk, H_v, dk, dv,
+                                       dtype, scale, l2, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API gdn_status gdn_get_device_error(void *workspace, cudaStream_t stream)
+{
+    if (!workspace || !aligned(workspace, 16)) return GDN_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
+    gdn::DeviceError h{};
+    if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (h.status != 0) {
+        const gdn::DeviceError zero{};
+        if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    return static_cast<gdn_status>(h.status);
+}
+
+GDN_API const char *gdn_status_string(gdn_status status)
+{
+    switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: no kernel for this combination";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA call or launch failed";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a bounded device wait gave up";
+    }
+    return "unknown gdn_status";
+}

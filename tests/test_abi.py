@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/gdn.h declares, and rejects bad arguments before launching."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_token_b200 as gdn
+from linear_attention_token_b200 import build as gdn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    gdn_build.build()          # nvcc cross-compiles without a GPU
+    return gdn.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    assert declared_functions() == sorted(gdn.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    # nothing else with the gdn_ prefix leaks out of the library
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", gdn._binding.LIB_PATH],
+                         capture_output=True, text=True, check=True).stdout
+    exported = sorted(set(re.findall(r"\b(gdn_[a-z_]+)$", out, flags=re.M)))
+    assert exported == declared_functions()
+
+
+def test_status_strings(L):
+    for s in range(5):
+        assert gdn.gdn_status_string(s).startswith("GDN_")
+    assert "unknown" in gdn.gdn_status_string(99)
+
+
+def test_workspace_size(L):
+    assert gdn.gdn_prefill_workspace_size(8, 135000, 16, 128, 128) >= 256
+
+
+# fake, 256-byte aligned device-looking addresses: never dereferenced because every
+# call below fails validation on the host before any CUDA call
+A = 0x7f0000000000
+P = ctypes.c_void_p
+
+
+def _prefill(L, **over):
+    args = dict(q=A, k=A + 0x1000, v=A + 0x2000, g=A + 0x3000, beta=A + 0x4000, S0=None,
+                out=A + 0x5000, S_final=None, cu=None, num_seqs=0, B=1, T=64, H_qk=2, H_v=4,
+                dk=128, dv=128, dtype=1, scale=1.0, flags=0, ws=A + 0x6000, ws_bytes=256)
+    args.update(over)
+    a = args
+    return L.gdn_prefill(P(a["q"]), P(a["k"]), P(a["v"]), P(a["g"]), P(a["beta"]), P(a["S0"]),
+                         P(a["out"]), P(a["S_final"]), P(a["cu"]), a["num_seqs"], a["B"], a["T"],
+                         a["H_qk"], a["H_v"], a["dk"], a["dv"], a["dtype"], a["scale"],
+                         a["flags"], P(a["ws"]), a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(beta=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(out=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_v=3), gdn.GDN_ERR_INVALID_ARG),             # H_v % H_qk != 0
+    (dict(H_qk=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=96), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dv=32), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dtype=7), gdn.GDN_ERR_INVALID_ARG),
+    (dict(flags=64), gdn.GDN_ERR_INVALID_ARG),
+    (dict(v=A + 0x2008), gdn.GDN_ERR_INVALID_ARG),      # 8-byte aligned only
+    (dict(g=A + 0x3002), gdn.GDN_ERR_INVALID_ARG),
+    (dict(S0=A + 0x7004), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ws=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ws_bytes=16), gdn.GDN_ERR_INVALID_ARG),
+    (dict(cu=A + 0x8000, B=2, num_seqs=2), gdn.GDN_ERR_INVALID_ARG),   # varlen needs B == 1
+    (dict(cu=A + 0x8000, num_seqs=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(T=-5), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_prefill_rejects_on_host(L, over, expect):
+    assert _prefill(L, **over) == expect
+
+
+def _decode(L, **over):
+    a = dict(q=A, k=A + 0x1000, v=A + 0x2000, g=A + 0x3000, beta=A + 0x4000, S=A + 0x5000,
+             out=A + 0x6000, N=4, H_qk=2, H_v=4, dk=128, dv=128, dtype=1, scale=1.0, flags=0)
+    a.update(over)
+    return L.gdn_decode_step(P(a["q"]), P(a["k"]), P(a["v"]), P(a["g"]), P(a["beta"]), P(a["S"]),
+                             P(a["out"]), a["N"], a["H_qk"], a["H_v"], a["dk"], a["dv"],
+                             a["dtype"], a["scale"], a["flags"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(S=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(S=A + 0x5004), gdn.GDN_ERR_INVALID_ARG),
+    (dict(k=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_v=6, H_qk=4), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk=256), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dtype=3), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_decode_rejects_on_host(L, over, expect):
+    assert _decode(L, **over) == expect
+
+
+def test_decode_with_no_sequences_is_a_no_op(L):
+    assert _decode(L, N=0) == gdn.GDN_OK
+
+
+def test_get_device_error_rejects_null(L):
+    assert L.gdn_get_device_error(None, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 2, 128)
+    with pytest.raises(ValueError):
+        gdn.gdn_decode_step(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2),
+                            torch.zeros(4, 2, 128, 128))
