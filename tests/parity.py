@@ -17,7 +17,7 @@ TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 
 def err(x, ref) -> float:
     x = x.detach().double().cpu().numpy() if hasattr(x, "detach") else np.asarray(x, np.float64)
-    ref = np.asarray(ref, np.float64)
+    ref = ref.detach().double().cpu().numpy() if hasattr(ref, "detach") else np.asarray(ref, np.float64)
     if x.size == 0:
         return 0.0
     den = np.max(np.abs(ref))
