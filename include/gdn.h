@@ -108,6 +108,31 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const fl
                            int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype,
                            float scale, uint32_t flags, cudaStream_t stream);
 
+/* gdn_prefill for callers that cannot allocate device memory: the same computation
+ * and arguments, minus the workspace.  The paper has no counterpart; this is a
+ * deployment convenience.  Some callers cannot call cudaMalloc (for instance code
+ * running inside another runtime's memory pool, or in a context where allocation is
+ * forbidden), so they cannot provide the few bytes of device scratch gdn_prefill
+ * needs.  This entry point instead uses a scratch array of GDN_STATIC_SCRATCH_BYTES
+ * that the library keeps in every GPU that loads it, for as long as the library is
+ * loaded; it calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The first call on a device looks up that array's device address (with that
+ *     device current); make this first call before any stream capture.
+ *   - Every call on a device shares the one array: calls that may overlap on the GPU
+ *     (different streams, or different host threads) race on it.
+ *   - Each call clears the array's error word before it launches.  A device-side
+ *     timeout on this path is recorded there but not reported back (there is no
+ *     workspace to hand to gdn_get_device_error).
+ *   - Returns GDN_ERR_UNSUPPORTED if these sizes need more scratch than
+ *     GDN_STATIC_SCRATCH_BYTES (gdn_prefill_workspace_size(...) > the maximum). */
+#define GDN_STATIC_SCRATCH_BYTES 4096u
+gdn_status gdn_prefill_static_scratch(const void *q, const void *k, const void *v,
+                                      const float *g, const float *beta, const float *S0,
+                                      void *out, float *S_final, const int32_t *cu_seqlens,
+                                      int32_t num_seqs, int32_t B, int64_t T, int32_t H_qk,
+                                      int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype,
+                                      float scale, uint32_t flags, cudaStream_t stream);
+
 /* Synchronises `stream`, returns the first device-side error recorded in
  * `workspace` (GDN_OK if none) and clears it.  GDN_ERR_CUDA if the stream itself
  * reports an error. */

@@ -23,7 +23,7 @@ GDN_FLAG_FORCE_CUDA_CORE = 2
 
 # every symbol include/gdn.h declares
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
-            "gdn_get_device_error", "gdn_status_string")
+            "gdn_get_device_error", "gdn_status_string", "gdn_prefill_static_scratch")
 
 _lib = None
 
@@ -49,6 +49,9 @@ def lib():
         L.gdn_prefill.argtypes = [P, P, P, P, P, P, P, P, P, I32, I32, I64, I32, I32, I32, I32,
                                   ctypes.c_int, F, U32, P, SZ, P]
         L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_prefill_static_scratch.argtypes = [P, P, P, P, P, P, P, P, P, I32, I32, I64, I32,
+                                                 I32, I32, I32, ctypes.c_int, F, U32, P]
+        L.gdn_prefill_static_scratch.restype = ctypes.c_int
         L.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, ctypes.c_int,
                                       F, U32, P]
         L.gdn_decode_step.restype = ctypes.c_int
@@ -137,6 +140,33 @@ def gdn_prefill(q, k, v, g, beta, S0=None, cu_seqlens=None, *, out=None, S_final
         dk, dv, _dtype_code(q), float(scale), int(flags), _dev(workspace, "workspace"),
         workspace.numel(), _stream(stream))
     _check(st, "gdn_prefill")
+    return out, S_final
+
+
+def gdn_prefill_static_scratch(q, k, v, g, beta, S0=None, cu_seqlens=None, *, out, S_final,
+                               scale: float = 1.0, flags: int = 0, stream=None):
+    """gdn_prefill through the entry point that takes no workspace and allocates nothing.
+
+    For callers that cannot allocate device memory: the library supplies its own
+    static scratch.  ``out`` and ``S_final`` must be given (this call allocates nothing);
+    S_final may be None to skip the final state.  Shapes as for gdn_prefill.
+    """
+    if cu_seqlens is not None:
+        T_total, H_qk, dk = q.shape[-3:]
+        B, T, N = 1, T_total, cu_seqlens.numel() - 1
+    else:
+        if q.dim() == 4:
+            B, T, H_qk, dk = q.shape
+        else:
+            B, (T, H_qk, dk) = 1, q.shape
+        N = B
+    H_v, dv = v.shape[-2:]
+    st = lib().gdn_prefill_static_scratch(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+        _dev(S0, "S0"), _dev(out, "out"), _dev(S_final, "S_final"),
+        _dev(cu_seqlens, "cu_seqlens"), N if cu_seqlens is not None else 0, B, T, H_qk, H_v,
+        dk, dv, _dtype_code(q), float(scale), int(flags), _stream(stream))
+    _check(st, "gdn_prefill_static_scratch")
     return out, S_final
 
 

@@ -23,6 +23,8 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               const int32_t *cu, int N, long long T_dense, long long T_total,
                               int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
                               cudaStream_t stream);
+size_t static_scratch_capacity();
+cudaError_t static_scratch_ptr(void **out);
 }  // namespace gdn
 
 namespace {
@@ -125,6 +127,64 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v, 
     const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     cudaError_t e = gdn::launch_decode(q, k, v, g, beta, S_inout, out, N, H_qk, H_v, dk, dv,
                                        dtype, scale, l2, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// gdn_prefill without a caller-provided workspace (see include/gdn.h): the kernels
+// receive the library's static scratch instead.
+GDN_API gdn_status gdn_prefill_static_scratch(const void *q, const void *k, const void *v,
+                                              const float *g, const float *beta,
+                                              const float *S0, void *out, float *S_final,
+                                              const int32_t *cu_seqlens, int32_t num_seqs,
+                                              int32_t B, int64_t T, int32_t H_qk, int32_t H_v,
+                                              int32_t dk, int32_t dv, gdn_dtype dtype,
+                                              float scale, uint32_t flags, cudaStream_t stream)
+{
+    if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    const bool has_tokens = (cu_seqlens ? (long long)T : (long long)B * T) > 0;
+    gdn_status st = common_checks(q, k, v, g, beta, out, H_qk, H_v, dk, dv, dtype, flags,
+                                  has_tokens);
+    if (st != GDN_OK) return st;
+    int N;
+    if (cu_seqlens) {
+        if (B != 1 || num_seqs < 0 || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+        N = num_seqs;
+    } else {
+        N = B;
+    }
+    if (N > 0 && H_v > 65535) return GDN_ERR_UNSUPPORTED;
+    if ((S0 && !aligned(S0, 16)) || (S_final && !aligned(S_final, 16))) return GDN_ERR_INVALID_ARG;
+    const long long T_total = cu_seqlens ? (long long)T : (long long)B * T;
+    // the sizes must fit the library-held scratch
+    if (gdn_prefill_workspace_size(N, T_total, H_v, dk, dv) > gdn::static_scratch_capacity())
+        return GDN_ERR_UNSUPPORTED;
+    if (N == 0 || T_total == 0) {
+        if (S_final && N > 0) {
+            const size_t bytes = (size_t)N * H_v * dk * dv * sizeof(float);
+            cudaError_t e = S0 ? (S0 == S_final ? cudaSuccess
+                                                : cudaMemcpyAsync(S_final, S0, bytes,
+                                                                  cudaMemcpyDeviceToDevice, stream))
+                               : cudaMemsetAsync(S_final, 0, bytes, stream);
+            if (e != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        return GDN_OK;
+    }
+    void *scratch = nullptr;
+    if (gdn::static_scratch_ptr(&scratch) != cudaSuccess) return GDN_ERR_CUDA;
+    // the error word must start at zero; earlier calls may have left one behind
+    if (cudaMemsetAsync(scratch, 0, sizeof(gdn::DeviceError), stream) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    cudaError_t e;
+    if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
+        e = gdn::launch_prefill_tc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                   cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v, scale, l2,
+                                   reinterpret_cast<gdn::DeviceError *>(scratch), stream);
+    } else {
+        e = gdn::launch_prefill_cc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                   cu_seqlens ? 0 : (long long)T, H_qk, H_v, dk, dv, dtype, scale,
+                                   l2, stream);
+    }
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
