@@ -18,6 +18,7 @@
 // independently, so tiles need no communication.  The state tile lives in
 // shared memory for the whole sequence.
 #include "common.cuh"
+#include "tri_inverse.cuh"
 
 namespace gdn {
 
@@ -146,17 +147,8 @@ prefill_cc_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
         }
         __syncthreads();
 
-        // 4. T = (I + A)^-1: column j, four threads split the sum over m (m = s mod 4)
-        {
-            const int j = tid >> 2, s = tid & 3;
-            for (int i = 1; i < CC_C; ++i) {
-                float part = 0.f;
-                for (int m = s; m < i; m += 4) part += sm.A[i][m] * sm.T[m][j];
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                if (j < i && s == (i & 3)) sm.T[i][j] = -part;
-            }
-        }
+        // 4. T = (I + A)^-1 (blocked, fp32)
+        invert_unit_lower_64<CC_TP>(&sm.A[0][0], &sm.T[0][0], tid);
         __syncthreads();
 
         // 5. K S and Q S (64x32 each); R = diag(beta) V - diag(beta gamma) K S

@@ -41,6 +41,24 @@
 namespace gdn {
 using namespace sm100;
 
+// Profiling aid, compiled in only with -DGDN_PHASE_TIMERS: CTA (0, 0) records
+// clock64() at each phase boundary of its first 64 chunks.
+#ifdef GDN_PHASE_TIMERS
+__device__ unsigned long long g_phase_clock[64][32];
+#define PHASE_MARK(k) gdn_phase_mark(tid, c, k)
+__device__ __forceinline__ void gdn_phase_mark(int tid, int c, int k) {
+    if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && c < 64) g_phase_clock[c][k] = clock64();
+}
+#define GDN_TRI_MARK(k) gdn_phase_mark(tid, dbg_chunk, k)
+#else
+#define PHASE_MARK(k) do { } while (0)
+#define GDN_TRI_MARK(k) do { } while (0)
+#endif
+
+}  // namespace gdn
+#include "tri_inverse.cuh"
+namespace gdn {
+
 namespace {
 
 constexpr int TC_C = 64;
@@ -65,7 +83,8 @@ constexpr uint32_t SM_AF = 172032;     // fp32 A, 64 x 65
 constexpr uint32_t SM_TF = 188672;     // fp32 T, 64 x 65
 constexpr uint32_t SM_VEC = 205312;    // g, beta, G, gamma, decay-to-end: 5 x 64 fp32
 constexpr uint32_t SM_BAR = 206592;    // 4 mbarriers + TMEM base address
-constexpr uint32_t SM_END = SM_BAR + 64;
+constexpr uint32_t SM_OST = 206848;    // 16 KB output staging, rows i x 128 bf16 (v contiguous)
+constexpr uint32_t SM_END = SM_OST + 16384;
 constexpr uint32_t SMEM_BYTES = SM_END + 1024;
 constexpr int TP = 65;                 // fp32 matrix pitch
 
@@ -234,13 +253,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int L = (int)min((long long)TC_C, t_end - t0);
         const int vb = c & 1;
         unsigned char *Vt = sm + SM_V + vb * 16384;
+        PHASE_MARK(0);
         if (c + 1 < nchunks) issue_v(c + 1);          // its buffer was released by chunk c-1
+        PHASE_MARK(16);
 
         // ---- A: inputs of the chunk
-        if (!cta_wait(bar_kq, pend.kq_done)) { fail_where = 1; break; }
+        {
+            const bool ok = mbar_wait(bar_kq, (uint32_t)(pend.kq_done & 1), budget) &&
+                            mbar_wait(bar_v + vb, (uint32_t)(pend.v_done[vb] & 1), budget);
+            if (__syncthreads_or(!ok)) { fail_where = 1; break; }
+        }
         ++pend.kq_done;
-        if (!cta_wait(bar_v + vb, pend.v_done[vb])) { fail_where = 2; break; }
+        PHASE_MARK(17);
         ++pend.v_done[vb];
+        PHASE_MARK(1);
         if (L < TC_C) {            // zero rows L..63 of K, Q (both halves) and V
             const int zr = TC_C - L;
             for (int e = tid; e < 6 * zr * 8; e += TC_THREADS) {
@@ -292,15 +318,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             dte[2 * lane] = expf(Gend - G0); dte[2 * lane + 1] = expf(Gend - G1);
         }
         handoff();
+        PHASE_MARK(2);
 
-        // ---- B: P1 = [K;Q] K^T on the tensor core; meanwhile K~ = diag(decay-to-end) K
+        // ---- B: P1 = [K;Q] K^T and S1' (Q S)^T = S^T Q^T on the tensor core;
+        //         meanwhile K~ = diag(decay-to-end) K on the CUDA cores
         if (tid == 0) {
             const uint32_t id = idesc_bf16(128, 64, false, false);
-            const uint32_t kq = smem_u32(sm + SM_KQ);
+            const uint32_t kq = smem_u32(sm + SM_KQ), st = smem_u32(sm + SM_ST);
+            const uint32_t qb = kq + 8192;
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const uint32_t a = kq + (s / 4) * 16384 + (s % 4) * 32;
                 umma_bf16(tmem + TM_KQ, sdesc_kmajor(a), sdesc_kmajor(a), id, s > 0);
+            }
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t o = (s / 4) * 16384 + (s % 4) * 32;
+                umma_bf16(tmem + TM_O, sdesc_kmajor(st + o), sdesc_kmajor(qb + o), id, s > 0);
             }
         }
         commit_mma();
@@ -316,24 +350,40 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         fence_proxy_async();
         if (!mma_sync_wait()) { fail_where = 3; break; }
+        PHASE_MARK(3);
 
         // ---- C: A (fp32) from K K^T, P (bf16) from Q K^T; T := I
         if (wg == 0) {
             float x[64];
             ld64(tmem + lane_off + TM_KQ, x);
-            if (quad < 2) {
-                const int i = row;
-                const float Gi = Gs[i], bi = bs[i];
+            PHASE_MARK(18);
+            // loads of G are issued ahead of the stores (they may not be reordered
+            // across stores to shared memory by the compiler)
+            const bool is_a = quad < 2;
+            const int i = is_a ? row : row - 64;
+            const float Gi = Gs[i], wi = is_a ? bs[i] : 1.f;
 #pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    Af[i * TP + j] = (j < i) ? bi * expf(Gi - Gs[j]) * x[j] : 0.f;
+            for (int j0 = 0; j0 < 64; j0 += 16) {
+                float gj[16];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(Gs + j0 + 4 * u);
+                    gj[4 * u] = t4.x; gj[4 * u + 1] = t4.y; gj[4 * u + 2] = t4.z; gj[4 * u + 3] = t4.w;
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {   // branch-free: clamped exponent times a 0/1 mask
+                    const int j = j0 + u;
+                    const float keep = (is_a ? (j < i) : (j <= i)) ? 1.f : 0.f;
+                    x[j] = (wi * keep) * __expf(fminf(Gi - gj[u], 0.f)) * x[j];
+                }
+            }
+            if (is_a) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) Af[i * TP + j] = x[j];
             } else {
-                const int i = row - 64;
-                const float Gi = Gs[i];
-#pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] = (j <= i) ? expf(Gi - Gs[j]) * x[j] : 0.f;
                 store_row_bf16(sm + SM_P, i, x);
             }
+            PHASE_MARK(19);
         } else {
             for (int e = tid - 128; e < 64 * 64; e += 128) {
                 const int i = e >> 6, j = e & 63;
@@ -341,35 +391,37 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
         __syncthreads();
+        PHASE_MARK(4);
 
-        // ---- D: T = (I + A)^-1; column j, the four threads of a column split m mod 4
-        {
-            const int j = tid >> 2, s = tid & 3;
-#pragma unroll 1
-            for (int i = 1; i < TC_C; ++i) {
-                float part = 0.f;
-                for (int m = s; m < i; m += 4) part += Af[i * TP + m] * Tf[m * TP + j];
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                if (j < i && s == (i & 3)) Tf[i * TP + j] = -part;
-            }
-        }
+        // ---- D: T = (I + A)^-1 (blocked; merges on the warp-level tensor cores in tf32)
+        invert_unit_lower_64_tf32<TP>(Af, Tf, tid, c);
         __syncthreads();
-        for (int e = tid; e < 1024; e += TC_THREADS) {      // T' and T'' rows, 16 B at a time
-            const int which = e >> 9, i = (e >> 3) & 63, cc = e & 7;
-            float x[8];
+        PHASE_MARK(5);
+        {   // T' = T diag(beta gamma), T'' = T diag(beta): thread = (matrix, row i, 32 columns)
+            const int which = tid >> 7, i = (tid >> 1) & 63, j0 = (tid & 1) * 32;
+            float x[32];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const int j = 8 * cc + jj;
-                const float t = (j <= i) ? Tf[i * TP + j] : 0.f;
-                x[jj] = t * bs[j] * (which == 0 ? gam[j] : 1.f);
+            for (int u = 0; u < 32; ++u) x[u] = Tf[i * TP + j0 + u];
+#pragma unroll
+            for (int u = 0; u < 32; u += 4) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(bs + j0 + u);
+                const float4 g4 = which == 0 ? *reinterpret_cast<const float4 *>(gam + j0 + u)
+                                             : make_float4(1.f, 1.f, 1.f, 1.f);
+                const float bb[4] = {b4.x * g4.x, b4.y * g4.y, b4.z * g4.z, b4.w * g4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[u + e] = (j0 + u + e <= i) ? x[u + e] * bb[e] : 0.f;
             }
-            uint4 w;
-            w.x = pack_bf16(x[0], x[1]); w.y = pack_bf16(x[2], x[3]);
-            w.z = pack_bf16(x[4], x[5]); w.w = pack_bf16(x[6], x[7]);
-            *reinterpret_cast<uint4 *>(sm + (which ? SM_TPP : SM_TP) + sw128(i, cc)) = w;
+            unsigned char *dst = sm + (which ? SM_TPP : SM_TP);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint4 w;
+                w.x = pack_bf16(x[8 * cc + 0], x[8 * cc + 1]); w.y = pack_bf16(x[8 * cc + 2], x[8 * cc + 3]);
+                w.z = pack_bf16(x[8 * cc + 4], x[8 * cc + 5]); w.w = pack_bf16(x[8 * cc + 6], x[8 * cc + 7]);
+                *reinterpret_cast<uint4 *>(dst + sw128(i, j0 / 8 + cc)) = w;
+            }
         }
         handoff();
+        PHASE_MARK(6);
 
         // ---- E: P2 W^T = K^T T'^T ; P3 U~^T = V^T T''^T
         if (tid == 0) {
@@ -385,6 +437,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         commit_mma();
         if (!mma_sync_wait()) { fail_where = 4; break; }
+        PHASE_MARK(7);
+        if (c + 1 < nchunks) issue_kq(c + 1);        // K and Q of this chunk are no longer read
 
         // ---- F: W^T (lane d) -> bf16 rows d of the MN-major B operand
         if (wg == 0) {
@@ -393,23 +447,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             store_row_bf16(sm + SM_WT, row, x);
         }
         handoff();
+        PHASE_MARK(8);
 
-        // ---- G: S1 U^T = U~^T - S^T W^T ; S1' (Q S)^T = S^T Q^T
+        // ---- G: S1 U^T = U~^T - S^T W^T
         if (tid == 0) {
             const uint32_t st = smem_u32(sm + SM_ST), wt = smem_u32(sm + SM_WT);
-            const uint32_t qb = smem_u32(sm + SM_KQ + 8192);
             const uint32_t id_neg = idesc_bf16(128, 64, false, true, true);
-            const uint32_t id_q = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const uint64_t a = sdesc_kmajor(st + (s / 4) * 16384 + (s % 4) * 32);
                 umma_bf16(tmem + TM_U, a, sdesc_mnmajor(wt + s * 2048, 16384), id_neg, 1);
-                umma_bf16(tmem + TM_O, a, sdesc_kmajor(qb + (s / 4) * 16384 + (s % 4) * 32), id_q, s > 0);
             }
         }
         commit_mma();
         if (!mma_sync_wait()) { fail_where = 5; break; }
-        if (c + 1 < nchunks) issue_kq(c + 1);        // K and Q of this chunk are no longer read
+        PHASE_MARK(9);
 
         // ---- H: U^T -> bf16 A operand (WG0); state scaled by gamma_end in TMEM (WG1)
         if (wg == 0) {
@@ -430,6 +482,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tmem_wait_st();
         }
         handoff();
+        PHASE_MARK(10);
 
         // ---- I: S2 S^T += U^T K~ ; S2' (P U)^T = U^T P^T
         if (tid == 0) {
@@ -445,6 +498,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         commit_mma();
         if (!mma_sync_wait()) { fail_where = 6; break; }
+        PHASE_MARK(11);
 
         // ---- J: new state -> bf16 S^T (or S_final); outputs
         const bool last = (c + 1 == nchunks);
@@ -473,25 +527,40 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
             }
+            PHASE_MARK(21);
         } else {
+            // o_i = scale (gamma_i (Q S)_i + (P U)_i): column v of the chunk's outputs,
+            // staged row-major in shared memory, then written as 16-byte row pieces
             const int v = row;
+            __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(sm + SM_OST);
 #pragma unroll 1
             for (int i0 = 0; i0 < TC_C; i0 += 32) {
                 uint32_t o[32], pu[32];
                 tmem_ld32(tmem + lane_off + TM_O + i0, o);
                 tmem_ld32(tmem + lane_off + TM_PU + i0, pu);
                 tmem_wait_ld();
+                float gg[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int i = i0 + j;
-                    if (i < L) {
-                        const float val = scale * (gam[i] * __uint_as_float(o[j]) + __uint_as_float(pu[j]));
-                        out[((size_t)(t0 + i) * H_v + h) * TC_D + v] = __float2bfloat16_rn(val);
-                    }
+                for (int u = 0; u < 32; u += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(gam + i0 + u);
+                    gg[u] = g4.x; gg[u + 1] = g4.y; gg[u + 2] = g4.z; gg[u + 3] = g4.w;
                 }
+                __nv_bfloat16 ov[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    ov[j] = __float2bfloat16_rn(scale * (gg[j] * __uint_as_float(o[j]) + __uint_as_float(pu[j])));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ost[(i0 + j) * TC_D + v] = ov[j];
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");       // the four output warps
+            for (int e = tid - 128; e < L * 16; e += 128) {
+                const int i = e >> 4, cc = e & 15;
+                const uint4 val = *reinterpret_cast<const uint4 *>(ost + i * TC_D + cc * 8);
+                *reinterpret_cast<uint4 *>(out + ((size_t)(t0 + i) * H_v + h) * TC_D + cc * 8) = val;
             }
         }
         handoff();
+        PHASE_MARK(12);
     }
 
     if (fail_where) {
@@ -585,6 +654,13 @@ cudaError_t static_scratch_ptr(void **out)
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
 }
+
+#ifdef GDN_PHASE_TIMERS
+extern "C" __attribute__((visibility("default"))) int gdn_debug_phase_clock(void *host)
+{
+    return (int)cudaMemcpyFromSymbol(host, g_phase_clock, sizeof(g_phase_clock));
+}
+#endif
 
 bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype)
 {
