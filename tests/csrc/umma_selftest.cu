@@ -30,7 +30,9 @@ umma_kernel(const __nv_bfloat16 *A, const __nv_bfloat16 *B, float *D, int varian
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const bool a_mn = variant & 1, b_mn = variant & 2, neg = variant & 4;
-    const int M = 128, N = (variant & 8) ? 128 : 64, K = (variant & 16) ? 128 : 64;
+    const int M = (variant & 32) ? 64 : 128;
+    const int N = (variant & 64) ? 32 : ((variant & 8) ? 128 : 64);
+    const int K = (variant & 16) ? 128 : 64;
     unsigned char *As = base;                  // up to 32 KB
     unsigned char *Bs = base + 32768;          // up to 32 KB
     __shared__ uint64_t bar;
@@ -89,13 +91,17 @@ umma_kernel(const __nv_bfloat16 *A, const __nv_bfloat16 *B, float *D, int varian
     const bool ok = mbar_wait(&bar, 0, 1u << 20);
     if (!ok && tid == 0) atomicExch(status, 4);
     tc_fence_after();
-    // warp w reads lanes 32w..32w+31 = rows m
-    const int m = warp * 32 + (tid & 31);
+    // warp w reads lanes 32w..32w+31.  M = 128: lane = row.  M = 64: rows 16w..16w+15
+    // sit in lanes 32w..32w+15 (the other 16 lanes of each quadrant are not written).
+    const int l = tid & 31;
+    const int m = (M == 128) ? warp * 32 + l : warp * 16 + l;
+    const bool has_row = (M == 128) || l < 16;
     for (int c0 = 0; c0 < N; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tm + ((uint32_t)(warp * 32) << 16) + c0, r);
         tmem_wait_ld();
-        for (int j = 0; j < 32; ++j) D[m * N + c0 + j] = __uint_as_float(r[j]);
+        if (has_row)
+            for (int j = 0; j < 32; ++j) D[m * N + c0 + j] = __uint_as_float(r[j]);
     }
     tc_fence_before();
     __syncthreads();
@@ -126,7 +132,55 @@ __global__ void tma_kernel(const __grid_constant__ CUtensorMap map, int h, int t
     }
 }
 
+// Four CTAs of one cluster: each fills 16 KB with a pattern, copies it into the next
+// CTA's shared memory with a bulk copy that completes on that CTA's mbarrier, pings the
+// next CTA's second mbarrier with a remote arrive, and checks what it received.
+__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(128, 1)
+cluster_kernel(int *out)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t recv_bar, ping_bar;
+    uint32_t *sendbuf = reinterpret_cast<uint32_t *>(base);
+    uint32_t *recvbuf = reinterpret_cast<uint32_t *>(base + 16384);
+    const int tid = threadIdx.x;
+    const uint32_t rank = cluster_rank();
+    const uint32_t next = (rank + 1) & 3, prev = (rank + 3) & 3;
+    for (int i = tid; i < 4096; i += blockDim.x) { sendbuf[i] = rank * 100000u + i; recvbuf[i] = 0xdeadbeefu; }
+    if (tid == 0) {
+        mbar_init(&recv_bar, 1);
+        mbar_init(&ping_bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&recv_bar, 16384);          // expect one 16 KB copy
+    }
+    fence_proxy_async();
+    cluster_sync();                                        // barriers and buffers ready everywhere
+    if (tid == 0) {
+        bulk_copy_to_cluster(map_to_rank(recvbuf, next), sendbuf, 16384, map_to_rank(&recv_bar, next));
+        mbar_arrive_remote(map_to_rank(&ping_bar, next));
+    }
+    const bool ok1 = mbar_wait_cluster(&recv_bar, 0, 1u << 20);
+    const bool ok2 = mbar_wait_cluster(&ping_bar, 0, 1u << 20);
+    int bad = (!ok1 || !ok2) ? 1 : 0;
+    if (ok1)
+        for (int i = tid; i < 4096; i += blockDim.x)
+            if (recvbuf[i] != prev * 100000u + i) bad = 2;
+    bad = __syncthreads_or(bad);
+    if (tid == 0) out[blockIdx.x] = bad ? (ok1 && ok2 ? 2 : 1) : 0;
+    cluster_sync();                                        // nobody leaves while others may copy
+}
+
 }  // namespace
+
+extern "C" __attribute__((visibility("default")))
+int selftest_cluster(int *out)
+{
+    const int smem = 32768 + 1024;
+    cudaFuncSetAttribute(cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cluster_kernel<<<8, 128, smem>>>(out);
+    return (int)cudaDeviceSynchronize();
+}
 
 extern "C" __attribute__((visibility("default")))
 int selftest_umma(const void *A, const void *B, float *D, int variant, int *status)

@@ -25,5 +25,6 @@ def load():
     L = ctypes.CDLL(build())
     P = ctypes.c_void_p
     L.selftest_umma.argtypes = [P, P, P, ctypes.c_int, P]
+    L.selftest_cluster.argtypes = [P]
     L.selftest_tma.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
     return L

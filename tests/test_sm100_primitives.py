@@ -26,14 +26,19 @@ def L():
     2 | 8,             # U^T K~    : A K-major, B MN-major, N=128, K=64
     0 | 16 | 8,        # A K-major, B K-major, N=128, K=128
     1 | 2 | 16 | 8,    # both MN-major, N=128, K=128
+    32 | 64 | 16,      # M=64, N=32, K=128: W S (A K-major, B K-major with 32 rows)
+    32 | 64,           # M=64, N=32, K=64:  P U
+    32 | 2 | 8,        # M=64, N=128, K=64: T' K with B MN-major
+    64 | 1,            # M=128, N=32, K=64: K~^T U with A MN-major
 ])
 def test_umma_placements(L, variant):
     torch.manual_seed(variant)
-    N = 128 if variant & 8 else 64
+    M = 64 if variant & 32 else 128
+    N = 32 if variant & 64 else (128 if variant & 8 else 64)
     K = 128 if variant & 16 else 64
-    A = torch.randn(128, K, device="cuda").to(torch.bfloat16)
+    A = torch.randn(M, K, device="cuda").to(torch.bfloat16)
     B = torch.randn(N, K, device="cuda").to(torch.bfloat16)
-    D = torch.zeros(128, N, device="cuda", dtype=torch.float32)
+    D = torch.zeros(M, N, device="cuda", dtype=torch.float32)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = L.selftest_umma(ctypes.c_void_p(A.data_ptr()), ctypes.c_void_p(B.data_ptr()),
                          ctypes.c_void_p(D.data_ptr()), variant, ctypes.c_void_p(st.data_ptr()))
@@ -56,3 +61,10 @@ def test_tma_tile_load(L, t0):
     rows = min(64, T - t0)
     assert torch.equal(out[:rows], x[t0:t0 + rows, h])
     assert torch.all(out[rows:] == 0)          # past the tensor end: zero fill
+
+
+def test_cluster_dsmem_copy_and_remote_arrive(L):
+    out = torch.full((8,), -1, dtype=torch.int32, device="cuda")
+    rc = L.selftest_cluster(ctypes.c_void_p(out.data_ptr()))
+    assert rc == 0
+    assert out.tolist() == [0] * 8
