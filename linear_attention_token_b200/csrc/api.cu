@@ -18,6 +18,11 @@ cudaError_t launch_prefill_cc(const void *q, const void *k, const void *v, const
                               int dv, gdn_dtype dtype, float scale, int l2norm,
                               cudaStream_t stream);
 bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype);
+cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *v, const float *g,
+                                      const float *beta, const float *S0, void *out, float *S_final,
+                                      const int32_t *cu, int N, long long T_dense, long long T_total,
+                                      int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
+                                      cudaStream_t stream);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *S0, void *out, float *S_final,
                               const int32_t *cu, int N, long long T_dense, long long T_total,
@@ -101,9 +106,10 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, cons
     const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     cudaError_t e;
     if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
-        e = gdn::launch_prefill_tc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
-                                   cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v, scale, l2,
-                                   reinterpret_cast<gdn::DeviceError *>(workspace), stream);
+        e = gdn::launch_prefill_tc_cluster(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                           cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v,
+                                           scale, l2,
+                                           reinterpret_cast<gdn::DeviceError *>(workspace), stream);
     } else {
         e = gdn::launch_prefill_cc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
                                    cu_seqlens ? 0 : (long long)T, H_qk, H_v, dk, dv, dtype, scale,
@@ -177,9 +183,10 @@ GDN_API gdn_status gdn_prefill_static_scratch(const void *q, const void *k, cons
     const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     cudaError_t e;
     if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
-        e = gdn::launch_prefill_tc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
-                                   cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v, scale, l2,
-                                   reinterpret_cast<gdn::DeviceError *>(scratch), stream);
+        e = gdn::launch_prefill_tc_cluster(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                           cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v,
+                                           scale, l2,
+                                           reinterpret_cast<gdn::DeviceError *>(scratch), stream);
     } else {
         e = gdn::launch_prefill_cc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
                                    cu_seqlens ? 0 : (long long)T, H_qk, H_v, dk, dv, dtype, scale,

@@ -1,0 +1,867 @@
+// Chunked prefill of the gated delta rule, dk = dv = 128, bf16 I/O, on a cluster of
+// four sm_100a CTAs per (sequence, value head).
+//
+// Rule: "論文解説: Qwen3.8-Next の設計" (ta-paperlens), section "GDNの中身", Eq. (1)
+//   S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,  o_t = S_t^T q_t.
+// Chunk algebra (C = 64; G_i = in-chunk cumsum of g, gamma_i = exp G_i, S the state
+// entering the chunk; an exact re-association of the rule):
+//   A_ij = beta_i exp(G_i - G_j) k_i.k_j (j < i),  T = (I + A)^-1
+//   W = T diag(beta gamma) K,  U~ = T diag(beta) V,  U = U~ - W S
+//   O = diag(gamma) Q S + P U,  P_ij = exp(G_i - G_j) q_i.k_j (j <= i)
+//   S <- gamma_end S + K~^T U,  K~_j = exp(G_end - G_j) k_j
+//
+// Work split.  The value columns of S evolve independently, so CTA r of the cluster
+// owns columns [32r, 32r + 32) of S, U and O for the whole sequence and runs the
+// sequential state chain for them:
+//     WS = W S_r -> U_r = U~_r - WS -> S_r <- gamma_end S_r + K~^T U_r -> next chunk,
+// with Q S_r and P U_r for the outputs off that chain.  The per-chunk quantities that
+// do not depend on the value columns (P, the inverse T, W, U~) are computed once per
+// chunk, by CTA (chunk mod 4), and copied into all four CTAs' shared memory with
+// bulk DSMEM copies that complete on the receivers' mbarriers.  Each CTA therefore
+// prepares every fourth chunk, several chunks ahead of the state chain.
+//
+// Roles inside a CTA (320 threads):
+//   warps 0-3  chain group:  K~ build, U epilogue, state epilogue, output epilogue
+//   warps 4-7  prep group:   inputs fix-up, A/P epilogue, triangular inverse, T'/T'',
+//                            W/U~ epilogue into the send staging
+//   warp 8     chain issuer: TMA for Q, MMAs QS, WS, S2 (K~^T U), PU, ring bookkeeping
+//   warp 9     prep issuer:  TMA for the prepared chunk, MMAs P1 ([K;Q]K^T), W, U~, sends
+// Accumulators live in TMEM; the state slice S_r (128 x 32 fp32) stays in TMEM for the
+// whole sequence.  Every wait is bounded; a CTA whose wait runs out records
+// GDN_ERR_TIMEOUT, raises its abort flag so its other roles stop, drains its own
+// copies and MMAs, and leaves through the final cluster barrier.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <stdlib.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "tri_inverse.cuh"
+
+namespace gdn {
+using namespace sm100;
+
+namespace {
+
+constexpr int K4_C = 64;                 // chunk
+constexpr int K4_D = 128;                // dk = dv
+constexpr int K4_SL = 32;                // value columns per CTA
+constexpr int K4_THREADS = 320;
+constexpr uint32_t K4_DEFAULT_BUDGET = 1u << 22;
+constexpr uint32_t K4_RING_BYTES = 28672;    // W 16 KB + P 8 KB + U~ slice 4 KB
+
+// TMEM columns (512 allocated)
+constexpr uint32_t T4_S = 0;       // 32: S_r (lane = key dim d, col = value v)
+constexpr uint32_t T4_WS = 32;     // 32: W S_r      (M = 64 layout)
+constexpr uint32_t T4_QS = 64;     // 2 x 32: Q S_r  (M = 64 layout, double-buffered)
+constexpr uint32_t T4_PU = 128;    // 2 x 32: P U_r  (M = 64 layout, double-buffered)
+constexpr uint32_t T4_KQ = 192;    // 64: [K;Q] K^T (M = 128)
+constexpr uint32_t T4_W = 256;     // 128: T' K     (M = 64 layout)
+constexpr uint32_t T4_U = 384;     // 128: T'' V    (M = 64 layout)
+
+// shared memory (offsets from a 1024-aligned base)
+constexpr uint32_t S4_CQ = 0;          // 16 KB Q of the chain's chunk [cg0 | cg1]
+constexpr uint32_t S4_CK = 16384;      // 16 KB K of the chain's chunk
+constexpr uint32_t S4_CKT = 32768;     // 16 KB K~
+constexpr uint32_t S4_ST = 49152;      // 8 KB S_r^T bf16, rows v (K-major B), [cg0 | cg1] 4 KB each
+constexpr uint32_t S4_UT = 57344;      // 4 KB U_r^T bf16, rows v (K-major B)
+constexpr uint32_t S4_RING = 61440;    // 2 slots x 28 KB: W (16 KB) | P (8 KB) | U~_r (4 KB)
+constexpr uint32_t S4_PKQ = 118784;    // 32 KB [K cg0 | Q cg0 | K cg1 | Q cg1] of the prepared chunk
+constexpr uint32_t S4_PV = 151552;     // 16 KB V of the prepared chunk
+constexpr uint32_t S4_TP = 167936;     // 8 KB T' = T diag(beta gamma)
+constexpr uint32_t S4_TPP = 176128;    // 8 KB T'' = T diag(beta)
+constexpr uint32_t S4_PSTG = 184320;   // 8 KB P staging (send source)
+constexpr uint32_t S4_AF = 192512;     // fp32 A 64 x 65 (overlaid later by the W staging)
+constexpr uint32_t S4_TF = 209152;     // fp32 T 64 x 65 (overlaid later by the U~ staging)
+constexpr uint32_t S4_WSTG = 192512;   // 16 KB W staging
+constexpr uint32_t S4_USTG = 208896;   // 16 KB U~ staging, 4 slices x [64 rows x 32 v]
+constexpr uint32_t S4_CVEC = 225792;   // chain vectors, 2 buffers x {g, beta, G, gamma, dte} x 64
+constexpr uint32_t S4_PVEC = 228352;   // prep vectors {g, beta, G, gamma} x 64
+constexpr uint32_t S4_BAR = 229376;    // mbarriers
+constexpr uint32_t S4_MISC = S4_BAR + 32 * 8;   // tmem base, abort flag
+constexpr uint32_t S4_END = S4_MISC + 16;
+constexpr uint32_t K4_SMEM = S4_END + 1024;
+constexpr int TP4 = 65;
+
+enum Bar {
+    B_CQ = 0, B_CK, B_FULL0, B_FULL1, B_QS, B_WS, B_S2, B_KT, B_U, B_ST, B_OFREE0, B_OFREE1,
+    B_PKQ, B_PV, B_P1, B_TT, B_WU, B_STG, B_EMPTY, B_SENT, B_PIN, B_CQN, B_COUNT
+};
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ float2 unpack2(uint32_t x) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x));
+}
+template <int ID>
+__device__ __forceinline__ void group_sync() {
+    asm volatile("bar.sync %0, 128;" ::"n"(ID) : "memory");
+}
+// all 128 threads of named barrier ID must call; returns the AND of `v`
+template <int ID>
+__device__ __forceinline__ bool group_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"(v ? 1u : 0u), "n"(ID) : "memory");
+    return r != 0;
+}
+// element (row r, column c) of a 128-byte-swizzled tile whose rows hold 64 bf16
+__device__ __forceinline__ void store_bf16_at(unsigned char *tile, int r, int c, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(tile + sw128(r, c >> 3) + (c & 7) * 2) = __float2bfloat16_rn(x);
+}
+// wait for the last of `issued` phases of `bar` (phases complete in order); used only
+// while draining after an abort, so it ignores the abort flag
+__device__ __forceinline__ void drain_bar(uint64_t *bar, int issued, bool cluster_scope,
+                                          uint32_t budget = K4_DEFAULT_BUDGET) {
+    if (issued <= 0) return;
+    const uint32_t par = (uint32_t)((issued - 1) & 1);
+    if (cluster_scope) mbar_wait_cluster(bar, par, budget);
+    else mbar_wait(bar, par, budget);
+}
+
+}  // namespace
+
+__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(K4_THREADS, 1)
+prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g,
+                          const float *__restrict__ beta, const float *S0,
+                          __nv_bfloat16 *__restrict__ out, float *S_final,
+                          const int32_t *__restrict__ cu_seqlens, long long T_dense, int H_qk,
+                          int H_v, float scale, int l2norm, DeviceError *err, uint32_t budget)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t r = cluster_rank();
+    const int n = blockIdx.x >> 2, h = blockIdx.y;
+    const int hq = h / (H_v / H_qk);
+    long long t_begin, t_end;
+    if (cu_seqlens) { t_begin = cu_seqlens[n]; t_end = cu_seqlens[n + 1]; }
+    else { t_begin = (long long)n * T_dense; t_end = t_begin + T_dense; }
+    const int nch = (int)((t_end - t_begin + K4_C - 1) / K4_C);
+    const size_t s_off = ((size_t)n * H_v + h) * K4_D * K4_D;
+    const int v0 = (int)r * K4_SL;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S4_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S4_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S4_MISC + 4);
+
+    if (warp == 8) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+    if (tid == 256) {
+        for (int b = 0; b < B_COUNT; ++b) mbar_init(bars + b, (b == B_EMPTY || b == B_SENT) ? 4 : 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // bounded wait; gives up early if another role of this CTA has aborted
+    auto wait_bar = [&](int b, uint32_t parity, bool cluster_scope) -> bool {
+        uint64_t *bar = bars + b;
+        for (uint32_t i = 0; i < budget; ++i) {
+            if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+            if (*abort_flag) return false;
+        }
+        return false;
+    };
+    auto fail = [&](int where) {
+        if (!*abort_flag) {
+            *abort_flag = 1;
+            record_error(err, GDN_ERR_TIMEOUT, where);
+        }
+    };
+
+    if (warp < 4) {
+        // =========================================================== chain group
+        const int t = tid, q = warp, l = lane;
+        const int d = 32 * q + l;                        // TMEM lane = key dim of S_r
+        const int i_row = 16 * q + l;                    // row of M = 64 results (l < 16)
+        const uint32_t loff = (uint32_t)(32 * q) << 16;
+        float *cvec0 = reinterpret_cast<float *>(sm + S4_CVEC);
+        unsigned char *ring = sm + S4_RING;
+        int k_issued = nch > 0 ? 1 : 0;                  // K tiles requested (the first by warp 8)
+
+        // g, beta of chunk c: fetched into registers early, finished into shared memory later
+        float pre_g = 0.f, pre_b = 0.f;
+        auto fetch_vectors = [&](int c) {
+            const long long t0 = t_begin + (long long)c * K4_C;
+            const int L = (int)min((long long)K4_C, t_end - t0);
+            pre_g = (t < L) ? g[(size_t)(t0 + t) * H_v + h] : 0.f;
+            pre_b = (t < L) ? beta[(size_t)(t0 + t) * H_v + h] : 0.f;
+        };
+        auto load_vectors = [&](int c) {                 // g, beta, G, gamma, dte of chunk c
+            float *cv = cvec0 + (c & 1) * 320;
+            float *cg = cv, *cb = cv + 64, *cG = cv + 128, *cgam = cv + 192, *cdte = cv + 256;
+            if (t < K4_C) { cg[t] = pre_g; cb[t] = pre_b; }
+            group_sync<1>();
+            if (q == 0) {
+                const float a0 = cg[2 * l], a1 = cg[2 * l + 1];
+                float s = a0 + a1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, s, o);
+                    if (l >= o) s += y;
+                }
+                const float G0 = s - a1, G1 = s, Ge = __shfl_sync(0xffffffffu, s, 31);
+                cG[2 * l] = G0; cG[2 * l + 1] = G1;
+                cgam[2 * l] = expf(G0); cgam[2 * l + 1] = expf(G1);
+                cdte[2 * l] = expf(Ge - G0); cdte[2 * l + 1] = expf(Ge - G1);
+            }
+            group_sync<1>();
+        };
+
+        // initial state slice: D_S = gamma_end(0) S0_r, S_r^T (bf16) = S0_r
+        float x[32];
+        {
+            const float *src = S0 ? S0 + s_off + (size_t)d * K4_D + v0 : nullptr;
+#pragma unroll
+            for (int v = 0; v < 32; v += 4) {
+                const float4 f = src ? *reinterpret_cast<const float4 *>(src + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                x[v] = f.x; x[v + 1] = f.y; x[v + 2] = f.z; x[v + 3] = f.w;
+            }
+        }
+        if (nch == 0) {
+            if (S_final) {
+                float *dst = S_final + s_off + (size_t)d * K4_D + v0;
+#pragma unroll
+                for (int v = 0; v < 32; v += 4) *reinterpret_cast<float4 *>(dst + v) = make_float4(x[v], x[v + 1], x[v + 2], x[v + 3]);
+            }
+        } else {
+            if (t < K4_C) fetch_vectors(0);
+            load_vectors(0);
+            const float ge0 = cvec0[192 + 63];
+            uint32_t rr[32];
+#pragma unroll
+            for (int v = 0; v < 32; ++v) {
+                store_bf16_at(sm + S4_ST + (d >> 6) * 4096, v, d & 63, x[v]);
+                rr[v] = __float_as_uint(ge0 * x[v]);
+            }
+            tmem_st32(tmem + loff + T4_S, rr);
+            tmem_wait_st();
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync<1>();
+            if (t == 0) {
+                mbar_arrive_local(bars + B_ST);
+                mbar_arrive_local(bars + B_OFREE0);
+                mbar_arrive_local(bars + B_OFREE1);
+            }
+        }
+
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+            const long long t0 = t_begin + (long long)c * K4_C;
+            const int L = (int)min((long long)K4_C, t_end - t0);
+            const int s = c & 1;
+            float *cv = cvec0 + s * 320;
+            const float *cgam = cv + 192, *cdte = cv + 256;
+            if (t < K4_C && c + 1 < nch) fetch_vectors(c + 1);   // lands while this chunk runs
+
+            // ---- K~(c) = diag(decay to chunk end) K; rows past the end get weight 0
+            if (!group_all<1>(wait_bar(B_CK, c & 1, false))) { fail(10); break; }
+            if (l2norm) {                      // rows of K: 2 threads per row, one 128-B half each
+                const int row = t >> 1, half = t & 1;
+                unsigned char *rp = sm + S4_CK + half * 8192 + row * 128;
+                float ss = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ss += f.x * f.x + f.y * f.y; }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                const float rn = rsqrtf(ss + 1e-6f);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
+                    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ws[e] = pack2(f.x * rn, f.y * rn); }
+                    *reinterpret_cast<uint4 *>(rp + cc * 16) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+                }
+                group_sync<1>();
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = t + 128 * u;
+                const int cg = e >> 9, row = (e >> 3) & 63, cc = e & 7;
+                const uint4 w = *reinterpret_cast<const uint4 *>(sm + S4_CK + cg * 8192 + row * 128 + cc * 16);
+                const float wt = row < L ? cdte[row] : 0.f;
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) { const float2 f = unpack2(ws[e2]); o[e2] = pack2(f.x * wt, f.y * wt); }
+                *reinterpret_cast<uint4 *>(sm + S4_CKT + cg * 8192 + row * 128 + cc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            fence_proxy_async();
+            group_sync<1>();
+            if (t == 0) {
+                mbar_arrive_local(bars + B_KT);
+                if (c + 1 < nch) {             // K of the next chunk into the free buffer
+                    ++k_issued;
+                    const int tn = (int)(t0 + K4_C);
+                    mbar_arrive_expect_tx(bars + B_CK, 16384);
+                    tma_load_3d(sm + S4_CK, &tm_k, bars + B_CK, 0, hq, tn);
+                    tma_load_3d(sm + S4_CK + 8192, &tm_k, bars + B_CK, 64, hq, tn);
+                }
+            }
+            if (l2norm) {                      // Q of this chunk, for Q S
+                if (!group_all<1>(wait_bar(B_CQ, c & 1, false))) { fail(11); break; }
+                const int row = t >> 1, half = t & 1;
+                unsigned char *rp = sm + S4_CQ + half * 8192 + row * 128;
+                float ss = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ss += f.x * f.x + f.y * f.y; }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                const float rn = rsqrtf(ss + 1e-6f);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
+                    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ws[e] = pack2(f.x * rn, f.y * rn); }
+                    *reinterpret_cast<uint4 *>(rp + cc * 16) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+                }
+                fence_proxy_async();
+                group_sync<1>();
+                if (t == 0) mbar_arrive_local(bars + B_CQN);
+            }
+
+            // ---- U_r = U~_r - W S_r  ->  U_r^T (bf16, rows v)
+            if (!group_all<1>(wait_bar(B_WS, c & 1, false))) { fail(12); break; }
+            tc_fence_after();
+            {
+                uint32_t ws[32];
+                tmem_ld32(tmem + loff + T4_WS, ws);
+                tmem_wait_ld();
+                if (l < 16) {
+                    const unsigned char *us = ring + s * K4_RING_BYTES + 24576 + i_row * 64;
+                    float uu[32];
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(us + cc * 16);
+                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = unpack2(wv[e]);
+                            uu[8 * cc + 2 * e] = f.x; uu[8 * cc + 2 * e + 1] = f.y;
+                        }
+                    }
+#pragma unroll
+                    for (int v = 0; v < 32; ++v)
+                        store_bf16_at(sm + S4_UT, v, i_row, uu[v] - __uint_as_float(ws[v]));
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync<1>();
+            if (t == 0) mbar_arrive_local(bars + B_U);
+
+            // ---- vectors of the next chunk (its gamma_end scales the state below)
+            if (c + 1 < nch) load_vectors(c + 1);
+            const float ge_next = (c + 1 < nch) ? cvec0[((c + 1) & 1) * 320 + 192 + 63] : 1.f;
+
+            // ---- state: S_r^T (bf16) for the next chunk's products, D_S <- gamma_end(c+1) S_r
+            if (!group_all<1>(wait_bar(B_S2, c & 1, false))) { fail(13); break; }
+            tc_fence_after();
+            {
+                uint32_t rs[32];
+                tmem_ld32(tmem + loff + T4_S, rs);
+                tmem_wait_ld();
+                if (c + 1 == nch) {
+                    if (S_final) {
+                        float *dst = S_final + s_off + (size_t)d * K4_D + v0;
+#pragma unroll
+                        for (int v = 0; v < 32; v += 4)
+                            *reinterpret_cast<float4 *>(dst + v) = make_float4(
+                                __uint_as_float(rs[v]), __uint_as_float(rs[v + 1]),
+                                __uint_as_float(rs[v + 2]), __uint_as_float(rs[v + 3]));
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < 32; ++v) {
+                        const float xv = __uint_as_float(rs[v]);
+                        store_bf16_at(sm + S4_ST + (d >> 6) * 4096, v, d & 63, xv);
+                        rs[v] = __float_as_uint(ge_next * xv);
+                    }
+                    tmem_st32(tmem + loff + T4_S, rs);
+                    tmem_wait_st();
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync<1>();
+            if (t == 0) mbar_arrive_local(bars + B_ST);
+
+            // ---- outputs: o_i = scale (gamma_i (Q S_r)_i + (P U_r)_i), columns [v0, v0 + 32)
+            {
+                uint32_t qs[32], pu[32];
+                tmem_ld32(tmem + loff + T4_QS + 32 * s, qs);
+                tmem_ld32(tmem + loff + T4_PU + 32 * s, pu);
+                tmem_wait_ld();
+                if (l < 16 && i_row < L) {
+                    const float gi = cgam[i_row];
+                    __nv_bfloat16 *dst = out + ((size_t)(t0 + i_row) * H_v + h) * K4_D + v0;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        uint4 w;
+                        uint32_t *pw = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int v = 8 * cc + 2 * e;
+                            pw[e] = pack2(scale * (gi * __uint_as_float(qs[v]) + __uint_as_float(pu[v])),
+                                          scale * (gi * __uint_as_float(qs[v + 1]) + __uint_as_float(pu[v + 1])));
+                        }
+                        *reinterpret_cast<uint4 *>(dst + 8 * cc) = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            group_sync<1>();
+            if (t == 0) mbar_arrive_local(bars + (s ? B_OFREE1 : B_OFREE0));
+        }
+        if (*abort_flag && t == 0) drain_bar(bars + B_CK, k_issued, false);
+    } else if (warp < 8) {
+        // ============================================================= prep group
+        const int t = tid - 128, q = warp - 4, l = lane;
+        const int row = 32 * q + l;                        // TMEM lane
+        const uint32_t loff = (uint32_t)(32 * q) << 16;
+        float *pg = reinterpret_cast<float *>(sm + S4_PVEC);
+        float *pb = pg + 64, *pG = pg + 128, *pgam = pg + 192;
+        float *Af = reinterpret_cast<float *>(sm + S4_AF);
+        float *Tf = reinterpret_cast<float *>(sm + S4_TF);
+
+#pragma unroll 1
+        for (int k = 0;; ++k) {
+            const int p = (int)r + 4 * k;
+            if (p >= nch) break;
+            const long long t0 = t_begin + (long long)p * K4_C;
+            const int L = (int)min((long long)K4_C, t_end - t0);
+            if (t < K4_C) {
+                pg[t] = t < L ? g[(size_t)(t0 + t) * H_v + h] : 0.f;
+                pb[t] = t < L ? beta[(size_t)(t0 + t) * H_v + h] : 0.f;
+            }
+            group_sync<2>();
+            if (q == 0) {
+                const float a0 = pg[2 * l], a1 = pg[2 * l + 1];
+                float s = a0 + a1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, s, o);
+                    if (l >= o) s += y;
+                }
+                const float G0 = s - a1, G1 = s;
+                pG[2 * l] = G0; pG[2 * l + 1] = G1;
+                pgam[2 * l] = expf(G0); pgam[2 * l + 1] = expf(G1);
+            }
+            // ---- inputs: rows past the end zeroed, optional q/k normalisation
+            if (!group_all<2>(wait_bar(B_PKQ, k & 1, false) && wait_bar(B_PV, k & 1, false))) { fail(20); break; }
+            if (L < K4_C) {
+                const int zr = K4_C - L;
+                for (int e = t; e < 6 * zr * 8; e += 128) {
+                    const int region = e / (zr * 8), rr = L + (e % (zr * 8)) / 8, cc = e % 8;
+                    unsigned char *base = region < 4 ? sm + S4_PKQ + region * 8192 : sm + S4_PV + (region - 4) * 8192;
+                    *reinterpret_cast<uint4 *>(base + rr * 128 + cc * 16) = make_uint4(0, 0, 0, 0);
+                }
+                group_sync<2>();
+            }
+            if (l2norm) {                  // thread t: row t of [K;Q] (both 128-byte halves)
+                unsigned char *r0 = sm + S4_PKQ + (t >= 64 ? 8192 : 0) + (t & 63) * 128;
+                float ss = 0.f;
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(r0 + half * 16384 + cc * 16);
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ss += f.x * f.x + f.y * f.y; }
+                    }
+                const float rn = rsqrtf(ss + 1e-6f);
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint4 w = *reinterpret_cast<const uint4 *>(r0 + half * 16384 + cc * 16);
+                        uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ws[e] = pack2(f.x * rn, f.y * rn); }
+                        *reinterpret_cast<uint4 *>(r0 + half * 16384 + cc * 16) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+                    }
+            }
+            fence_proxy_async();
+            group_sync<2>();
+            if (t == 0) mbar_arrive_local(bars + B_PIN);
+
+            // ---- the staging of the previous production must have reached every CTA
+            if (k >= 1 && !group_all<2>(wait_bar(B_SENT, (k - 1) & 1, true))) { fail(21); break; }
+            if (!group_all<2>(wait_bar(B_P1, k & 1, false))) { fail(22); break; }
+            tc_fence_after();
+
+            // ---- A (fp32, rows 0..63) and P (bf16, rows 64..127) from [K;Q] K^T
+            {
+                uint32_t ra[32], rb[32];
+                tmem_ld32(tmem + loff + T4_KQ, ra);
+                tmem_ld32(tmem + loff + T4_KQ + 32, rb);
+                tmem_wait_ld();
+                const bool is_a = q < 2;
+                const int i = is_a ? row : row - 64;
+                const float Gi = pG[i], wi = is_a ? pb[i] : 1.f;
+                float xv[64];
+#pragma unroll
+                for (int j0 = 0; j0 < 64; j0 += 16) {
+                    float gj[16];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4 g4 = *reinterpret_cast<const float4 *>(pG + j0 + 4 * u);
+                        gj[4 * u] = g4.x; gj[4 * u + 1] = g4.y; gj[4 * u + 2] = g4.z; gj[4 * u + 3] = g4.w;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int j = j0 + u;
+                        const float keep = (is_a ? (j < i) : (j <= i)) ? 1.f : 0.f;
+                        const float kk = __uint_as_float(j < 32 ? ra[j] : rb[j - 32]);
+                        xv[j] = (wi * keep) * __expf(fminf(Gi - gj[u], 0.f)) * kk;
+                    }
+                }
+                if (is_a) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) Af[i * TP4 + j] = xv[j];
+                } else {
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint4 w;
+                        w.x = pack2(xv[8 * cc + 0], xv[8 * cc + 1]); w.y = pack2(xv[8 * cc + 2], xv[8 * cc + 3]);
+                        w.z = pack2(xv[8 * cc + 4], xv[8 * cc + 5]); w.w = pack2(xv[8 * cc + 6], xv[8 * cc + 7]);
+                        *reinterpret_cast<uint4 *>(sm + S4_PSTG + sw128(i, cc)) = w;
+                    }
+                }
+#pragma unroll 4
+                for (int e = t; e < 64 * 64; e += 128) {
+                    const int ii = e >> 6, jj = e & 63;
+                    Tf[ii * TP4 + jj] = (ii == jj) ? 1.f : 0.f;
+                }
+            }
+            tc_fence_before();
+            group_sync<2>();
+
+            // ---- T = (I + A)^-1
+            invert_unit_lower_64_tf32_wg<TP4>(Af, Tf, t, [] { group_sync<2>(); });
+            group_sync<2>();
+
+            // ---- T' = T diag(beta gamma), T'' = T diag(beta) (bf16, K-major rows i)
+            {
+                const int which = t >> 6, i = t & 63;
+                float tv[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) tv[j] = Tf[i * TP4 + j];
+                unsigned char *dst = sm + (which ? S4_TPP : S4_TP);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    float w8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = 8 * cc + e;
+                        const float sc = which ? pb[j] : pb[j] * pgam[j];
+                        w8[e] = (j <= i) ? tv[j] * sc : 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(dst + sw128(i, cc)) =
+                        make_uint4(pack2(w8[0], w8[1]), pack2(w8[2], w8[3]), pack2(w8[4], w8[5]), pack2(w8[6], w8[7]));
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync<2>();
+            if (t == 0) mbar_arrive_local(bars + B_TT);
+
+            // ---- W and U~ (M = 64 layout) into the send staging
+            if (!group_all<2>(wait_bar(B_WU, k & 1, false))) { fail(23); break; }
+            tc_fence_after();
+            const int i = 16 * q + l;                        // valid for l < 16
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t rw[32];
+                tmem_ld32(tmem + loff + T4_W + 32 * cb, rw);
+                tmem_wait_ld();
+                if (l < 16) {
+                    unsigned char *dst = sm + S4_WSTG + (cb >> 1) * 8192;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const uint32_t *f = rw + 8 * cc;
+                        *reinterpret_cast<uint4 *>(dst + sw128(i, (cb & 1) * 4 + cc)) = make_uint4(
+                            pack2(__uint_as_float(f[0]), __uint_as_float(f[1])), pack2(__uint_as_float(f[2]), __uint_as_float(f[3])),
+                            pack2(__uint_as_float(f[4]), __uint_as_float(f[5])), pack2(__uint_as_float(f[6]), __uint_as_float(f[7])));
+                    }
+                }
+                tmem_ld32(tmem + loff + T4_U + 32 * cb, rw);
+                tmem_wait_ld();
+                if (l < 16) {
+                    unsigned char *dst = sm + S4_USTG + cb * 4096 + i * 64;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const uint32_t *f = rw + 8 * cc;
+                        *reinterpret_cast<uint4 *>(dst + cc * 16) = make_uint4(
+                            pack2(__uint_as_float(f[0]), __uint_as_float(f[1])), pack2(__uint_as_float(f[2]), __uint_as_float(f[3])),
+                            pack2(__uint_as_float(f[4]), __uint_as_float(f[5])), pack2(__uint_as_float(f[6]), __uint_as_float(f[7])));
+                    }
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            group_sync<2>();
+            if (t == 0) mbar_arrive_local(bars + B_STG);
+        }
+    } else if (warp == 8) {
+        // ========================================================== chain issuer
+        if (lane == 0) {
+            // requests made by this thread, for draining after an abort
+            int q_req = 0, qs_req = 0, ws_req = 0, s2_req = 0, full_req[2] = {0, 0};
+            if (nch > 0) {
+                q_req = 1;
+                full_req[0] = 1;
+                full_req[1] = nch > 1 ? 1 : 0;
+                const int tb = (int)t_begin;
+                mbar_arrive_expect_tx(bars + B_CQ, 16384);
+                tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tb);
+                tma_load_3d(sm + S4_CQ + 8192, &tm_q, bars + B_CQ, 64, hq, tb);
+                mbar_arrive_expect_tx(bars + B_CK, 16384);
+                tma_load_3d(sm + S4_CK, &tm_k, bars + B_CK, 0, hq, tb);
+                tma_load_3d(sm + S4_CK + 8192, &tm_k, bars + B_CK, 64, hq, tb);
+                mbar_arrive_expect_tx(bars + B_FULL0, K4_RING_BYTES);
+                if (nch > 1) mbar_arrive_expect_tx(bars + B_FULL1, K4_RING_BYTES);
+            }
+            const uint32_t id_m64 = idesc_bf16(64, 32, false, false);
+            const uint32_t id_s2 = idesc_bf16(128, 32, true, false);
+#pragma unroll 1
+            for (int c = 0; c < nch; ++c) {
+                const int s = c & 1;
+                const uint32_t ring_s = smem_u32(sm + S4_RING + s * K4_RING_BYTES);
+                const uint32_t st = smem_u32(sm + S4_ST), ut = smem_u32(sm + S4_UT);
+                if (!wait_bar(l2norm ? B_CQN : B_CQ, c & 1, false)) { fail(30); break; }
+                if (!wait_bar(B_ST, c & 1, false)) { fail(31); break; }
+                if (!wait_bar(s ? B_OFREE1 : B_OFREE0, (c >> 1) & 1, false)) { fail(32); break; }
+                tc_fence_after();
+                {   // Q S_r -> D_QS[s]
+                    const uint32_t cq = smem_u32(sm + S4_CQ);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t o4 = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        const uint32_t ob = (ks >> 2) * 4096 + (ks & 3) * 32;
+                        umma_bf16(tmem + T4_QS + 32 * s, sdesc_kmajor(cq + o4), sdesc_kmajor(st + ob), id_m64, ks > 0);
+                    }
+                    umma_commit(bars + B_QS);
+                    ++qs_req;
+                }
+                if (!wait_bar(s ? B_FULL1 : B_FULL0, (c >> 1) & 1, true)) { fail(33); break; }
+                mbar_arrive_remote(map_to_rank(bars + B_SENT, (uint32_t)(c & 3)));
+                tc_fence_after();
+                {   // W S_r -> D_WS
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t o4 = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        const uint32_t ob = (ks >> 2) * 4096 + (ks & 3) * 32;
+                        umma_bf16(tmem + T4_WS, sdesc_kmajor(ring_s + o4), sdesc_kmajor(st + ob), id_m64, ks > 0);
+                    }
+                    umma_commit(bars + B_WS);
+                    ++ws_req;
+                }
+                if (!wait_bar(B_QS, c & 1, false)) { fail(34); break; }
+                if (c + 1 < nch) {             // Q of the next chunk into the free buffer
+                    ++q_req;
+                    const int tn = (int)(t_begin + (long long)(c + 1) * K4_C);
+                    mbar_arrive_expect_tx(bars + B_CQ, 16384);
+                    tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tn);
+                    tma_load_3d(sm + S4_CQ + 8192, &tm_q, bars + B_CQ, 64, hq, tn);
+                }
+                if (!wait_bar(B_U, c & 1, false)) { fail(35); break; }
+                if (!wait_bar(B_KT, c & 1, false)) { fail(36); break; }
+                tc_fence_after();
+                {   // S_r += K~^T U_r ; P U_r -> D_PU[s]
+                    const uint32_t kt = smem_u32(sm + S4_CKT);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + T4_S, sdesc_mnmajor(kt + ks * 2048, 8192), sdesc_kmajor(ut + ks * 32), id_s2, 1);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + T4_PU + 32 * s, sdesc_kmajor(ring_s + 16384 + ks * 32), sdesc_kmajor(ut + ks * 32), id_m64, ks > 0);
+                    umma_commit(bars + B_S2);
+                    ++s2_req;
+                }
+                if (!wait_bar(B_S2, c & 1, false)) { fail(37); break; }
+                if (c + 2 < nch) {             // slot s is free for chunk c + 2
+                    ++full_req[s];
+                    mbar_arrive_expect_tx(bars + (s ? B_FULL1 : B_FULL0), K4_RING_BYTES);
+                    mbar_arrive_remote(map_to_rank(bars + B_EMPTY, (uint32_t)((c + 2) & 3)));
+                }
+            }
+            if (*abort_flag) {
+                // let this thread's loads, MMAs and the copies other CTAs may still be
+                // writing into this CTA's ring land before shared memory and TMEM go away
+                drain_bar(bars + B_CQ, q_req, false);
+                drain_bar(bars + B_QS, qs_req, false);
+                drain_bar(bars + B_WS, ws_req, false);
+                drain_bar(bars + B_S2, s2_req, false);
+                // a producer that sent anything has done so long ago; one that aborted first
+                // never will, so these two waits are kept short
+                drain_bar(bars + B_FULL0, full_req[0], true, 1u << 16);
+                drain_bar(bars + B_FULL1, full_req[1], true, 1u << 16);
+            }
+        }
+        __syncwarp();
+    } else {
+        // =========================================================== prep issuer
+        if (lane == 0) {
+            int in_req = 0, p1_req = 0, wu_req = 0;
+            const uint32_t id_p1 = idesc_bf16(128, 64, false, false);
+            const uint32_t id_wu = idesc_bf16(64, 128, false, true);
+#pragma unroll 1
+            for (int k = 0;; ++k) {
+                const int p = (int)r + 4 * k;
+                if (p >= nch) break;
+                const int tp = (int)(t_begin + (long long)p * K4_C);
+                ++in_req;
+                mbar_arrive_expect_tx(bars + B_PKQ, 32768);
+                tma_load_3d(sm + S4_PKQ, &tm_k, bars + B_PKQ, 0, hq, tp);
+                tma_load_3d(sm + S4_PKQ + 16384, &tm_k, bars + B_PKQ, 64, hq, tp);
+                tma_load_3d(sm + S4_PKQ + 8192, &tm_q, bars + B_PKQ, 0, hq, tp);
+                tma_load_3d(sm + S4_PKQ + 24576, &tm_q, bars + B_PKQ, 64, hq, tp);
+                mbar_arrive_expect_tx(bars + B_PV, 16384);
+                tma_load_3d(sm + S4_PV, &tm_v, bars + B_PV, 0, h, tp);
+                tma_load_3d(sm + S4_PV + 8192, &tm_v, bars + B_PV, 64, h, tp);
+                if (!wait_bar(B_PIN, k & 1, false)) { fail(40); break; }
+                tc_fence_after();
+                {   // P1: [K;Q] K^T
+                    const uint32_t kq = smem_u32(sm + S4_PKQ);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t a = kq + (ks >> 2) * 16384 + (ks & 3) * 32;
+                        umma_bf16(tmem + T4_KQ, sdesc_kmajor(a), sdesc_kmajor(a), id_p1, ks > 0);
+                    }
+                    umma_commit(bars + B_P1);
+                    ++p1_req;
+                }
+                if (!wait_bar(B_TT, k & 1, false)) { fail(41); break; }
+                tc_fence_after();
+                {   // W = T' K ; U~ = T'' V   (M = 64, N = 128)
+                    const uint32_t kq = smem_u32(sm + S4_PKQ), pv = smem_u32(sm + S4_PV);
+                    const uint32_t tpa = smem_u32(sm + S4_TP), tppa = smem_u32(sm + S4_TPP);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + T4_W, sdesc_kmajor(tpa + ks * 32), sdesc_mnmajor(kq + ks * 2048, 16384), id_wu, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + T4_U, sdesc_kmajor(tppa + ks * 32), sdesc_mnmajor(pv + ks * 2048, 8192), id_wu, ks > 0);
+                    umma_commit(bars + B_WU);
+                    ++wu_req;
+                }
+                if (!wait_bar(B_WU, k & 1, false)) { fail(42); break; }
+                if (!wait_bar(B_STG, k & 1, false)) { fail(43); break; }
+                // every consumer has released slot (p & 1) (it finished chunk p - 2)
+                if ((int)r >= 2) {
+                    if (!wait_bar(B_EMPTY, k & 1, true)) { fail(44); break; }
+                } else if (k >= 1) {
+                    if (!wait_bar(B_EMPTY, (k - 1) & 1, true)) { fail(44); break; }
+                }
+                const int s = p & 1;
+                unsigned char *slot = sm + S4_RING + s * K4_RING_BYTES;
+#pragma unroll 1
+                for (uint32_t dst = 0; dst < 4; ++dst) {
+                    const uint32_t bar = map_to_rank(bars + (s ? B_FULL1 : B_FULL0), dst);
+                    bulk_copy_to_cluster(map_to_rank(slot, dst), sm + S4_WSTG, 16384, bar);
+                    bulk_copy_to_cluster(map_to_rank(slot + 16384, dst), sm + S4_PSTG, 8192, bar);
+                    bulk_copy_to_cluster(map_to_rank(slot + 24576, dst), sm + S4_USTG + dst * 4096, 4096, bar);
+                }
+            }
+            if (*abort_flag) {
+                drain_bar(bars + B_PKQ, in_req, false);
+                drain_bar(bars + B_PV, in_req, false);
+                drain_bar(bars + B_P1, p1_req, false);
+                drain_bar(bars + B_WU, wu_req, false);
+            }
+        }
+        __syncwarp();
+    }
+
+    // ------------------------------------------------------------------ teardown
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 8) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------------ host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder4() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool make_map4(CUtensorMap *map, const void *base, long long T_total, int H) {
+    auto enc = encoder4();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T_total};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+uint32_t wait_budget4() {
+    const char *env = getenv("GDN_TEST_WAIT_BUDGET");
+    return env ? (uint32_t)strtoul(env, nullptr, 10) : K4_DEFAULT_BUDGET;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *v, const float *g,
+                                      const float *beta, const float *S0, void *out, float *S_final,
+                                      const int32_t *cu, int N, long long T_dense, long long T_total,
+                                      int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
+                                      cudaStream_t stream)
+{
+    if (T_total >= (1LL << 31) || (long long)N * 4 > 0x7fffffffLL) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv;
+    if (!make_map4(&mq, q, T_total, H_qk) || !make_map4(&mk, k, T_total, H_qk) ||
+        !make_map4(&mv, v, T_total, H_v))
+        return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_cluster_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, K4_SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid((unsigned)(4 * N), (unsigned)H_v);
+    prefill_tc_cluster_kernel<<<grid, K4_THREADS, K4_SMEM, stream>>>(
+        mq, mk, mv, g, beta, S0, (__nv_bfloat16 *)out, S_final, cu, T_dense, H_qk, H_v, scale,
+        l2norm, err, wait_budget4());
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

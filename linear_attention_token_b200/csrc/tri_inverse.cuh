@@ -204,4 +204,45 @@ __device__ __forceinline__ void invert_unit_lower_64_tf32(float *A, float *T, in
     }
 }
 
+// Warpgroup version: the same algorithm run by 128 threads (t = 0..127) that
+// synchronise with `sync()` (a named barrier over exactly those threads).
+template <int TP, typename Sync>
+__device__ __forceinline__ void invert_unit_lower_64_tf32_wg(float *A, float *T, int t, Sync sync)
+{
+    const int warp = t >> 5, lane = t & 31;
+    if (t < 64) {
+        const int b = t >> 4, col = t & 15;
+        const float *Ab = A + (16 * b) * TP + 16 * b;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int m = 0; m + 1 < r; m += 2) {
+                acc0 = fmaf(Ab[r * TP + m], x[m], acc0);
+                acc1 = fmaf(Ab[r * TP + m + 1], x[m + 1], acc1);
+            }
+            if (r & 1) acc0 = fmaf(Ab[r * TP + r - 1], x[r - 1], acc0);
+            x[r] = (r == col) ? 1.f : ((r < col) ? 0.f : -(acc0 + acc1));
+        }
+        float *Tb = T + (16 * b) * TP + 16 * b;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tb[r * TP + col] = x[r];
+    }
+    sync();
+    if (warp < 2) {
+        const int lo = 32 * warp, hi = lo + 16;
+        warp_gemm_16x16<TP, 16>(A + hi * TP + lo, T + lo * TP + lo, A + lo * TP + hi, 1.f, lane);
+        __syncwarp();
+        warp_gemm_16x16<TP, 16>(T + hi * TP + hi, A + lo * TP + hi, T + hi * TP + lo, -1.f, lane);
+    }
+    sync();
+    {
+        const int mb = (warp >> 1) * 16, nb = (warp & 1) * 16;
+        warp_gemm_16x16<TP, 32>(A + (32 + mb) * TP, T + nb, A + mb * TP + 32 + nb, 1.f, lane);
+        sync();
+        warp_gemm_16x16<TP, 32>(T + (32 + mb) * TP + 32, A + 32 + nb, T + (32 + mb) * TP + nb, -1.f, lane);
+    }
+}
+
 }  // namespace gdn
