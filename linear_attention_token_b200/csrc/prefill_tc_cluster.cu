@@ -127,6 +127,23 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, int issued, bool cluste
 
 }  // namespace
 
+// Profiling aid, compiled in only with -DGDN_PHASE_TIMERS: CTA (0, 0) records clock64()
+// at fixed points of its chain (per chunk) and of its preparations (per production).
+#ifdef GDN_PHASE_TIMERS
+__device__ unsigned long long g4_chain[64][16];
+__device__ unsigned long long g4_prep[16][16];
+#define CMARK(c, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (c) < 64) g4_chain[(c)][(k)] = clock64(); } while (0)
+#define PMARK(kk, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (kk) < 16) g4_prep[(kk)][(k)] = clock64(); } while (0)
+extern "C" __attribute__((visibility("default"))) int gdn_debug_cluster_timeline(void *chain, void *prep)
+{
+    if (cudaMemcpyFromSymbol(chain, g4_chain, sizeof(g4_chain)) != cudaSuccess) return 1;
+    return (int)cudaMemcpyFromSymbol(prep, g4_prep, sizeof(g4_prep));
+}
+#else
+#define CMARK(c, k) do { } while (0)
+#define PMARK(kk, k) do { } while (0)
+#endif
+
 __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(K4_THREADS, 1)
 prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -269,6 +286,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 
             // ---- K~(c) = diag(decay to chunk end) K; rows past the end get weight 0
             if (!group_all<1>(wait_bar(B_CK, c & 1, false))) { fail(10); break; }
+            if (t == 0) CMARK(c, 7);
             if (l2norm) {                      // rows of K: 2 threads per row, one 128-B half each
                 const int row = t >> 1, half = t & 1;
                 unsigned char *rp = sm + S4_CK + half * 8192 + row * 128;
@@ -307,6 +325,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             group_sync<1>();
             if (t == 0) {
+                CMARK(c, 8);
                 mbar_arrive_local(bars + B_KT);
                 if (c + 1 < nch) {             // K of the next chunk into the free buffer
                     ++k_issued;
@@ -345,6 +364,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 
             // ---- U_r = U~_r - W S_r  ->  U_r^T (bf16, rows v)
             if (!group_all<1>(wait_bar(B_WS, c & 1, false))) { fail(12); break; }
+            if (t == 0) CMARK(c, 9);
             tc_fence_after();
             {
                 uint32_t ws[32];
@@ -371,14 +391,16 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<1>();
-            if (t == 0) mbar_arrive_local(bars + B_U);
+            if (t == 0) { mbar_arrive_local(bars + B_U); CMARK(c, 10); }
 
             // ---- vectors of the next chunk (its gamma_end scales the state below)
             if (c + 1 < nch) load_vectors(c + 1);
             const float ge_next = (c + 1 < nch) ? cvec0[((c + 1) & 1) * 320 + 192 + 63] : 1.f;
 
             // ---- state: S_r^T (bf16) for the next chunk's products, D_S <- gamma_end(c+1) S_r
+            if (t == 0) CMARK(c, 11);
             if (!group_all<1>(wait_bar(B_S2, c & 1, false))) { fail(13); break; }
+            if (t == 0) CMARK(c, 12);
             tc_fence_after();
             {
                 uint32_t rs[32];
@@ -407,7 +429,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<1>();
-            if (t == 0) mbar_arrive_local(bars + B_ST);
+            if (t == 0) { mbar_arrive_local(bars + B_ST); CMARK(c, 13); }
 
             // ---- outputs: o_i = scale (gamma_i (Q S_r)_i + (P U_r)_i), columns [v0, v0 + 32)
             {
@@ -434,7 +456,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             tc_fence_before();
             group_sync<1>();
-            if (t == 0) mbar_arrive_local(bars + (s ? B_OFREE1 : B_OFREE0));
+            if (t == 0) { mbar_arrive_local(bars + (s ? B_OFREE1 : B_OFREE0)); CMARK(c, 14); }
         }
         if (*abort_flag && t == 0) drain_bar(bars + B_CK, k_issued, false);
     } else if (warp < 8) {
@@ -453,6 +475,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (p >= nch) break;
             const long long t0 = t_begin + (long long)p * K4_C;
             const int L = (int)min((long long)K4_C, t_end - t0);
+            if (t == 0) PMARK(k, 0);
             if (t < K4_C) {
                 pg[t] = t < L ? g[(size_t)(t0 + t) * H_v + h] : 0.f;
                 pb[t] = t < L ? beta[(size_t)(t0 + t) * H_v + h] : 0.f;
@@ -472,6 +495,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             // ---- inputs: rows past the end zeroed, optional q/k normalisation
             if (!group_all<2>(wait_bar(B_PKQ, k & 1, false) && wait_bar(B_PV, k & 1, false))) { fail(20); break; }
+            if (t == 0) PMARK(k, 1);
             if (L < K4_C) {
                 const int zr = K4_C - L;
                 for (int e = t; e < 6 * zr * 8; e += 128) {
@@ -511,7 +535,9 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 
             // ---- the staging of the previous production must have reached every CTA
             if (k >= 1 && !group_all<2>(wait_bar(B_SENT, (k - 1) & 1, true))) { fail(21); break; }
+            if (t == 0) PMARK(k, 2);
             if (!group_all<2>(wait_bar(B_P1, k & 1, false))) { fail(22); break; }
+            if (t == 0) PMARK(k, 3);
             tc_fence_after();
 
             // ---- A (fp32, rows 0..63) and P (bf16, rows 64..127) from [K;Q] K^T
@@ -561,9 +587,11 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             tc_fence_before();
             group_sync<2>();
 
+            if (t == 0) PMARK(k, 4);
             // ---- T = (I + A)^-1
             invert_unit_lower_64_tf32_wg<TP4>(Af, Tf, t, [] { group_sync<2>(); });
             group_sync<2>();
+            if (t == 0) PMARK(k, 5);
 
             // ---- T' = T diag(beta gamma), T'' = T diag(beta) (bf16, K-major rows i)
             {
@@ -588,10 +616,11 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<2>();
-            if (t == 0) mbar_arrive_local(bars + B_TT);
+            if (t == 0) { mbar_arrive_local(bars + B_TT); PMARK(k, 6); }
 
             // ---- W and U~ (M = 64 layout) into the send staging
             if (!group_all<2>(wait_bar(B_WU, k & 1, false))) { fail(23); break; }
+            if (t == 0) PMARK(k, 7);
             tc_fence_after();
             const int i = 16 * q + l;                        // valid for l < 16
 #pragma unroll 1
@@ -625,7 +654,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<2>();
-            if (t == 0) mbar_arrive_local(bars + B_STG);
+            if (t == 0) { mbar_arrive_local(bars + B_STG); PMARK(k, 8); }
         }
     } else if (warp == 8) {
         // ========================================================== chain issuer
@@ -653,11 +682,30 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int s = c & 1;
                 const uint32_t ring_s = smem_u32(sm + S4_RING + s * K4_RING_BYTES);
                 const uint32_t st = smem_u32(sm + S4_ST), ut = smem_u32(sm + S4_UT);
-                if (!wait_bar(l2norm ? B_CQN : B_CQ, c & 1, false)) { fail(30); break; }
+                CMARK(c, 0);
+                // W S_r is on the state chain: it needs S_r^T of the previous chunk and W of
+                // this one, and goes first
                 if (!wait_bar(B_ST, c & 1, false)) { fail(31); break; }
+                if (!wait_bar(s ? B_FULL1 : B_FULL0, (c >> 1) & 1, true)) { fail(33); break; }
+                CMARK(c, 1);
+                tc_fence_after();
+                {
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t o4 = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        const uint32_t ob = (ks >> 2) * 4096 + (ks & 3) * 32;
+                        umma_bf16(tmem + T4_WS, sdesc_kmajor(ring_s + o4), sdesc_kmajor(st + ob), id_m64, ks > 0);
+                    }
+                    umma_commit(bars + B_WS);
+                    ++ws_req;
+                }
+                CMARK(c, 2);
+                mbar_arrive_remote_relaxed(map_to_rank(bars + B_SENT, (uint32_t)(c & 3)));
+                // Q S_r feeds only the outputs
+                if (!wait_bar(l2norm ? B_CQN : B_CQ, c & 1, false)) { fail(30); break; }
                 if (!wait_bar(s ? B_OFREE1 : B_OFREE0, (c >> 1) & 1, false)) { fail(32); break; }
                 tc_fence_after();
-                {   // Q S_r -> D_QS[s]
+                {
                     const uint32_t cq = smem_u32(sm + S4_CQ);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
@@ -668,27 +716,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     umma_commit(bars + B_QS);
                     ++qs_req;
                 }
-                if (!wait_bar(s ? B_FULL1 : B_FULL0, (c >> 1) & 1, true)) { fail(33); break; }
-                mbar_arrive_remote(map_to_rank(bars + B_SENT, (uint32_t)(c & 3)));
-                tc_fence_after();
-                {   // W S_r -> D_WS
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t o4 = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        const uint32_t ob = (ks >> 2) * 4096 + (ks & 3) * 32;
-                        umma_bf16(tmem + T4_WS, sdesc_kmajor(ring_s + o4), sdesc_kmajor(st + ob), id_m64, ks > 0);
-                    }
-                    umma_commit(bars + B_WS);
-                    ++ws_req;
-                }
-                if (!wait_bar(B_QS, c & 1, false)) { fail(34); break; }
-                if (c + 1 < nch) {             // Q of the next chunk into the free buffer
-                    ++q_req;
-                    const int tn = (int)(t_begin + (long long)(c + 1) * K4_C);
-                    mbar_arrive_expect_tx(bars + B_CQ, 16384);
-                    tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tn);
-                    tma_load_3d(sm + S4_CQ + 8192, &tm_q, bars + B_CQ, 64, hq, tn);
-                }
+                CMARK(c, 3);
                 if (!wait_bar(B_U, c & 1, false)) { fail(35); break; }
                 if (!wait_bar(B_KT, c & 1, false)) { fail(36); break; }
                 tc_fence_after();
@@ -703,11 +731,22 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     umma_commit(bars + B_S2);
                     ++s2_req;
                 }
+                CMARK(c, 4);
+                // Q of the next chunk into the buffer Q S_r has finished reading
+                if (!wait_bar(B_QS, c & 1, false)) { fail(34); break; }
+                if (c + 1 < nch) {
+                    ++q_req;
+                    const int tn = (int)(t_begin + (long long)(c + 1) * K4_C);
+                    mbar_arrive_expect_tx(bars + B_CQ, 16384);
+                    tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tn);
+                    tma_load_3d(sm + S4_CQ + 8192, &tm_q, bars + B_CQ, 64, hq, tn);
+                }
                 if (!wait_bar(B_S2, c & 1, false)) { fail(37); break; }
+                CMARK(c, 5);
                 if (c + 2 < nch) {             // slot s is free for chunk c + 2
                     ++full_req[s];
                     mbar_arrive_expect_tx(bars + (s ? B_FULL1 : B_FULL0), K4_RING_BYTES);
-                    mbar_arrive_remote(map_to_rank(bars + B_EMPTY, (uint32_t)((c + 2) & 3)));
+                    mbar_arrive_remote_relaxed(map_to_rank(bars + B_EMPTY, (uint32_t)((c + 2) & 3)));
                 }
             }
             if (*abort_flag) {
@@ -730,10 +769,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             int in_req = 0, p1_req = 0, wu_req = 0;
             const uint32_t id_p1 = idesc_bf16(128, 64, false, false);
             const uint32_t id_wu = idesc_bf16(64, 128, false, true);
-#pragma unroll 1
-            for (int k = 0;; ++k) {
-                const int p = (int)r + 4 * k;
-                if (p >= nch) break;
+            auto load_inputs = [&](int p) {       // K, Q, V of chunk p into the prep buffers
                 const int tp = (int)(t_begin + (long long)p * K4_C);
                 ++in_req;
                 mbar_arrive_expect_tx(bars + B_PKQ, 32768);
@@ -744,6 +780,12 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 mbar_arrive_expect_tx(bars + B_PV, 16384);
                 tma_load_3d(sm + S4_PV, &tm_v, bars + B_PV, 0, h, tp);
                 tma_load_3d(sm + S4_PV + 8192, &tm_v, bars + B_PV, 64, h, tp);
+            };
+            if ((int)r < nch) load_inputs((int)r);
+#pragma unroll 1
+            for (int k = 0;; ++k) {
+                const int p = (int)r + 4 * k;
+                if (p >= nch) break;
                 if (!wait_bar(B_PIN, k & 1, false)) { fail(40); break; }
                 tc_fence_after();
                 {   // P1: [K;Q] K^T
@@ -771,6 +813,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     ++wu_req;
                 }
                 if (!wait_bar(B_WU, k & 1, false)) { fail(42); break; }
+                if (p + 4 < nch) load_inputs(p + 4);   // the prep buffers are free again
                 if (!wait_bar(B_STG, k & 1, false)) { fail(43); break; }
                 // every consumer has released slot (p & 1) (it finished chunk p - 2)
                 if ((int)r >= 2) {
@@ -778,6 +821,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 } else if (k >= 1) {
                     if (!wait_bar(B_EMPTY, (k - 1) & 1, true)) { fail(44); break; }
                 }
+                PMARK(k, 9);
                 const int s = p & 1;
                 unsigned char *slot = sm + S4_RING + s * K4_RING_BYTES;
 #pragma unroll 1

@@ -171,7 +171,168 @@ cluster_kernel(int *out)
     cluster_sync();                                        // nobody leaves while others may copy
 }
 
+// Timing probe: `reps` rounds of `nmma` MMAs of one placement, each round committed and
+// waited for; records clock64 per round (issue of the first MMA to completion seen).
+__global__ void __launch_bounds__(128, 1)
+umma_timing_kernel(int variant, int nmma, int reps, long long *cycles, int streams)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const bool a_mn = variant & 1, b_mn = variant & 2;
+    const int M = (variant & 32) ? 64 : 128;
+    const int N = (variant & 64) ? 32 : ((variant & 8) ? 128 : 64);
+    unsigned char *As = base, *Bs = base + 65536;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    for (int i = tid; i < 32768; i += 128) reinterpret_cast<uint32_t *>(base)[i] = 0x3c003c00u;
+    if (warp == 0) { tmem_alloc(&tmem_base, 512); tmem_relinquish(); }
+    if (tid == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(M, N, a_mn, b_mn, false);
+        for (int rep = 0; rep < reps; ++rep) {
+            const long long t0 = clock64();
+            for (int s = 0; s < nmma; ++s) {
+                const uint32_t ks = s & 7;
+                const uint32_t a_addr = a_mn ? smem_u32(As) + ks * 2048 : smem_u32(As) + (ks / 4) * (M * 128) + (ks % 4) * 32;
+                const uint32_t b_addr = b_mn ? smem_u32(Bs) + ks * 2048 : smem_u32(Bs) + (ks / 4) * (N * 128) + (ks % 4) * 32;
+                const uint64_t ad = a_mn ? sdesc_mnmajor(a_addr, 16384) : sdesc_kmajor(a_addr);
+                const uint64_t bd = b_mn ? sdesc_mnmajor(b_addr, 16384) : sdesc_kmajor(b_addr);
+                // `streams` independent accumulators, used round-robin
+                const int st = s % streams;
+                umma_bf16(tmem_base + st * N, ad, bd, id, s >= streams);
+            }
+            umma_commit(&bar);
+            mbar_wait(&bar, rep & 1, 1u << 22);
+            cycles[rep] = clock64() - t0;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem_base, 512);
+}
+
+// Timing probe with compile-time shape: NMMA MMAs (M x N x 16, both operands K-major),
+// descriptors precomputed, fully unrolled; D accumulates in place.
+template <int M, int N, int NMMA>
+__global__ void __launch_bounds__(128, 1) umma_timing2_kernel(int reps, long long *cycles)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char *As = base, *Bs = base + 65536;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    for (int i = tid; i < 32768; i += 128) reinterpret_cast<uint32_t *>(base)[i] = 0x3c003c00u;
+    if (warp == 0) { tmem_alloc(&tmem_base, 512); tmem_relinquish(); }
+    if (tid == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+        constexpr uint32_t id = idesc_bf16(M, N, false, false, false);
+        uint64_t ad[8], bd[8];
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            ad[ks] = sdesc_kmajor(smem_u32(As) + (ks / 4) * (M * 128) + (ks % 4) * 32);
+            bd[ks] = sdesc_kmajor(smem_u32(Bs) + (ks / 4) * (N * 128) + (ks % 4) * 32);
+        }
+        const uint32_t d = tmem_base;
+        for (int rep = 0; rep < reps; ++rep) {
+            const long long t0 = clock64();
+#pragma unroll
+            for (int s2 = 0; s2 < NMMA; ++s2) umma_bf16(d, ad[s2 & 7], bd[s2 & 7], id, s2 > 0);
+            umma_commit(&bar);
+            mbar_wait(&bar, rep & 1, 1u << 22);
+            cycles[rep] = clock64() - t0;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem_base, 512);
+}
+
+// Timing probe: one TMA tile load of `boxes` boxes (64 tokens x 128 B each) of a
+// [T, H, 128] bf16 tensor, issue to completion seen, repeated `reps` times.
+__global__ void tma_timing_kernel(const __grid_constant__ CUtensorMap map, int boxes, int reps,
+                                  int stride_tokens, long long *cycles)
+{
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        for (int rep = 0; rep < reps; ++rep) {
+            const long long t0 = clock64();
+            mbar_arrive_expect_tx(&bar, boxes * 8192);
+            for (int b = 0; b < boxes; ++b)
+                tma_load_3d(base + b * 8192, &map, &bar, (b & 1) * 64, (b >> 1), rep * stride_tokens);
+            mbar_wait(&bar, rep & 1, 1u << 22);
+            cycles[rep] = clock64() - t0;
+        }
+    }
+}
+
 }  // namespace
+
+extern "C" __attribute__((visibility("default")))
+int selftest_umma_timing(int variant, int nmma, int reps, long long *cycles, int streams)
+{
+    const int smem = 131072 + 1024;
+    cudaFuncSetAttribute(umma_timing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    umma_timing_kernel<<<1, 128, smem>>>(variant, nmma, reps, cycles, streams);
+    return (int)cudaDeviceSynchronize();
+}
+
+#define GDN_T2(Mv, Nv, Kn)                                                                   \
+    if (M == Mv && N == Nv && nmma == Kn) {                                                  \
+        cudaFuncSetAttribute(umma_timing2_kernel<Mv, Nv, Kn>,                                \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);              \
+        umma_timing2_kernel<Mv, Nv, Kn><<<1, 128, smem>>>(reps, cycles);                      \
+        return (int)cudaDeviceSynchronize();                                                 \
+    }
+extern "C" __attribute__((visibility("default")))
+int selftest_umma_timing2(int M, int N, int nmma, int reps, long long *cycles)
+{
+    const int smem = 131072 + 1024;
+    GDN_T2(128, 256, 8) GDN_T2(128, 256, 32) GDN_T2(128, 128, 8) GDN_T2(128, 128, 32)
+    GDN_T2(128, 64, 8) GDN_T2(128, 64, 32) GDN_T2(128, 32, 8) GDN_T2(128, 32, 32)
+    GDN_T2(64, 32, 8) GDN_T2(64, 32, 32) GDN_T2(64, 128, 32) GDN_T2(128, 256, 1) GDN_T2(128, 32, 1)
+    return -1;
+}
+
+extern "C" __attribute__((visibility("default")))
+int selftest_tma_timing(const void *src, int T, int H, int boxes, int reps, int stride_tokens,
+                        long long *cycles)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", (void **)&encode, cudaEnableDefault, &q)
+            != cudaSuccess || !encode)
+        return -1;
+    CUtensorMap map;
+    cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)T};
+    cuuint64_t strides[2] = {128 * 2, (cuuint64_t)H * 128 * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(src), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return -2;
+    const int smem = 65536 + 1024;
+    cudaFuncSetAttribute(tma_timing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    tma_timing_kernel<<<1, 32, smem>>>(map, boxes, reps, stride_tokens, cycles);
+    return (int)cudaDeviceSynchronize();
+}
 
 extern "C" __attribute__((visibility("default")))
 int selftest_cluster(int *out)
