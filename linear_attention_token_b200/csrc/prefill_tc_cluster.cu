@@ -46,7 +46,7 @@ namespace {
 constexpr int K4_C = 64;                 // chunk
 constexpr int K4_D = 128;                // dk = dv
 constexpr int K4_SL = 32;                // value columns per CTA
-constexpr int K4_THREADS = 320;
+constexpr int K4_THREADS = 448;
 constexpr uint32_t K4_DEFAULT_BUDGET = 1u << 22;
 constexpr uint32_t K4_RING_BYTES = 28672;    // W 16 KB + P 8 KB + U~ slice 4 KB
 
@@ -85,7 +85,7 @@ constexpr int TP4 = 65;
 
 enum Bar {
     B_CQ = 0, B_CK, B_FULL0, B_FULL1, B_QS, B_WS, B_S2, B_KT, B_U, B_ST, B_OFREE0, B_OFREE1,
-    B_PKQ, B_PV, B_P1, B_TT, B_WU, B_STG, B_EMPTY, B_SENT, B_PIN, B_CQN, B_COUNT
+    B_PKQ, B_PV, B_P1, B_TT, B_WU, B_STG, B_EMPTY, B_SENT, B_PIN, B_CQN, B_VEC, B_PU, B_COUNT
 };
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -200,42 +200,14 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (warp < 4) {
         // =========================================================== chain group
+        // U and state epilogues only: the two CUDA-core steps on the state chain
         const int t = tid, q = warp, l = lane;
         const int d = 32 * q + l;                        // TMEM lane = key dim of S_r
         const int i_row = 16 * q + l;                    // row of M = 64 results (l < 16)
         const uint32_t loff = (uint32_t)(32 * q) << 16;
-        float *cvec0 = reinterpret_cast<float *>(sm + S4_CVEC);
-        unsigned char *ring = sm + S4_RING;
-        int k_issued = nch > 0 ? 1 : 0;                  // K tiles requested (the first by warp 8)
-
-        // g, beta of chunk c: fetched into registers early, finished into shared memory later
-        float pre_g = 0.f, pre_b = 0.f;
-        auto fetch_vectors = [&](int c) {
-            const long long t0 = t_begin + (long long)c * K4_C;
-            const int L = (int)min((long long)K4_C, t_end - t0);
-            pre_g = (t < L) ? g[(size_t)(t0 + t) * H_v + h] : 0.f;
-            pre_b = (t < L) ? beta[(size_t)(t0 + t) * H_v + h] : 0.f;
-        };
-        auto load_vectors = [&](int c) {                 // g, beta, G, gamma, dte of chunk c
-            float *cv = cvec0 + (c & 1) * 320;
-            float *cg = cv, *cb = cv + 64, *cG = cv + 128, *cgam = cv + 192, *cdte = cv + 256;
-            if (t < K4_C) { cg[t] = pre_g; cb[t] = pre_b; }
-            group_sync<1>();
-            if (q == 0) {
-                const float a0 = cg[2 * l], a1 = cg[2 * l + 1];
-                float s = a0 + a1;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, s, o);
-                    if (l >= o) s += y;
-                }
-                const float G0 = s - a1, G1 = s, Ge = __shfl_sync(0xffffffffu, s, 31);
-                cG[2 * l] = G0; cG[2 * l + 1] = G1;
-                cgam[2 * l] = expf(G0); cgam[2 * l + 1] = expf(G1);
-                cdte[2 * l] = expf(Ge - G0); cdte[2 * l + 1] = expf(Ge - G1);
-            }
-            group_sync<1>();
-        };
+        const float *cvec0 = reinterpret_cast<const float *>(sm + S4_CVEC);
+        const unsigned char *ring = sm + S4_RING;
+        bool ok = true;
 
         // initial state slice: D_S = gamma_end(0) S0_r, S_r^T (bf16) = S0_r
         float x[32];
@@ -253,9 +225,10 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int v = 0; v < 32; v += 4) *reinterpret_cast<float4 *>(dst + v) = make_float4(x[v], x[v + 1], x[v + 2], x[v + 3]);
             }
+        } else if (!group_all<1>(t != 0 || wait_bar(B_VEC, 0, false))) {
+            fail(15);
+            ok = false;
         } else {
-            if (t < K4_C) fetch_vectors(0);
-            load_vectors(0);
             const float ge0 = cvec0[192 + 63];
             uint32_t rr[32];
 #pragma unroll
@@ -268,102 +241,14 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<1>();
-            if (t == 0) {
-                mbar_arrive_local(bars + B_ST);
-                mbar_arrive_local(bars + B_OFREE0);
-                mbar_arrive_local(bars + B_OFREE1);
-            }
+            if (t == 0) mbar_arrive_local(bars + B_ST);
         }
 
 #pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-            const long long t0 = t_begin + (long long)c * K4_C;
-            const int L = (int)min((long long)K4_C, t_end - t0);
+        for (int c = 0; ok && c < nch; ++c) {
             const int s = c & 1;
-            float *cv = cvec0 + s * 320;
-            const float *cgam = cv + 192, *cdte = cv + 256;
-            if (t < K4_C && c + 1 < nch) fetch_vectors(c + 1);   // lands while this chunk runs
-
-            // ---- K~(c) = diag(decay to chunk end) K; rows past the end get weight 0
-            if (!group_all<1>(wait_bar(B_CK, c & 1, false))) { fail(10); break; }
-            if (t == 0) CMARK(c, 7);
-            if (l2norm) {                      // rows of K: 2 threads per row, one 128-B half each
-                const int row = t >> 1, half = t & 1;
-                unsigned char *rp = sm + S4_CK + half * 8192 + row * 128;
-                float ss = 0.f;
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ss += f.x * f.x + f.y * f.y; }
-                }
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                const float rn = rsqrtf(ss + 1e-6f);
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
-                    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ws[e] = pack2(f.x * rn, f.y * rn); }
-                    *reinterpret_cast<uint4 *>(rp + cc * 16) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
-                }
-                group_sync<1>();
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = t + 128 * u;
-                const int cg = e >> 9, row = (e >> 3) & 63, cc = e & 7;
-                const uint4 w = *reinterpret_cast<const uint4 *>(sm + S4_CK + cg * 8192 + row * 128 + cc * 16);
-                const float wt = row < L ? cdte[row] : 0.f;
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                uint32_t o[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) { const float2 f = unpack2(ws[e2]); o[e2] = pack2(f.x * wt, f.y * wt); }
-                *reinterpret_cast<uint4 *>(sm + S4_CKT + cg * 8192 + row * 128 + cc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-            fence_proxy_async();
-            group_sync<1>();
-            if (t == 0) {
-                CMARK(c, 8);
-                mbar_arrive_local(bars + B_KT);
-                if (c + 1 < nch) {             // K of the next chunk into the free buffer
-                    ++k_issued;
-                    const int tn = (int)(t0 + K4_C);
-                    mbar_arrive_expect_tx(bars + B_CK, 16384);
-                    tma_load_3d(sm + S4_CK, &tm_k, bars + B_CK, 0, hq, tn);
-                    tma_load_3d(sm + S4_CK + 8192, &tm_k, bars + B_CK, 64, hq, tn);
-                }
-            }
-            if (l2norm) {                      // Q of this chunk, for Q S
-                if (!group_all<1>(wait_bar(B_CQ, c & 1, false))) { fail(11); break; }
-                const int row = t >> 1, half = t & 1;
-                unsigned char *rp = sm + S4_CQ + half * 8192 + row * 128;
-                float ss = 0.f;
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ss += f.x * f.x + f.y * f.y; }
-                }
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                const float rn = rsqrtf(ss + 1e-6f);
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
-                    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) { const float2 f = unpack2(ws[e]); ws[e] = pack2(f.x * rn, f.y * rn); }
-                    *reinterpret_cast<uint4 *>(rp + cc * 16) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
-                }
-                fence_proxy_async();
-                group_sync<1>();
-                if (t == 0) mbar_arrive_local(bars + B_CQN);
-            }
-
             // ---- U_r = U~_r - W S_r  ->  U_r^T (bf16, rows v)
-            if (!group_all<1>(wait_bar(B_WS, c & 1, false))) { fail(12); break; }
+            if (!group_all<1>(t != 0 || wait_bar(B_WS, c & 1, false))) { fail(12); break; }
             if (t == 0) CMARK(c, 9);
             tc_fence_after();
             {
@@ -393,13 +278,16 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             group_sync<1>();
             if (t == 0) { mbar_arrive_local(bars + B_U); CMARK(c, 10); }
 
-            // ---- vectors of the next chunk (its gamma_end scales the state below)
-            if (c + 1 < nch) load_vectors(c + 1);
-            const float ge_next = (c + 1 < nch) ? cvec0[((c + 1) & 1) * 320 + 192 + 63] : 1.f;
+            // ---- gamma_end of the next chunk (it scales the state below)
+            float ge_next = 1.f;
+            if (c + 1 < nch) {
+                if (!group_all<1>(t != 0 || wait_bar(B_VEC, (c + 1) & 1, false))) { fail(16); break; }
+                ge_next = cvec0[((c + 1) & 1) * 320 + 192 + 63];
+            }
 
             // ---- state: S_r^T (bf16) for the next chunk's products, D_S <- gamma_end(c+1) S_r
             if (t == 0) CMARK(c, 11);
-            if (!group_all<1>(wait_bar(B_S2, c & 1, false))) { fail(13); break; }
+            if (!group_all<1>(t != 0 || wait_bar(B_S2, c & 1, false))) { fail(13); break; }
             if (t == 0) CMARK(c, 12);
             tc_fence_after();
             {
@@ -430,8 +318,123 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             tc_fence_before();
             group_sync<1>();
             if (t == 0) { mbar_arrive_local(bars + B_ST); CMARK(c, 13); }
+        }
+    } else if (warp >= 10) {
+        // ============================================================ aux group
+        // per-chunk vectors, K~ build, Q normalisation, output epilogue (all off the chain)
+        const int t = tid - 320, qd = warp & 3, l = lane;
+        const int i_row = 16 * qd + l;                   // row of M = 64 results (l < 16)
+        const uint32_t loff = (uint32_t)(32 * qd) << 16;
+        float *cvec0 = reinterpret_cast<float *>(sm + S4_CVEC);
+        int k_issued = nch > 0 ? 1 : 0;                  // K tiles requested (the first by warp 8)
+        float pre_g = 0.f, pre_b = 0.f;
+        auto fetch_vectors = [&](int c) {                // g, beta of chunk c into registers
+            const long long t0 = t_begin + (long long)c * K4_C;
+            const int L = (int)min((long long)K4_C, t_end - t0);
+            pre_g = (t < L) ? g[(size_t)(t0 + t) * H_v + h] : 0.f;
+            pre_b = (t < L) ? beta[(size_t)(t0 + t) * H_v + h] : 0.f;
+        };
+        auto finish_vectors = [&](int c) {               // G, gamma, decay-to-end; then signal
+            float *cv = cvec0 + (c & 1) * 320;
+            float *cg = cv, *cb = cv + 64, *cG = cv + 128, *cgam = cv + 192, *cdte = cv + 256;
+            if (t < K4_C) { cg[t] = pre_g; cb[t] = pre_b; }
+            group_sync<3>();
+            if (qd == 0 && warp == 12) {
+                const float a0 = cg[2 * l], a1 = cg[2 * l + 1];
+                float sc = a0 + a1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, sc, o);
+                    if (l >= o) sc += y;
+                }
+                const float G0 = sc - a1, G1 = sc, Ge = __shfl_sync(0xffffffffu, sc, 31);
+                cG[2 * l] = G0; cG[2 * l + 1] = G1;
+                cgam[2 * l] = expf(G0); cgam[2 * l + 1] = expf(G1);
+                cdte[2 * l] = expf(Ge - G0); cdte[2 * l + 1] = expf(Ge - G1);
+            }
+            group_sync<3>();
+            if (t == 0) mbar_arrive_local(bars + B_VEC);
+        };
+        auto normalise_rows = [&](unsigned char *tile) {  // 64 rows x 128 bf16, two threads per row
+            const int row = t >> 1, half = t & 1;
+            unsigned char *rp = tile + half * 8192 + row * 128;
+            float ss = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
+                const uint32_t wsv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) { const float2 f = unpack2(wsv[e]); ss += f.x * f.x + f.y * f.y; }
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            const float rn = rsqrtf(ss + 1e-6f);
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                uint4 w = *reinterpret_cast<const uint4 *>(rp + cc * 16);
+                uint32_t wsv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) { const float2 f = unpack2(wsv[e]); wsv[e] = pack2(f.x * rn, f.y * rn); }
+                *reinterpret_cast<uint4 *>(rp + cc * 16) = make_uint4(wsv[0], wsv[1], wsv[2], wsv[3]);
+            }
+        };
+
+        if (nch > 0) {
+            if (t < K4_C) fetch_vectors(0);
+            finish_vectors(0);
+        }
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+            const long long t0 = t_begin + (long long)c * K4_C;
+            const int L = (int)min((long long)K4_C, t_end - t0);
+            const int s = c & 1;
+            const float *cv = cvec0 + s * 320;
+            const float *cgam = cv + 192, *cdte = cv + 256;
+            if (t < K4_C && c + 1 < nch) fetch_vectors(c + 1);   // lands while this chunk runs
+
+            // ---- K~(c) = diag(decay to chunk end) K; rows past the end get weight 0
+            if (!group_all<3>(t != 0 || wait_bar(B_CK, c & 1, false))) { fail(10); break; }
+            if (c >= 1 && !group_all<3>(t != 0 || wait_bar(B_S2, (c - 1) & 1, false))) { fail(17); break; }
+            if (t == 0) CMARK(c, 7);
+            if (l2norm) { normalise_rows(sm + S4_CK); group_sync<3>(); }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = t + 128 * u;
+                const int cg = e >> 9, row = (e >> 3) & 63, cc = e & 7;
+                const uint4 w = *reinterpret_cast<const uint4 *>(sm + S4_CK + cg * 8192 + row * 128 + cc * 16);
+                const float wt = row < L ? cdte[row] : 0.f;
+                const uint32_t wsv[4] = {w.x, w.y, w.z, w.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) { const float2 f = unpack2(wsv[e2]); o[e2] = pack2(f.x * wt, f.y * wt); }
+                *reinterpret_cast<uint4 *>(sm + S4_CKT + cg * 8192 + row * 128 + cc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            fence_proxy_async();
+            group_sync<3>();
+            if (t == 0) {
+                CMARK(c, 8);
+                mbar_arrive_local(bars + B_KT);
+                if (c + 1 < nch) {             // K of the next chunk into the free buffer
+                    ++k_issued;
+                    const int tn = (int)(t0 + K4_C);
+                    mbar_arrive_expect_tx(bars + B_CK, 16384);
+                    tma_load_3d(sm + S4_CK, &tm_k, bars + B_CK, 0, hq, tn);
+                    tma_load_3d(sm + S4_CK + 8192, &tm_k, bars + B_CK, 64, hq, tn);
+                }
+            }
+            if (l2norm) {                      // Q of this chunk, for Q S_r
+                if (!group_all<3>(t != 0 || wait_bar(B_CQ, c & 1, false))) { fail(11); break; }
+                normalise_rows(sm + S4_CQ);
+                fence_proxy_async();
+                group_sync<3>();
+                if (t == 0) mbar_arrive_local(bars + B_CQN);
+            }
+
+            // ---- vectors of the next chunk (the chain scales the state by its gamma_end)
+            if (c + 1 < nch) finish_vectors(c + 1);
 
             // ---- outputs: o_i = scale (gamma_i (Q S_r)_i + (P U_r)_i), columns [v0, v0 + 32)
+            if (!group_all<3>(t != 0 || wait_bar(B_PU, c & 1, false))) { fail(14); break; }
+            tc_fence_after();
             {
                 uint32_t qs[32], pu[32];
                 tmem_ld32(tmem + loff + T4_QS + 32 * s, qs);
@@ -455,7 +458,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
             }
             tc_fence_before();
-            group_sync<1>();
+            group_sync<3>();
             if (t == 0) { mbar_arrive_local(bars + (s ? B_OFREE1 : B_OFREE0)); CMARK(c, 14); }
         }
         if (*abort_flag && t == 0) drain_bar(bars + B_CK, k_issued, false);
@@ -494,7 +497,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 pgam[2 * l] = expf(G0); pgam[2 * l + 1] = expf(G1);
             }
             // ---- inputs: rows past the end zeroed, optional q/k normalisation
-            if (!group_all<2>(wait_bar(B_PKQ, k & 1, false) && wait_bar(B_PV, k & 1, false))) { fail(20); break; }
+            if (!group_all<2>(t != 0 || (wait_bar(B_PKQ, k & 1, false) && wait_bar(B_PV, k & 1, false)))) { fail(20); break; }
             if (t == 0) PMARK(k, 1);
             if (L < K4_C) {
                 const int zr = K4_C - L;
@@ -534,48 +537,43 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (t == 0) mbar_arrive_local(bars + B_PIN);
 
             // ---- the staging of the previous production must have reached every CTA
-            if (k >= 1 && !group_all<2>(wait_bar(B_SENT, (k - 1) & 1, true))) { fail(21); break; }
+            if (k >= 1 && !group_all<2>(t != 0 || wait_bar(B_SENT, (k - 1) & 1, true))) { fail(21); break; }
             if (t == 0) PMARK(k, 2);
-            if (!group_all<2>(wait_bar(B_P1, k & 1, false))) { fail(22); break; }
+            if (!group_all<2>(t != 0 || wait_bar(B_P1, k & 1, false))) { fail(22); break; }
             if (t == 0) PMARK(k, 3);
             tc_fence_after();
 
             // ---- A (fp32, rows 0..63) and P (bf16, rows 64..127) from [K;Q] K^T
             {
-                uint32_t ra[32], rb[32];
-                tmem_ld32(tmem + loff + T4_KQ, ra);
-                tmem_ld32(tmem + loff + T4_KQ + 32, rb);
-                tmem_wait_ld();
                 const bool is_a = q < 2;
                 const int i = is_a ? row : row - 64;
                 const float Gi = pG[i], wi = is_a ? pb[i] : 1.f;
-                float xv[64];
-#pragma unroll
+#pragma unroll 1
                 for (int j0 = 0; j0 < 64; j0 += 16) {
-                    float gj[16];
+                    uint32_t kr[16];
+                    tmem_ld16(tmem + loff + T4_KQ + j0, kr);
+                    float gj[16], xv[16];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const float4 g4 = *reinterpret_cast<const float4 *>(pG + j0 + 4 * u);
                         gj[4 * u] = g4.x; gj[4 * u + 1] = g4.y; gj[4 * u + 2] = g4.z; gj[4 * u + 3] = g4.w;
                     }
+                    tmem_wait_ld();
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const int j = j0 + u;
                         const float keep = (is_a ? (j < i) : (j <= i)) ? 1.f : 0.f;
-                        const float kk = __uint_as_float(j < 32 ? ra[j] : rb[j - 32]);
-                        xv[j] = (wi * keep) * __expf(fminf(Gi - gj[u], 0.f)) * kk;
+                        xv[u] = (wi * keep) * __expf(fminf(Gi - gj[u], 0.f)) * __uint_as_float(kr[u]);
                     }
-                }
-                if (is_a) {
+                    if (is_a) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) Af[i * TP4 + j] = xv[j];
-                } else {
+                        for (int u = 0; u < 16; ++u) Af[i * TP4 + j0 + u] = xv[u];
+                    } else {
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        uint4 w;
-                        w.x = pack2(xv[8 * cc + 0], xv[8 * cc + 1]); w.y = pack2(xv[8 * cc + 2], xv[8 * cc + 3]);
-                        w.z = pack2(xv[8 * cc + 4], xv[8 * cc + 5]); w.w = pack2(xv[8 * cc + 6], xv[8 * cc + 7]);
-                        *reinterpret_cast<uint4 *>(sm + S4_PSTG + sw128(i, cc)) = w;
+                        for (int h2 = 0; h2 < 2; ++h2)
+                            *reinterpret_cast<uint4 *>(sm + S4_PSTG + sw128(i, (j0 >> 3) + h2)) = make_uint4(
+                                pack2(xv[8 * h2 + 0], xv[8 * h2 + 1]), pack2(xv[8 * h2 + 2], xv[8 * h2 + 3]),
+                                pack2(xv[8 * h2 + 4], xv[8 * h2 + 5]), pack2(xv[8 * h2 + 6], xv[8 * h2 + 7]));
                     }
                 }
 #pragma unroll 4
@@ -596,18 +594,15 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             // ---- T' = T diag(beta gamma), T'' = T diag(beta) (bf16, K-major rows i)
             {
                 const int which = t >> 6, i = t & 63;
-                float tv[64];
-#pragma unroll
-                for (int j = 0; j < 64; ++j) tv[j] = Tf[i * TP4 + j];
                 unsigned char *dst = sm + (which ? S4_TPP : S4_TP);
-#pragma unroll
+#pragma unroll 2
                 for (int cc = 0; cc < 8; ++cc) {
                     float w8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = 8 * cc + e;
                         const float sc = which ? pb[j] : pb[j] * pgam[j];
-                        w8[e] = (j <= i) ? tv[j] * sc : 0.f;
+                        w8[e] = (j <= i) ? Tf[i * TP4 + j] * sc : 0.f;
                     }
                     *reinterpret_cast<uint4 *>(dst + sw128(i, cc)) =
                         make_uint4(pack2(w8[0], w8[1]), pack2(w8[2], w8[3]), pack2(w8[4], w8[5]), pack2(w8[6], w8[7]));
@@ -619,7 +614,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (t == 0) { mbar_arrive_local(bars + B_TT); PMARK(k, 6); }
 
             // ---- W and U~ (M = 64 layout) into the send staging
-            if (!group_all<2>(wait_bar(B_WU, k & 1, false))) { fail(23); break; }
+            if (!group_all<2>(t != 0 || wait_bar(B_WU, k & 1, false))) { fail(23); break; }
             if (t == 0) PMARK(k, 7);
             tc_fence_after();
             const int i = 16 * q + l;                        // valid for l < 16
@@ -660,7 +655,8 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         // ========================================================== chain issuer
         if (lane == 0) {
             // requests made by this thread, for draining after an abort
-            int q_req = 0, qs_req = 0, ws_req = 0, s2_req = 0, full_req[2] = {0, 0};
+            int q_req = 0, qs_req = 0, ws_req = 0, s2_req = 0, pu_req = 0, full_req[2] = {0, 0};
+            int sent_acked = -1;               // last chunk whose receipt was acknowledged
             if (nch > 0) {
                 q_req = 1;
                 full_req[0] = 1;
@@ -674,6 +670,8 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tma_load_3d(sm + S4_CK + 8192, &tm_k, bars + B_CK, 64, hq, tb);
                 mbar_arrive_expect_tx(bars + B_FULL0, K4_RING_BYTES);
                 if (nch > 1) mbar_arrive_expect_tx(bars + B_FULL1, K4_RING_BYTES);
+                mbar_arrive_local(bars + B_OFREE0);     // both output buffers start free
+                mbar_arrive_local(bars + B_OFREE1);
             }
             const uint32_t id_m64 = idesc_bf16(64, 32, false, false);
             const uint32_t id_s2 = idesc_bf16(128, 32, true, false);
@@ -700,8 +698,13 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     ++ws_req;
                 }
                 CMARK(c, 2);
-                mbar_arrive_remote_relaxed(map_to_rank(bars + B_SENT, (uint32_t)(c & 3)));
-                // Q S_r feeds only the outputs
+                if (sent_acked < c) {
+                    mbar_arrive_remote_relaxed(map_to_rank(bars + B_SENT, (uint32_t)(c & 3)));
+                    sent_acked = c;
+                }
+                // Q S_r (outputs only) reads the same S_r^T, so it must be issued before S2
+                // (the state epilogue rewrites S_r^T once S2's commit completes); it runs
+                // while the U epilogue works, ahead of S2 in the pipe
                 if (!wait_bar(l2norm ? B_CQN : B_CQ, c & 1, false)) { fail(30); break; }
                 if (!wait_bar(s ? B_OFREE1 : B_OFREE0, (c >> 1) & 1, false)) { fail(32); break; }
                 tc_fence_after();
@@ -716,20 +719,22 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     umma_commit(bars + B_QS);
                     ++qs_req;
                 }
-                CMARK(c, 3);
                 if (!wait_bar(B_U, c & 1, false)) { fail(35); break; }
                 if (!wait_bar(B_KT, c & 1, false)) { fail(36); break; }
+                CMARK(c, 3);
                 tc_fence_after();
-                {   // S_r += K~^T U_r ; P U_r -> D_PU[s]
+                {   // S_r += K~^T U_r (on the chain) ; P U_r -> D_PU[s]
                     const uint32_t kt = smem_u32(sm + S4_CKT);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         umma_bf16(tmem + T4_S, sdesc_mnmajor(kt + ks * 2048, 8192), sdesc_kmajor(ut + ks * 32), id_s2, 1);
+                    umma_commit(bars + B_S2);
+                    ++s2_req;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         umma_bf16(tmem + T4_PU + 32 * s, sdesc_kmajor(ring_s + 16384 + ks * 32), sdesc_kmajor(ut + ks * 32), id_m64, ks > 0);
-                    umma_commit(bars + B_S2);
-                    ++s2_req;
+                    umma_commit(bars + B_PU);
+                    ++pu_req;
                 }
                 CMARK(c, 4);
                 // Q of the next chunk into the buffer Q S_r has finished reading
@@ -741,7 +746,21 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tn);
                     tma_load_3d(sm + S4_CQ + 8192, &tm_q, bars + B_CQ, 64, hq, tn);
                 }
-                if (!wait_bar(B_S2, c & 1, false)) { fail(37); break; }
+                {   // wait for S2; meanwhile acknowledge the next chunk's data as soon as it lands
+                    bool ok = false;
+                    const int cn = c + 1;
+                    for (uint32_t it = 0; it < budget; ++it) {
+                        if (cn < nch && sent_acked < cn &&
+                            mbar_try_wait_cluster(bars + ((cn & 1) ? B_FULL1 : B_FULL0), (uint32_t)((cn >> 1) & 1))) {
+                            mbar_arrive_remote_relaxed(map_to_rank(bars + B_SENT, (uint32_t)(cn & 3)));
+                            sent_acked = cn;
+                        }
+                        if (mbar_try_wait(bars + B_S2, (uint32_t)(c & 1))) { ok = true; break; }
+                        if (*abort_flag) break;
+                    }
+                    if (!ok) { fail(37); break; }
+                }
+                if (!wait_bar(B_PU, c & 1, false)) { fail(38); break; }
                 CMARK(c, 5);
                 if (c + 2 < nch) {             // slot s is free for chunk c + 2
                     ++full_req[s];
@@ -756,6 +775,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 drain_bar(bars + B_QS, qs_req, false);
                 drain_bar(bars + B_WS, ws_req, false);
                 drain_bar(bars + B_S2, s2_req, false);
+                drain_bar(bars + B_PU, pu_req, false);
                 // a producer that sent anything has done so long ago; one that aborted first
                 // never will, so these two waits are kept short
                 drain_bar(bars + B_FULL0, full_req[0], true, 1u << 16);
