@@ -345,7 +345,7 @@ def run_ours(args):
     flops = prefill_flops_per_token_head(wp.dk, wp.dv) * tok * wp.H_v
     pf_tflops = flops / (ms_prefill * 1e-3) / 1e12
     pf_bytes = prefill_bytes(wp)
-    tc_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "prefill_tc.cu")
+    tc_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "prefill_tc_cluster.cu")
     dec_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode.cu")
     ms_dec_step = ms_decode_pass / wd.decode_steps
     dec_bytes = decode_bytes_per_step(wd)

@@ -20,12 +20,16 @@
 // bulk DSMEM copies that complete on the receivers' mbarriers.  Each CTA therefore
 // prepares every fourth chunk, several chunks ahead of the state chain.
 //
-// Roles inside a CTA (320 threads):
-//   warps 0-3  chain group:  K~ build, U epilogue, state epilogue, output epilogue
-//   warps 4-7  prep group:   inputs fix-up, A/P epilogue, triangular inverse, T'/T'',
-//                            W/U~ epilogue into the send staging
-//   warp 8     chain issuer: TMA for Q, MMAs QS, WS, S2 (K~^T U), PU, ring bookkeeping
-//   warp 9     prep issuer:  TMA for the prepared chunk, MMAs P1 ([K;Q]K^T), W, U~, sends
+// Roles inside a CTA (448 threads):
+//   warps 0-3    chain group:  U epilogue and state epilogue; its first thread issues
+//                              the chain's MMAs WS = W S_r and S2 = K~^T U_r; thread 32
+//                              issues PU = P U_r
+//   warps 4-7    prep group:   inputs fix-up, A/P epilogue, triangular inverse, T'/T'',
+//                              W/U~ epilogue into the send staging
+//   warp 8       chain issuer: TMA for Q, MMA QS = Q S_r (queued behind WS), ring
+//                              bookkeeping
+//   warp 9       prep issuer:  TMA for the prepared chunk, MMAs P1 ([K;Q]K^T), W, U~, sends
+//   warps 10-13  aux group:    per-chunk vectors, K~ build, output epilogue
 // Accumulators live in TMEM; the state slice S_r (128 x 32 fp32) stays in TMEM for the
 // whole sequence.  Every wait is bounded; a CTA whose wait runs out records
 // GDN_ERR_TIMEOUT, raises its abort flag so its other roles stop, drains its own
@@ -49,6 +53,13 @@ constexpr int K4_SL = 32;                // value columns per CTA
 constexpr int K4_THREADS = 448;
 constexpr uint32_t K4_DEFAULT_BUDGET = 1u << 22;
 constexpr uint32_t K4_RING_BYTES = 28672;    // W 16 KB + P 8 KB + U~ slice 4 KB
+// Prepared chunks travel through L2: the producer writes W, P and all four U~ slices of a
+// chunk into one 40 KB global chunk slot (already in the shared-memory tile layout), and
+// each consumer bulk-loads W, P and its own slice into its ring.  A cluster owns 8 chunk
+// slots (chunk p uses slot p mod 8), taken from a library-held pool.
+constexpr uint32_t K4_GCHUNK = 40960;        // W 16 KB | P 8 KB | U~ 4 x 4 KB
+constexpr uint32_t K4_GCLUSTER = 8 * K4_GCHUNK;
+constexpr int K4_POOL = 64;                  // cluster slots (more than can be resident)
 
 // TMEM columns (512 allocated)
 constexpr uint32_t T4_S = 0;       // 32: S_r (lane = key dim d, col = value v)
@@ -63,30 +74,36 @@ constexpr uint32_t T4_U = 384;     // 128: T'' V    (M = 64 layout)
 constexpr uint32_t S4_CQ = 0;          // 16 KB Q of the chain's chunk [cg0 | cg1]
 constexpr uint32_t S4_CK = 16384;      // 16 KB K of the chain's chunk
 constexpr uint32_t S4_CKT = 32768;     // 16 KB K~
-constexpr uint32_t S4_ST = 49152;      // 8 KB S_r^T bf16, rows v (K-major B), [cg0 | cg1] 4 KB each
-constexpr uint32_t S4_UT = 57344;      // 4 KB U_r^T bf16, rows v (K-major B)
+constexpr uint32_t S4_ST = 49152;      // 8 KB S_r bf16, rows d of 64 B (MN-major B, 64-byte swizzle)
+constexpr uint32_t S4_UT = 57344;      // 4 KB U_r bf16, rows i of 64 B (MN-major B, 64-byte swizzle)
 constexpr uint32_t S4_RING = 61440;    // 2 slots x 28 KB: W (16 KB) | P (8 KB) | U~_r (4 KB)
 constexpr uint32_t S4_PKQ = 118784;    // 32 KB [K cg0 | Q cg0 | K cg1 | Q cg1] of the prepared chunk
 constexpr uint32_t S4_PV = 151552;     // 16 KB V of the prepared chunk
 constexpr uint32_t S4_TP = 167936;     // 8 KB T' = T diag(beta gamma)
 constexpr uint32_t S4_TPP = 176128;    // 8 KB T'' = T diag(beta)
-constexpr uint32_t S4_PSTG = 184320;   // 8 KB P staging (send source)
+constexpr uint32_t S4_PSTG = 184320;   // 8 KB P staging (store source)
 constexpr uint32_t S4_AF = 192512;     // fp32 A 64 x 65 (overlaid later by the W staging)
 constexpr uint32_t S4_TF = 209152;     // fp32 T 64 x 65 (overlaid later by the U~ staging)
 constexpr uint32_t S4_WSTG = 192512;   // 16 KB W staging
 constexpr uint32_t S4_USTG = 208896;   // 16 KB U~ staging, 4 slices x [64 rows x 32 v]
 constexpr uint32_t S4_CVEC = 225792;   // chain vectors, 2 buffers x {g, beta, G, gamma, dte} x 64
-constexpr uint32_t S4_PVEC = 228352;   // prep vectors {g, beta, G, gamma} x 64
-constexpr uint32_t S4_BAR = 229376;    // mbarriers
-constexpr uint32_t S4_MISC = S4_BAR + 32 * 8;   // tmem base, abort flag
+constexpr uint32_t S4_PVEC = 228352;   // prep vectors {g, beta, G, gamma, exp(-G)} x 64
+constexpr uint32_t S4_BAR = 229632;    // mbarriers
+constexpr uint32_t S4_MISC = S4_BAR + 48 * 8;   // tmem base, abort flag, cluster's ring slot
 constexpr uint32_t S4_END = S4_MISC + 16;
 constexpr uint32_t K4_SMEM = S4_END + 1024;
 constexpr int TP4 = 65;
 
 enum Bar {
-    B_CQ = 0, B_CK, B_FULL0, B_FULL1, B_QS, B_WS, B_S2, B_KT, B_U, B_ST, B_OFREE0, B_OFREE1,
-    B_PKQ, B_PV, B_P1, B_TT, B_WU, B_STG, B_EMPTY, B_SENT, B_PIN, B_CQN, B_VEC, B_PU, B_COUNT
+    B_CQ = 0, B_CK, B_FULL0, B_FULL1, B_QS, B_WS, B_S2, B_KT, B_OFREE0, B_OFREE1,
+    B_PKQ, B_PV, B_P1, B_TT, B_WU, B_PIN, B_CQN, B_VEC0, B_VEC1, B_PU0, B_PU1, B_WSI,
+    B_STG,                                 // producer: staging written
+    B_SFREE,                               // producer: staging read by the bulk stores
+    B_GFREE0, B_GFREE1,                    // producer: all four CTAs loaded its chunk slot
+    B_READY,                               // consumer: chunk p's slot written (8: p mod 8)
+    B_COUNT = B_READY + 8
 };
+static_assert(B_COUNT <= 48, "barrier area holds 48");
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -111,9 +128,15 @@ __device__ __forceinline__ bool group_all(bool v) {
         : "=r"(r) : "r"(v ? 1u : 0u), "n"(ID) : "memory");
     return r != 0;
 }
-// element (row r, column c) of a 128-byte-swizzled tile whose rows hold 64 bf16
-__device__ __forceinline__ void store_bf16_at(unsigned char *tile, int r, int c, float x) {
-    *reinterpret_cast<__nv_bfloat16 *>(tile + sw128(r, c >> 3) + (c & 7) * 2) = __float2bfloat16_rn(x);
+// row r (32 fp32 values, bit patterns) of a 64-byte-swizzled bf16 tile
+__device__ __forceinline__ void store_row32(unsigned char *tile, int r, const uint32_t (&x)[32]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4 *>(tile + sw64(r, c)) = make_uint4(
+            pack2(__uint_as_float(x[8 * c]), __uint_as_float(x[8 * c + 1])),
+            pack2(__uint_as_float(x[8 * c + 2]), __uint_as_float(x[8 * c + 3])),
+            pack2(__uint_as_float(x[8 * c + 4]), __uint_as_float(x[8 * c + 5])),
+            pack2(__uint_as_float(x[8 * c + 6]), __uint_as_float(x[8 * c + 7])));
 }
 // wait for the last of `issued` phases of `bar` (phases complete in order); used only
 // while draining after an abort, so it ignores the abort flag
@@ -127,23 +150,49 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, int issued, bool cluste
 
 }  // namespace
 
+// Library-held L2 ring for prepared chunks (see K4_GCHUNK) and the pool of its cluster
+// slots: a cluster claims a free slot when it starts and returns it when it ends.
+static __device__ __align__(1024) unsigned char g4_ring[(size_t)K4_POOL * K4_GCLUSTER];
+static __device__ int g4_pool[K4_POOL];
+
 // Profiling aid, compiled in only with -DGDN_PHASE_TIMERS: CTA (0, 0) records clock64()
 // at fixed points of its chain (per chunk) and of its preparations (per production).
 #ifdef GDN_PHASE_TIMERS
-__device__ unsigned long long g4_chain[64][16];
+__device__ unsigned long long g4_chain[64][32];
 __device__ unsigned long long g4_prep[16][16];
+__device__ unsigned long long g4_span[1024][2];      // per CTA: globaltimer at start and end
+#define SPAN(k) do { const unsigned idx_ = blockIdx.y * gridDim.x + blockIdx.x; if (threadIdx.x == 0 && idx_ < 1024) { \
+    unsigned long long gt_; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt_)); g4_span[idx_][(k)] = gt_; } } while (0)
 #define CMARK(c, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (c) < 64) g4_chain[(c)][(k)] = clock64(); } while (0)
 #define PMARK(kk, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (kk) < 16) g4_prep[(kk)][(k)] = clock64(); } while (0)
-extern "C" __attribute__((visibility("default"))) int gdn_debug_cluster_timeline(void *chain, void *prep)
+#define GMARK(c, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (c) < 64) { unsigned long long gt_; \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt_)); g4_chain[(c)][(k)] = gt_; } } while (0)
+extern "C" __attribute__((visibility("default"))) int gdn_debug_cluster_timeline(void *chain, void *prep, void *span)
 {
     if (cudaMemcpyFromSymbol(chain, g4_chain, sizeof(g4_chain)) != cudaSuccess) return 1;
+    if (cudaMemcpyFromSymbol(span, g4_span, sizeof(g4_span)) != cudaSuccess) return 1;
     return (int)cudaMemcpyFromSymbol(prep, g4_prep, sizeof(g4_prep));
 }
 #else
 #define CMARK(c, k) do { } while (0)
 #define PMARK(kk, k) do { } while (0)
+#define GMARK(c, k) do { } while (0)
+#define SPAN(k) do { } while (0)
 #endif
 
+// Cold path, kept out of line so its code is not repeated at every wait: the first role
+// of a CTA whose wait runs out records the error and raises the CTA's abort flag.
+__device__ __noinline__ void raise_abort(volatile int *abort_flag, DeviceError *err, int where)
+{
+    if (!*abort_flag) {
+        *abort_flag = 1;
+        record_error(err, GDN_ERR_TIMEOUT, where);
+    }
+}
+
+// L2N: q and k are L2-normalised in the kernel (a separate instantiation, so the common
+// case carries none of that code)
+template <bool L2N>
 __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(K4_THREADS, 1)
 prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -151,12 +200,13 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const float *__restrict__ beta, const float *S0,
                           __nv_bfloat16 *__restrict__ out, float *S_final,
                           const int32_t *__restrict__ cu_seqlens, long long T_dense, int H_qk,
-                          int H_v, float scale, int l2norm, DeviceError *err, uint32_t budget)
+                          int H_v, float scale, DeviceError *err, uint32_t budget)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    SPAN(0);
     const uint32_t r = cluster_rank();
     const int n = blockIdx.x >> 2, h = blockIdx.y;
     const int hq = h / (H_v / H_qk);
@@ -173,14 +223,26 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 
     if (warp == 8) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
     if (tid == 256) {
-        for (int b = 0; b < B_COUNT; ++b) mbar_init(bars + b, (b == B_EMPTY || b == B_SENT) ? 4 : 1);
+        for (int b = 0; b < B_COUNT; ++b) mbar_init(bars + b, (b == B_GFREE0 || b == B_GFREE1) ? 4 : 1);
         *abort_flag = 0;
         fence_mbar_init();
+        if (r == 0) {                          // claim a ring slot for the cluster
+            int slot = -1;
+            for (int round = 0; round < 4096 && slot < 0; ++round) {
+                for (int i = 0; i < K4_POOL && slot < 0; ++i)
+                    if (atomicCAS(&g4_pool[i], 0, 1) == 0) slot = i;
+                if (slot < 0) __nanosleep(1000);
+            }
+            *reinterpret_cast<volatile int *>(sm + S4_MISC + 8) = slot;
+        }
     }
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int ring_slot = (int)ld_cluster_u32(map_to_rank(sm + S4_MISC + 8, 0));
+    unsigned char *gring = g4_ring + (size_t)(ring_slot < 0 ? 0 : ring_slot) * K4_GCLUSTER;
+    if (ring_slot < 0 && tid == 0) record_error(err, GDN_ERR_TIMEOUT, 90);
 
     // bounded wait; gives up early if another role of this CTA has aborted
     auto wait_bar = [&](int b, uint32_t parity, bool cluster_scope) -> bool {
@@ -191,25 +253,48 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         return false;
     };
-    auto fail = [&](int where) {
-        if (!*abort_flag) {
-            *abort_flag = 1;
-            record_error(err, GDN_ERR_TIMEOUT, where);
-        }
-    };
+    auto fail = [&](int where) { raise_abort(abort_flag, err, where); };
 
-    if (warp < 4) {
+    if (ring_slot < 0) {
+        // no ring slot could be claimed: the error is recorded, nothing else runs
+    } else if (warp < 4) {
         // =========================================================== chain group
-        // U and state epilogues only: the two CUDA-core steps on the state chain
+        // The two CUDA-core steps of the state chain (U epilogue, state epilogue).  The
+        // group's first thread also issues the chain's MMAs itself (W S_r, then K~^T U_r
+        // with P U_r behind it), so no hand-off to another warp sits on the chain.
         const int t = tid, q = warp, l = lane;
         const int d = 32 * q + l;                        // TMEM lane = key dim of S_r
         const int i_row = 16 * q + l;                    // row of M = 64 results (l < 16)
         const uint32_t loff = (uint32_t)(32 * q) << 16;
         const float *cvec0 = reinterpret_cast<const float *>(sm + S4_CVEC);
         const unsigned char *ring = sm + S4_RING;
+        const uint32_t st = smem_u32(sm + S4_ST), ut = smem_u32(sm + S4_UT), kt = smem_u32(sm + S4_CKT);
+        const uint32_t id_m64 = idesc_bf16(64, 32, false, true);     // B = S_r or U_r rows
+        const uint32_t id_s2 = idesc_bf16(128, 32, true, true);
+        int ws_req = 0, s2_req = 0, pu_req0 = 0, pu_req1 = 0;    // MMA groups issued
         bool ok = true;
+        // descriptors step by a fixed amount per 16-deep K slice (the address field is in
+        // 16-byte units): K-major SW128 +32 B, 64-byte-row MN-major +1024 B, SW128
+        // MN-major +2048 B; the second 64-wide K block of a K-major tile is +8192 B
 
-        // initial state slice: D_S = gamma_end(0) S0_r, S_r^T (bf16) = S0_r
+        // W S_r for chunk cc once its ring slot has arrived (thread 0 only).  B_WSI tells
+        // the issuer warp, which then queues Q S_r behind it.
+        auto issue_ws = [&](int cc) -> bool {
+            const int sc = cc & 1;
+            if (!wait_bar(sc ? B_FULL1 : B_FULL0, (cc >> 1) & 1, false)) return false;
+            tc_fence_after();
+            const uint64_t d_w = sdesc_kmajor(smem_u32(sm + S4_RING + sc * K4_RING_BYTES));
+            const uint64_t d_st = sdesc_mn_sw64(st);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_bf16(tmem + T4_WS, d_w + (ks >> 2) * 512 + (ks & 3) * 2, d_st + ks * 64, id_m64, ks > 0);
+            umma_commit(bars + B_WS);
+            mbar_arrive_local(bars + B_WSI);
+            ++ws_req;
+            return true;
+        };
+
+        // initial state slice: D_S = gamma_end(0) S0_r, S_r (bf16) = S0_r
         float x[32];
         {
             const float *src = S0 ? S0 + s_off + (size_t)d * K4_D + v0 : nullptr;
@@ -225,30 +310,37 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                 for (int v = 0; v < 32; v += 4) *reinterpret_cast<float4 *>(dst + v) = make_float4(x[v], x[v + 1], x[v + 2], x[v + 3]);
             }
-        } else if (!group_all<1>(t != 0 || wait_bar(B_VEC, 0, false))) {
+        } else if (!group_all<1>(t != 0 || wait_bar(B_VEC0, 0, false))) {
             fail(15);
             ok = false;
         } else {
             const float ge0 = cvec0[192 + 63];
             uint32_t rr[32];
 #pragma unroll
-            for (int v = 0; v < 32; ++v) {
-                store_bf16_at(sm + S4_ST + (d >> 6) * 4096, v, d & 63, x[v]);
-                rr[v] = __float_as_uint(ge0 * x[v]);
-            }
+            for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(x[v]);
+            store_row32(sm + S4_ST, d, rr);
+#pragma unroll
+            for (int v = 0; v < 32; ++v) rr[v] = __float_as_uint(ge0 * x[v]);
             tmem_st32(tmem + loff + T4_S, rr);
             tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             group_sync<1>();
-            if (t == 0) mbar_arrive_local(bars + B_ST);
+            bool okw = true;
+            if (t == 0) okw = issue_ws(0);
+            if (!group_all<1>(okw)) { fail(31); ok = false; }
         }
 
 #pragma unroll 1
         for (int c = 0; ok && c < nch; ++c) {
             const int s = c & 1;
-            // ---- U_r = U~_r - W S_r  ->  U_r^T (bf16, rows v)
-            if (!group_all<1>(t != 0 || wait_bar(B_WS, c & 1, false))) { fail(12); break; }
+            // ---- U_r = U~_r - W S_r  ->  U_r (bf16, rows i).  The previous chunk's P U_r
+            // (issued by thread 32, so not covered by thread 0's commits) read U_r too.
+            if (!group_all<1>(t != 0 || (wait_bar(B_WS, c & 1, false) &&
+                                         (c == 0 || wait_bar((c & 1) ? B_PU0 : B_PU1, ((c - 1) >> 1) & 1, false))))) {
+                fail(12);
+                break;
+            }
             if (t == 0) CMARK(c, 9);
             tc_fence_after();
             {
@@ -257,7 +349,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_wait_ld();
                 if (l < 16) {
                     const unsigned char *us = ring + s * K4_RING_BYTES + 24576 + i_row * 64;
-                    float uu[32];
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {
                         const uint4 w = *reinterpret_cast<const uint4 *>(us + cc * 16);
@@ -265,59 +356,95 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 f = unpack2(wv[e]);
-                            uu[8 * cc + 2 * e] = f.x; uu[8 * cc + 2 * e + 1] = f.y;
+                            ws[8 * cc + 2 * e] = __float_as_uint(f.x - __uint_as_float(ws[8 * cc + 2 * e]));
+                            ws[8 * cc + 2 * e + 1] = __float_as_uint(f.y - __uint_as_float(ws[8 * cc + 2 * e + 1]));
                         }
                     }
-#pragma unroll
-                    for (int v = 0; v < 32; ++v)
-                        store_bf16_at(sm + S4_UT, v, i_row, uu[v] - __uint_as_float(ws[v]));
+                    store_row32(sm + S4_UT, i_row, ws);
                 }
             }
             fence_proxy_async();
             tc_fence_before();
             group_sync<1>();
-            if (t == 0) { mbar_arrive_local(bars + B_U); CMARK(c, 10); }
+            if (t == 0) CMARK(c, 10);
 
-            // ---- gamma_end of the next chunk (it scales the state below)
-            float ge_next = 1.f;
-            if (c + 1 < nch) {
-                if (!group_all<1>(t != 0 || wait_bar(B_VEC, (c + 1) & 1, false))) { fail(16); break; }
-                ge_next = cvec0[((c + 1) & 1) * 320 + 192 + 63];
+            // ---- S_r += K~^T U_r on the chain (thread 0) and P U_r -> D_PU[s] beside it
+            // (thread 32).  gamma_end of the next chunk is waited for before S2, so this
+            // group can never be lapped by the group that signals it.
+            {
+                bool oks = true;
+                if (t == 0) {
+                    oks = wait_bar(B_KT, c & 1, false) &&
+                          (c + 1 >= nch || wait_bar(((c + 1) & 1) ? B_VEC1 : B_VEC0, ((c + 1) >> 1) & 1, false));
+                    if (oks) {
+                        tc_fence_after();
+                        const uint64_t d_kt = sdesc_mnmajor(kt, 8192), d_ut = sdesc_mn_sw64(ut);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            umma_bf16(tmem + T4_S, d_kt + ks * 128, d_ut + ks * 64, id_s2, 1);
+                        umma_commit(bars + B_S2);
+                        ++s2_req;
+                        CMARK(c, 22);
+                    }
+                } else if (t == 32) {
+                    oks = wait_bar(s ? B_OFREE1 : B_OFREE0, (c >> 1) & 1, false);
+                    if (oks) {
+                        tc_fence_after();
+                        const uint64_t d_p = sdesc_kmajor(smem_u32(sm + S4_RING + s * K4_RING_BYTES + 16384));
+                        const uint64_t d_ut = sdesc_mn_sw64(ut);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            umma_bf16(tmem + T4_PU + 32 * s, d_p + ks * 2, d_ut + ks * 64, id_m64, ks > 0);
+                        umma_commit(bars + (s ? B_PU1 : B_PU0));
+                        if (s) ++pu_req1; else ++pu_req0;
+                    }
+                }
+                if (!group_all<1>(oks)) { fail(13); break; }
             }
+            const float ge_next = (c + 1 < nch) ? cvec0[((c + 1) & 1) * 320 + 192 + 63] : 1.f;
 
-            // ---- state: S_r^T (bf16) for the next chunk's products, D_S <- gamma_end(c+1) S_r
-            if (t == 0) CMARK(c, 11);
-            if (!group_all<1>(t != 0 || wait_bar(B_S2, c & 1, false))) { fail(13); break; }
+            // ---- state: S_r (bf16) for the next chunk's products first (that is what the
+            // next W S_r waits for), then D_S <- gamma_end(c+1) S_r (needed only by the next S2)
+            if (!group_all<1>(t != 0 || wait_bar(B_S2, c & 1, false))) { fail(14); break; }
             if (t == 0) CMARK(c, 12);
             tc_fence_after();
-            {
-                uint32_t rs[32];
-                tmem_ld32(tmem + loff + T4_S, rs);
-                tmem_wait_ld();
-                if (c + 1 == nch) {
-                    if (S_final) {
-                        float *dst = S_final + s_off + (size_t)d * K4_D + v0;
+            uint32_t rs[32];
+            tmem_ld32(tmem + loff + T4_S, rs);
+            tmem_wait_ld();
+            if (c + 1 == nch) {
+                if (S_final) {
+                    float *dst = S_final + s_off + (size_t)d * K4_D + v0;
 #pragma unroll
-                        for (int v = 0; v < 32; v += 4)
-                            *reinterpret_cast<float4 *>(dst + v) = make_float4(
-                                __uint_as_float(rs[v]), __uint_as_float(rs[v + 1]),
-                                __uint_as_float(rs[v + 2]), __uint_as_float(rs[v + 3]));
-                    }
-                } else {
-#pragma unroll
-                    for (int v = 0; v < 32; ++v) {
-                        const float xv = __uint_as_float(rs[v]);
-                        store_bf16_at(sm + S4_ST + (d >> 6) * 4096, v, d & 63, xv);
-                        rs[v] = __float_as_uint(ge_next * xv);
-                    }
-                    tmem_st32(tmem + loff + T4_S, rs);
-                    tmem_wait_st();
+                    for (int v = 0; v < 32; v += 4)
+                        *reinterpret_cast<float4 *>(dst + v) = make_float4(
+                            __uint_as_float(rs[v]), __uint_as_float(rs[v + 1]),
+                            __uint_as_float(rs[v + 2]), __uint_as_float(rs[v + 3]));
                 }
+                break;
             }
+            // Q S_r of this chunk reads the tile about to be replaced
+            if (!group_all<1>(t != 0 || wait_bar(B_QS, c & 1, false))) { fail(17); break; }
+            store_row32(sm + S4_ST, d, rs);
             fence_proxy_async();
-            tc_fence_before();
             group_sync<1>();
-            if (t == 0) { mbar_arrive_local(bars + B_ST); CMARK(c, 13); }
+            bool okw = true;
+            if (t == 0) { CMARK(c, 13); okw = issue_ws(c + 1); }
+#pragma unroll
+            for (int v = 0; v < 32; ++v) rs[v] = __float_as_uint(ge_next * __uint_as_float(rs[v]));
+            tmem_st32(tmem + loff + T4_S, rs);
+            tmem_wait_st();
+            tc_fence_before();
+            if (!group_all<1>(okw)) { fail(18); break; }
+            if (t == 0) CMARK(c, 15);
+        }
+        if (*abort_flag) {
+            if (t == 0) {
+                drain_bar(bars + B_WS, ws_req, false);
+                drain_bar(bars + B_S2, s2_req, false);
+            } else if (t == 32) {
+                drain_bar(bars + B_PU0, pu_req0, false);
+                drain_bar(bars + B_PU1, pu_req1, false);
+            }
         }
     } else if (warp >= 10) {
         // ============================================================ aux group
@@ -353,7 +480,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 cdte[2 * l] = expf(Ge - G0); cdte[2 * l + 1] = expf(Ge - G1);
             }
             group_sync<3>();
-            if (t == 0) mbar_arrive_local(bars + B_VEC);
+            if (t == 0) mbar_arrive_local(bars + ((c & 1) ? B_VEC1 : B_VEC0));
         };
         auto normalise_rows = [&](unsigned char *tile) {  // 64 rows x 128 bf16, two threads per row
             const int row = t >> 1, half = t & 1;
@@ -395,8 +522,8 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (!group_all<3>(t != 0 || wait_bar(B_CK, c & 1, false))) { fail(10); break; }
             if (c >= 1 && !group_all<3>(t != 0 || wait_bar(B_S2, (c - 1) & 1, false))) { fail(17); break; }
             if (t == 0) CMARK(c, 7);
-            if (l2norm) { normalise_rows(sm + S4_CK); group_sync<3>(); }
-#pragma unroll
+            if constexpr (L2N) { normalise_rows(sm + S4_CK); group_sync<3>(); }
+#pragma unroll 2
             for (int u = 0; u < 8; ++u) {
                 const int e = t + 128 * u;
                 const int cg = e >> 9, row = (e >> 3) & 63, cc = e & 7;
@@ -421,7 +548,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tma_load_3d(sm + S4_CK + 8192, &tm_k, bars + B_CK, 64, hq, tn);
                 }
             }
-            if (l2norm) {                      // Q of this chunk, for Q S_r
+            if constexpr (L2N) {               // Q of this chunk, for Q S_r
                 if (!group_all<3>(t != 0 || wait_bar(B_CQ, c & 1, false))) { fail(11); break; }
                 normalise_rows(sm + S4_CQ);
                 fence_proxy_async();
@@ -433,7 +560,8 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (c + 1 < nch) finish_vectors(c + 1);
 
             // ---- outputs: o_i = scale (gamma_i (Q S_r)_i + (P U_r)_i), columns [v0, v0 + 32)
-            if (!group_all<3>(t != 0 || wait_bar(B_PU, c & 1, false))) { fail(14); break; }
+            if (!group_all<3>(t != 0 || (wait_bar(B_QS, c & 1, false) &&
+                                         wait_bar(s ? B_PU1 : B_PU0, (c >> 1) & 1, false)))) { fail(19); break; }
             tc_fence_after();
             {
                 uint32_t qs[32], pu[32];
@@ -468,10 +596,19 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int row = 32 * q + l;                        // TMEM lane
         const uint32_t loff = (uint32_t)(32 * q) << 16;
         float *pg = reinterpret_cast<float *>(sm + S4_PVEC);
-        float *pb = pg + 64, *pG = pg + 128, *pgam = pg + 192;
+        float *pb = pg + 64, *pG = pg + 128, *pgam = pg + 192, *pinv = pg + 256;
         float *Af = reinterpret_cast<float *>(sm + S4_AF);
         float *Tf = reinterpret_cast<float *>(sm + S4_TF);
 
+        // g and beta of production k's chunk, loaded into registers one production ahead
+        float nxt_g = 0.f, nxt_b = 0.f;
+        auto fetch_gb = [&](int pp) {
+            const long long tt = t_begin + (long long)pp * K4_C;
+            const int LL = (int)min((long long)K4_C, t_end - tt);
+            nxt_g = (t < LL) ? g[(size_t)(tt + t) * H_v + h] : 0.f;
+            nxt_b = (t < LL) ? beta[(size_t)(tt + t) * H_v + h] : 0.f;
+        };
+        if ((int)r < nch && t < K4_C) fetch_gb((int)r);
 #pragma unroll 1
         for (int k = 0;; ++k) {
             const int p = (int)r + 4 * k;
@@ -479,11 +616,9 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             const long long t0 = t_begin + (long long)p * K4_C;
             const int L = (int)min((long long)K4_C, t_end - t0);
             if (t == 0) PMARK(k, 0);
-            if (t < K4_C) {
-                pg[t] = t < L ? g[(size_t)(t0 + t) * H_v + h] : 0.f;
-                pb[t] = t < L ? beta[(size_t)(t0 + t) * H_v + h] : 0.f;
-            }
+            if (t < K4_C) { pg[t] = nxt_g; pb[t] = nxt_b; }
             group_sync<2>();
+            if (t == 0) PMARK(k, 10);
             if (q == 0) {
                 const float a0 = pg[2 * l], a1 = pg[2 * l + 1];
                 float s = a0 + a1;
@@ -495,8 +630,10 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const float G0 = s - a1, G1 = s;
                 pG[2 * l] = G0; pG[2 * l + 1] = G1;
                 pgam[2 * l] = expf(G0); pgam[2 * l + 1] = expf(G1);
+                pinv[2 * l] = expf(-G0); pinv[2 * l + 1] = expf(-G1);
             }
             // ---- inputs: rows past the end zeroed, optional q/k normalisation
+            if (t == 0) PMARK(k, 11);
             if (!group_all<2>(t != 0 || (wait_bar(B_PKQ, k & 1, false) && wait_bar(B_PV, k & 1, false)))) { fail(20); break; }
             if (t == 0) PMARK(k, 1);
             if (L < K4_C) {
@@ -508,7 +645,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 group_sync<2>();
             }
-            if (l2norm) {                  // thread t: row t of [K;Q] (both 128-byte halves)
+            if constexpr (L2N) {           // thread t: row t of [K;Q] (both 128-byte halves)
                 unsigned char *r0 = sm + S4_PKQ + (t >= 64 ? 8192 : 0) + (t & 63) * 128;
                 float ss = 0.f;
 #pragma unroll
@@ -536,8 +673,9 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             group_sync<2>();
             if (t == 0) mbar_arrive_local(bars + B_PIN);
 
-            // ---- the staging of the previous production must have reached every CTA
-            if (k >= 1 && !group_all<2>(t != 0 || wait_bar(B_SENT, (k - 1) & 1, true))) { fail(21); break; }
+            // ---- the previous production's staging (overlaying A, T and P) has been read by
+            // its bulk stores
+            if (k >= 1 && !group_all<2>(t != 0 || wait_bar(B_SFREE, (k - 1) & 1, false))) { fail(21); break; }
             if (t == 0) PMARK(k, 2);
             if (!group_all<2>(t != 0 || wait_bar(B_P1, k & 1, false))) { fail(22); break; }
             if (t == 0) PMARK(k, 3);
@@ -548,22 +686,45 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const bool is_a = q < 2;
                 const int i = is_a ? row : row - 64;
                 const float Gi = pG[i], wi = is_a ? pb[i] : 1.f;
+                // exp(G_i - G_j) = exp(G_i) exp(-G_j) is exact enough and in range while the
+                // chunk's total log-decay stays above -80 (the usual case, uniform across
+                // the CTA); otherwise each factor is exponentiated from the clamped difference
+                const bool factored = pG[63] > -80.f;
+                const float wi_e = wi * pgam[i];
+                const int jend = 32 * ((q & 1) + 1);         // columns past this are masked for the warp
 #pragma unroll 1
                 for (int j0 = 0; j0 < 64; j0 += 16) {
-                    uint32_t kr[16];
-                    tmem_ld16(tmem + loff + T4_KQ + j0, kr);
-                    float gj[16], xv[16];
+                    float xv[16];
+                    if (j0 >= jend) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float4 g4 = *reinterpret_cast<const float4 *>(pG + j0 + 4 * u);
-                        gj[4 * u] = g4.x; gj[4 * u + 1] = g4.y; gj[4 * u + 2] = g4.z; gj[4 * u + 3] = g4.w;
-                    }
-                    tmem_wait_ld();
+                        for (int u = 0; u < 16; ++u) xv[u] = 0.f;
+                        if (is_a) continue;                  // the inverse never reads A above the diagonal
+                    } else {
+                        uint32_t kr[16];
+                        tmem_ld16(tmem + loff + T4_KQ + j0, kr);
+                        float fj[16];
+                        const float *fsrc = factored ? pinv : pG;
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int j = j0 + u;
-                        const float keep = (is_a ? (j < i) : (j <= i)) ? 1.f : 0.f;
-                        xv[u] = (wi * keep) * __expf(fminf(Gi - gj[u], 0.f)) * __uint_as_float(kr[u]);
+                        for (int u = 0; u < 4; ++u) {
+                            const float4 g4 = *reinterpret_cast<const float4 *>(fsrc + j0 + 4 * u);
+                            fj[4 * u] = g4.x; fj[4 * u + 1] = g4.y; fj[4 * u + 2] = g4.z; fj[4 * u + 3] = g4.w;
+                        }
+                        tmem_wait_ld();
+                        if (factored) {
+#pragma unroll
+                            for (int u = 0; u < 16; ++u) {
+                                const int j = j0 + u;
+                                const bool keep = is_a ? (j < i) : (j <= i);
+                                xv[u] = keep ? wi_e * fj[u] * __uint_as_float(kr[u]) : 0.f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 16; ++u) {
+                                const int j = j0 + u;
+                                const float keep = (is_a ? (j < i) : (j <= i)) ? 1.f : 0.f;
+                                xv[u] = (wi * keep) * __expf(fminf(Gi - fj[u], 0.f)) * __uint_as_float(kr[u]);
+                            }
+                        }
                     }
                     if (is_a) {
 #pragma unroll
@@ -576,16 +737,19 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                                 pack2(xv[8 * h2 + 4], xv[8 * h2 + 5]), pack2(xv[8 * h2 + 6], xv[8 * h2 + 7]));
                     }
                 }
-#pragma unroll 4
-                for (int e = t; e < 64 * 64; e += 128) {
-                    const int ii = e >> 6, jj = e & 63;
-                    Tf[ii * TP4 + jj] = (ii == jj) ? 1.f : 0.f;
+                // the inverse writes the diagonal 16 x 16 blocks and the blocks below them; of
+                // the blocks above, it reads only T[0:16, 16:32] and T[32:48, 48:64]
+#pragma unroll
+                for (int e = t; e < 512; e += 128) {
+                    const int blk = e >> 8, ii = (e >> 4) & 15, jj = e & 15;
+                    Tf[(32 * blk + ii) * TP4 + 32 * blk + 16 + jj] = 0.f;
                 }
             }
             tc_fence_before();
             group_sync<2>();
 
             if (t == 0) PMARK(k, 4);
+            if (p + 4 < nch && t < K4_C) fetch_gb(p + 4);    // lands during the inverse
             // ---- T = (I + A)^-1
             invert_unit_lower_64_tf32_wg<TP4>(Af, Tf, t, [] { group_sync<2>(); });
             group_sync<2>();
@@ -597,15 +761,18 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 unsigned char *dst = sm + (which ? S4_TPP : S4_TP);
 #pragma unroll 2
                 for (int cc = 0; cc < 8; ++cc) {
-                    float w8[8];
+                    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+                    if (8 * cc <= i) {                       // T is lower triangular
+                        float w8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = 8 * cc + e;
-                        const float sc = which ? pb[j] : pb[j] * pgam[j];
-                        w8[e] = (j <= i) ? Tf[i * TP4 + j] * sc : 0.f;
+                        for (int e = 0; e < 8; ++e) {
+                            const int j = 8 * cc + e;
+                            const float sc = which ? pb[j] : pb[j] * pgam[j];
+                            w8[e] = (j <= i) ? Tf[i * TP4 + j] * sc : 0.f;
+                        }
+                        o = make_uint4(pack2(w8[0], w8[1]), pack2(w8[2], w8[3]), pack2(w8[4], w8[5]), pack2(w8[6], w8[7]));
                     }
-                    *reinterpret_cast<uint4 *>(dst + sw128(i, cc)) =
-                        make_uint4(pack2(w8[0], w8[1]), pack2(w8[2], w8[3]), pack2(w8[4], w8[5]), pack2(w8[6], w8[7]));
+                    *reinterpret_cast<uint4 *>(dst + sw128(i, cc)) = o;
                 }
             }
             fence_proxy_async();
@@ -613,7 +780,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             group_sync<2>();
             if (t == 0) { mbar_arrive_local(bars + B_TT); PMARK(k, 6); }
 
-            // ---- W and U~ (M = 64 layout) into the send staging
+            // ---- W and U~ (M = 64 layout) into the staging
             if (!group_all<2>(t != 0 || wait_bar(B_WU, k & 1, false))) { fail(23); break; }
             if (t == 0) PMARK(k, 7);
             tc_fence_after();
@@ -653,14 +820,50 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
     } else if (warp == 8) {
         // ========================================================== chain issuer
+        // Off the chain: Q tiles, Q S_r, and the ring: chunk c's prepared data is loaded
+        // from its global chunk slot (once the producer has signalled it and ring slot c mod 2
+        // is free), and the producer is told as soon as it has landed, so it may reuse the
+        // global slot.  Every wait below also advances those two steps.
         if (lane == 0) {
-            // requests made by this thread, for draining after an abort
-            int q_req = 0, qs_req = 0, ws_req = 0, s2_req = 0, pu_req = 0, full_req[2] = {0, 0};
-            int sent_acked = -1;               // last chunk whose receipt was acknowledged
+            int q_req = 0, qs_req = 0, full_req0 = 0, full_req1 = 0;   // for draining after an abort
+            const uint32_t id_m64 = idesc_bf16(64, 32, false, true);
+            const uint64_t d_cq = sdesc_kmajor(smem_u32(sm + S4_CQ)), d_st = sdesc_mn_sw64(smem_u32(sm + S4_ST));
+            int next_load = 0;                  // next chunk to load
+            int load_limit = 1;                 // highest chunk whose ring slot is free
+            int acked = -1;                     // last chunk acknowledged to its producer
+            auto poll_ring = [&]() {
+                const int a = next_load;
+                if (a <= load_limit && a < nch &&
+                    mbar_try_wait_cluster(bars + B_READY + (a & 7), (uint32_t)((a >> 3) & 1))) {
+                    const int sa = a & 1;
+                    const unsigned char *src = gring + (size_t)(a & 7) * K4_GCHUNK;
+                    unsigned char *dst = sm + S4_RING + sa * K4_RING_BYTES;
+                    uint64_t *fb = bars + (sa ? B_FULL1 : B_FULL0);
+                    fence_proxy_async_global();
+                    mbar_arrive_expect_tx(fb, K4_RING_BYTES);
+                    bulk_load_global(dst, src, 24576, fb);                          // W | P
+                    bulk_load_global(dst + 24576, src + 24576 + r * 4096, 4096, fb);  // U~_r
+                    if (sa) ++full_req1; else ++full_req0;
+                    next_load = a + 1;
+                }
+                const int k = acked + 1;
+                if (k < next_load && mbar_try_wait(bars + ((k & 1) ? B_FULL1 : B_FULL0), (uint32_t)((k >> 1) & 1))) {
+                    // the loads this covers have completed, so there is nothing to publish
+                    mbar_arrive_remote_relaxed(map_to_rank(bars + B_GFREE0 + ((k >> 2) & 1), (uint32_t)(k & 3)));
+                    CMARK(k, 2);
+                    acked = k;
+                }
+            };
+            auto wait_ring = [&](int b, uint32_t parity) -> bool {
+                for (uint32_t i = 0; i < budget; ++i) {
+                    if (mbar_try_wait(bars + b, parity)) return true;
+                    poll_ring();
+                    if (*abort_flag) return false;
+                }
+                return false;
+            };
             if (nch > 0) {
                 q_req = 1;
-                full_req[0] = 1;
-                full_req[1] = nch > 1 ? 1 : 0;
                 const int tb = (int)t_begin;
                 mbar_arrive_expect_tx(bars + B_CQ, 16384);
                 tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tb);
@@ -668,77 +871,37 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 mbar_arrive_expect_tx(bars + B_CK, 16384);
                 tma_load_3d(sm + S4_CK, &tm_k, bars + B_CK, 0, hq, tb);
                 tma_load_3d(sm + S4_CK + 8192, &tm_k, bars + B_CK, 64, hq, tb);
-                mbar_arrive_expect_tx(bars + B_FULL0, K4_RING_BYTES);
-                if (nch > 1) mbar_arrive_expect_tx(bars + B_FULL1, K4_RING_BYTES);
                 mbar_arrive_local(bars + B_OFREE0);     // both output buffers start free
                 mbar_arrive_local(bars + B_OFREE1);
             }
-            const uint32_t id_m64 = idesc_bf16(64, 32, false, false);
-            const uint32_t id_s2 = idesc_bf16(128, 32, true, false);
 #pragma unroll 1
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1;
-                const uint32_t ring_s = smem_u32(sm + S4_RING + s * K4_RING_BYTES);
-                const uint32_t st = smem_u32(sm + S4_ST), ut = smem_u32(sm + S4_UT);
                 CMARK(c, 0);
-                // W S_r is on the state chain: it needs S_r^T of the previous chunk and W of
-                // this one, and goes first
-                if (!wait_bar(B_ST, c & 1, false)) { fail(31); break; }
-                if (!wait_bar(s ? B_FULL1 : B_FULL0, (c >> 1) & 1, true)) { fail(33); break; }
+                GMARK(c, 26);
+                // chunk c's prepared data has landed (and been acknowledged)
+                {
+                    bool okf = true;
+                    for (uint32_t i = 0; acked < c; ++i) {
+                        poll_ring();
+                        if (*abort_flag || i >= budget) { okf = false; break; }
+                    }
+                    if (!okf) { fail(33); break; }
+                }
                 CMARK(c, 1);
+                // Q S_r -> D_QS[s] right behind W S_r in the pipe (both read the same S_r tile)
+                if (!wait_ring(B_WSI, c & 1)) { fail(35); break; }
+                if (!wait_ring(L2N ? B_CQN : B_CQ, c & 1)) { fail(30); break; }
+                if (!wait_ring(s ? B_OFREE1 : B_OFREE0, (c >> 1) & 1)) { fail(32); break; }
                 tc_fence_after();
-                {
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t o4 = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        const uint32_t ob = (ks >> 2) * 4096 + (ks & 3) * 32;
-                        umma_bf16(tmem + T4_WS, sdesc_kmajor(ring_s + o4), sdesc_kmajor(st + ob), id_m64, ks > 0);
-                    }
-                    umma_commit(bars + B_WS);
-                    ++ws_req;
-                }
-                CMARK(c, 2);
-                if (sent_acked < c) {
-                    mbar_arrive_remote_relaxed(map_to_rank(bars + B_SENT, (uint32_t)(c & 3)));
-                    sent_acked = c;
-                }
-                // Q S_r (outputs only) reads the same S_r^T, so it must be issued before S2
-                // (the state epilogue rewrites S_r^T once S2's commit completes); it runs
-                // while the U epilogue works, ahead of S2 in the pipe
-                if (!wait_bar(l2norm ? B_CQN : B_CQ, c & 1, false)) { fail(30); break; }
-                if (!wait_bar(s ? B_OFREE1 : B_OFREE0, (c >> 1) & 1, false)) { fail(32); break; }
-                tc_fence_after();
-                {
-                    const uint32_t cq = smem_u32(sm + S4_CQ);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t o4 = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        const uint32_t ob = (ks >> 2) * 4096 + (ks & 3) * 32;
-                        umma_bf16(tmem + T4_QS + 32 * s, sdesc_kmajor(cq + o4), sdesc_kmajor(st + ob), id_m64, ks > 0);
-                    }
-                    umma_commit(bars + B_QS);
-                    ++qs_req;
-                }
-                if (!wait_bar(B_U, c & 1, false)) { fail(35); break; }
-                if (!wait_bar(B_KT, c & 1, false)) { fail(36); break; }
-                CMARK(c, 3);
-                tc_fence_after();
-                {   // S_r += K~^T U_r (on the chain) ; P U_r -> D_PU[s]
-                    const uint32_t kt = smem_u32(sm + S4_CKT);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tmem + T4_S, sdesc_mnmajor(kt + ks * 2048, 8192), sdesc_kmajor(ut + ks * 32), id_s2, 1);
-                    umma_commit(bars + B_S2);
-                    ++s2_req;
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tmem + T4_PU + 32 * s, sdesc_kmajor(ring_s + 16384 + ks * 32), sdesc_kmajor(ut + ks * 32), id_m64, ks > 0);
-                    umma_commit(bars + B_PU);
-                    ++pu_req;
-                }
-                CMARK(c, 4);
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16(tmem + T4_QS + 32 * s, d_cq + (ks >> 2) * 512 + (ks & 3) * 2, d_st + ks * 64, id_m64, ks > 0);
+                umma_commit(bars + B_QS);
+                ++qs_req;
+                CMARK(c, 19);
                 // Q of the next chunk into the buffer Q S_r has finished reading
-                if (!wait_bar(B_QS, c & 1, false)) { fail(34); break; }
+                if (!wait_ring(B_QS, c & 1)) { fail(34); break; }
                 if (c + 1 < nch) {
                     ++q_req;
                     const int tn = (int)(t_begin + (long long)(c + 1) * K4_C);
@@ -746,40 +909,19 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tn);
                     tma_load_3d(sm + S4_CQ + 8192, &tm_q, bars + B_CQ, 64, hq, tn);
                 }
-                {   // wait for S2; meanwhile acknowledge the next chunk's data as soon as it lands
-                    bool ok = false;
-                    const int cn = c + 1;
-                    for (uint32_t it = 0; it < budget; ++it) {
-                        if (cn < nch && sent_acked < cn &&
-                            mbar_try_wait_cluster(bars + ((cn & 1) ? B_FULL1 : B_FULL0), (uint32_t)((cn >> 1) & 1))) {
-                            mbar_arrive_remote_relaxed(map_to_rank(bars + B_SENT, (uint32_t)(cn & 3)));
-                            sent_acked = cn;
-                        }
-                        if (mbar_try_wait(bars + B_S2, (uint32_t)(c & 1))) { ok = true; break; }
-                        if (*abort_flag) break;
-                    }
-                    if (!ok) { fail(37); break; }
-                }
-                if (!wait_bar(B_PU, c & 1, false)) { fail(38); break; }
+                CMARK(c, 24);
+                // ring slot s is free for chunk c + 2 once P U_r (the last MMA reading it) is done
+                if (!wait_ring(s ? B_PU1 : B_PU0, (c >> 1) & 1)) { fail(38); break; }
+                load_limit = c + 2;
+                poll_ring();
                 CMARK(c, 5);
-                if (c + 2 < nch) {             // slot s is free for chunk c + 2
-                    ++full_req[s];
-                    mbar_arrive_expect_tx(bars + (s ? B_FULL1 : B_FULL0), K4_RING_BYTES);
-                    mbar_arrive_remote_relaxed(map_to_rank(bars + B_EMPTY, (uint32_t)((c + 2) & 3)));
-                }
             }
             if (*abort_flag) {
-                // let this thread's loads, MMAs and the copies other CTAs may still be
-                // writing into this CTA's ring land before shared memory and TMEM go away
+                // let this thread's loads land before shared memory goes away
                 drain_bar(bars + B_CQ, q_req, false);
                 drain_bar(bars + B_QS, qs_req, false);
-                drain_bar(bars + B_WS, ws_req, false);
-                drain_bar(bars + B_S2, s2_req, false);
-                drain_bar(bars + B_PU, pu_req, false);
-                // a producer that sent anything has done so long ago; one that aborted first
-                // never will, so these two waits are kept short
-                drain_bar(bars + B_FULL0, full_req[0], true, 1u << 16);
-                drain_bar(bars + B_FULL1, full_req[1], true, 1u << 16);
+                drain_bar(bars + B_FULL0, full_req0, false);
+                drain_bar(bars + B_FULL1, full_req1, false);
             }
         }
         __syncwarp();
@@ -810,7 +952,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tc_fence_after();
                 {   // P1: [K;Q] K^T
                     const uint32_t kq = smem_u32(sm + S4_PKQ);
-#pragma unroll
+#pragma unroll 1
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t a = kq + (ks >> 2) * 16384 + (ks & 3) * 32;
                         umma_bf16(tmem + T4_KQ, sdesc_kmajor(a), sdesc_kmajor(a), id_p1, ks > 0);
@@ -823,10 +965,10 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 {   // W = T' K ; U~ = T'' V   (M = 64, N = 128)
                     const uint32_t kq = smem_u32(sm + S4_PKQ), pv = smem_u32(sm + S4_PV);
                     const uint32_t tpa = smem_u32(sm + S4_TP), tppa = smem_u32(sm + S4_TPP);
-#pragma unroll
+#pragma unroll 1
                     for (int ks = 0; ks < 4; ++ks)
                         umma_bf16(tmem + T4_W, sdesc_kmajor(tpa + ks * 32), sdesc_mnmajor(kq + ks * 2048, 16384), id_wu, ks > 0);
-#pragma unroll
+#pragma unroll 1
                     for (int ks = 0; ks < 4; ++ks)
                         umma_bf16(tmem + T4_U, sdesc_kmajor(tppa + ks * 32), sdesc_mnmajor(pv + ks * 2048, 8192), id_wu, ks > 0);
                     umma_commit(bars + B_WU);
@@ -834,24 +976,26 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 if (!wait_bar(B_WU, k & 1, false)) { fail(42); break; }
                 if (p + 4 < nch) load_inputs(p + 4);   // the prep buffers are free again
+                // staging -> this production's global chunk slot (p mod 8), last used two
+                // productions ago: every CTA must have loaded that one first
                 if (!wait_bar(B_STG, k & 1, false)) { fail(43); break; }
-                // every consumer has released slot (p & 1) (it finished chunk p - 2)
-                if ((int)r >= 2) {
-                    if (!wait_bar(B_EMPTY, k & 1, true)) { fail(44); break; }
-                } else if (k >= 1) {
-                    if (!wait_bar(B_EMPTY, (k - 1) & 1, true)) { fail(44); break; }
-                }
-                PMARK(k, 9);
-                const int s = p & 1;
-                unsigned char *slot = sm + S4_RING + s * K4_RING_BYTES;
+                if (k >= 2 && !wait_bar(B_GFREE0 + (k & 1), ((k - 2) >> 1) & 1, true)) { fail(44); break; }
+                unsigned char *gchunk = gring + (size_t)(p & 7) * K4_GCHUNK;
+                bulk_store_global(gchunk, sm + S4_WSTG, 16384);
+                bulk_store_global(gchunk + 16384, sm + S4_PSTG, 8192);
+                bulk_store_global(gchunk + 24576, sm + S4_USTG, 16384);
+                bulk_commit();
+                bulk_wait_read_all();
+                mbar_arrive_local(bars + B_SFREE);
+                bulk_wait_all();
+                // the writes are complete: one release, then a signal to every CTA
+                fence_proxy_async_global();
+                fence_release_cluster();
 #pragma unroll 1
-                for (uint32_t dst = 0; dst < 4; ++dst) {
-                    const uint32_t bar = map_to_rank(bars + (s ? B_FULL1 : B_FULL0), dst);
-                    bulk_copy_to_cluster(map_to_rank(slot, dst), sm + S4_WSTG, 16384, bar);
-                    bulk_copy_to_cluster(map_to_rank(slot + 16384, dst), sm + S4_PSTG, 8192, bar);
-                    bulk_copy_to_cluster(map_to_rank(slot + 24576, dst), sm + S4_USTG + dst * 4096, 4096, bar);
-                }
+                for (uint32_t d = 0; d < 4; ++d) mbar_arrive_remote_relaxed(map_to_rank(bars + B_READY + (p & 7), d));
+                PMARK(k, 9);
             }
+            bulk_wait_all();
             if (*abort_flag) {
                 drain_bar(bars + B_PKQ, in_req, false);
                 drain_bar(bars + B_PV, in_req, false);
@@ -867,6 +1011,11 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     cluster_sync();
     tc_fence_after();
     if (warp == 8) tmem_dealloc(tmem, 512);
+    if (r == 0 && tid == 256 && ring_slot >= 0) {
+        __threadfence();
+        atomicExch(&g4_pool[ring_slot], 0);
+    }
+    SPAN(1);
 }
 
 // ------------------------------------------------------------------------ host side
@@ -916,15 +1065,19 @@ cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_cluster_kernel,
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_cluster_kernel<false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, K4_SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_tc_cluster_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, K4_SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     dim3 grid((unsigned)(4 * N), (unsigned)H_v);
-    prefill_tc_cluster_kernel<<<grid, K4_THREADS, K4_SMEM, stream>>>(
+    auto kern = l2norm ? prefill_tc_cluster_kernel<true> : prefill_tc_cluster_kernel<false>;
+    kern<<<grid, K4_THREADS, K4_SMEM, stream>>>(
         mq, mk, mv, g, beta, S0, (__nv_bfloat16 *)out, S_final, cu, T_dense, H_qk, H_v, scale,
-        l2norm, err, wait_budget4());
+        err, wait_budget4());
     return cudaGetLastError();
 }
 

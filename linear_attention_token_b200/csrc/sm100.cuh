@@ -142,6 +142,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
+// Shared-memory matrix descriptor, SWIZZLE_64B, MN-major operand of at most 32 MN-elements:
+// each K index is one 64-byte row (32 bf16), 8-row K groups (512 B atoms) at `sbo` bytes.
+// Tiles are 512-B aligned so the base-offset field stays 0.
+__device__ __forceinline__ uint64_t sdesc_mn_sw64(uint32_t saddr, uint32_t sbo = 512) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                  // leading offset (one MN block: not used)
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;                  // layout: 64-byte swizzle
+    return d;
+}
+
 __device__ __forceinline__ uint64_t sdesc_kmajor(uint32_t saddr, uint32_t sbo = 1024) {
     return sdesc_sw128(saddr, 16, sbo);
 }
@@ -208,6 +221,12 @@ __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];"
                  ::"r"(cluster_addr) : "memory");
 }
+// release fence at cluster scope: with relaxed arrives after it, one fence publishes this
+// thread's earlier writes to every CTA it then signals (each release-arrive would pay for
+// its own release)
+__device__ __forceinline__ void fence_release_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
 __device__ __forceinline__ void mbar_arrive_local(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -236,11 +255,60 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, const void *s
         ::"r"(dst), "r"(smem_u32(src)), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Generic-proxy global writes of this thread ordered before later async-proxy accesses
+// (a bulk copy another CTA issues after synchronising with this thread).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Bulk copy (non-tensor) of `bytes` contiguous bytes from global memory into this CTA's
+// shared memory, completing on `bar` (both addresses 16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_load_global(void *dst, const void *src, uint32_t bytes,
+                                                 uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+// Bulk copy (non-tensor) of `bytes` from this CTA's shared memory to global memory,
+// tracked by this thread's bulk async-groups (16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_store_global(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// this thread's committed bulk stores have finished reading their shared-memory sources
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// this thread's committed bulk stores have completed (their writes are performed)
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// 32-bit load from a shared::cluster address (another CTA's shared memory)
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+// 32-bit store to a shared::cluster address (another CTA's shared memory)
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled tile
 // whose rows are 128 bytes apart (tile base 1024-aligned): the chunk index is
 // XOR-ed with the row index modulo 8.
 __host__ __device__ constexpr uint32_t sw128(uint32_t r, uint32_t c) {
     return r * 128u + ((c ^ (r & 7u)) << 4);
+}
+
+// Byte offset of 16-byte chunk `c` (0..3) of row `r` in a 64-byte-swizzled tile whose
+// rows are 64 bytes apart (tile base 512-aligned): the chunk index is XOR-ed with bits
+// 1..2 of the row index (address bits 7..8 onto bits 4..5).
+__host__ __device__ constexpr uint32_t sw64(uint32_t r, uint32_t c) {
+    return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4);
 }
 
 }  // namespace sm100

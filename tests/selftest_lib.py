@@ -30,5 +30,8 @@ def load():
     L.selftest_umma_timing2.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
     L.selftest_tma_timing.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, P]
+    L.selftest_contention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+    L.selftest_dsmem_bw.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+    L.selftest_movement.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
     L.selftest_tma.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
     return L

@@ -30,6 +30,10 @@ def L():
     32 | 64,           # M=64, N=32, K=64:  P U
     32 | 2 | 8,        # M=64, N=128, K=64: T' K with B MN-major
     64 | 1,            # M=128, N=32, K=64: K~^T U with A MN-major
+    32 | 64 | 16 | 128,  # M=64, N=32, K=128: W S with S in 64-byte-swizzled rows d
+    32 | 64 | 128,       # M=64, N=32, K=64:  P U with U in 64-byte-swizzled rows i
+    64 | 1 | 128,        # M=128, N=32, K=64: K~^T U, A MN-major, U in 64-byte rows
+    64 | 16 | 128 | 4,   # M=128, N=32, K=128, negated 64-byte-swizzled B
 ])
 def test_umma_placements(L, variant):
     torch.manual_seed(variant)
