@@ -943,6 +943,21 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tma_load_3d(sm + S4_PV, &tm_v, bars + B_PV, 0, h, tp);
                 tma_load_3d(sm + S4_PV + 8192, &tm_v, bars + B_PV, 64, h, tp);
             };
+            // the bulk stores of a production complete while the next one starts: its P1 is
+            // issued first, then the stores are waited for, the staging released and the
+            // chunk signalled to every CTA
+            int pend = -1;                          // chunk whose stores are in flight
+            auto finish_stores = [&]() {
+                bulk_wait_read_all();
+                mbar_arrive_local(bars + B_SFREE);
+                bulk_wait_all();
+                // the writes are complete: one release, then a signal to every CTA
+                fence_proxy_async_global();
+                fence_release_cluster();
+#pragma unroll 1
+                for (uint32_t d = 0; d < 4; ++d) mbar_arrive_remote_relaxed(map_to_rank(bars + B_READY + (pend & 7), d));
+                pend = -1;
+            };
             if ((int)r < nch) load_inputs((int)r);
 #pragma unroll 1
             for (int k = 0;; ++k) {
@@ -960,6 +975,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     umma_commit(bars + B_P1);
                     ++p1_req;
                 }
+                if (pend >= 0) finish_stores();
                 if (!wait_bar(B_TT, k & 1, false)) { fail(41); break; }
                 tc_fence_after();
                 {   // W = T' K ; U~ = T'' V   (M = 64, N = 128)
@@ -985,16 +1001,10 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 bulk_store_global(gchunk + 16384, sm + S4_PSTG, 8192);
                 bulk_store_global(gchunk + 24576, sm + S4_USTG, 16384);
                 bulk_commit();
-                bulk_wait_read_all();
-                mbar_arrive_local(bars + B_SFREE);
-                bulk_wait_all();
-                // the writes are complete: one release, then a signal to every CTA
-                fence_proxy_async_global();
-                fence_release_cluster();
-#pragma unroll 1
-                for (uint32_t d = 0; d < 4; ++d) mbar_arrive_remote_relaxed(map_to_rank(bars + B_READY + (p & 7), d));
+                pend = p;
                 PMARK(k, 9);
             }
+            if (pend >= 0 && !*abort_flag) finish_stores();
             bulk_wait_all();
             if (*abort_flag) {
                 drain_bar(bars + B_PKQ, in_req, false);
