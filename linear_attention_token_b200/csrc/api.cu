@@ -23,11 +23,6 @@ cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *
                                       const int32_t *cu, int N, long long T_dense, long long T_total,
                                       int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
                                       cudaStream_t stream);
-cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
-                              const float *beta, const float *S0, void *out, float *S_final,
-                              const int32_t *cu, int N, long long T_dense, long long T_total,
-                              int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
-                              cudaStream_t stream);
 size_t static_scratch_capacity();
 cudaError_t static_scratch_ptr(void **out);
 }  // namespace gdn

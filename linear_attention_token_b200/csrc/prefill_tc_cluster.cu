@@ -1062,6 +1062,11 @@ uint32_t wait_budget4() {
 
 }  // namespace
 
+bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype)
+{
+    return dk == K4_D && dv == K4_D && dtype == GDN_BF16;
+}
+
 cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *v, const float *g,
                                       const float *beta, const float *S0, void *out, float *S_final,
                                       const int32_t *cu, int N, long long T_dense, long long T_total,

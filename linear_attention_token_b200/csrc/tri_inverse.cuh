@@ -148,64 +148,14 @@ __device__ __forceinline__ void warp_gemm_16x16(const float *X, const float *Y, 
     }
 }
 
-#ifndef GDN_TRI_MARK
-#define GDN_TRI_MARK(k) do { } while (0)
-#endif
-
-// dbg_chunk only feeds the optional profiling marks (GDN_TRI_MARK).
-template <int TP>
-__device__ __forceinline__ void invert_unit_lower_64_tf32(float *A, float *T, int tid, int dbg_chunk = 0)
-{
-    (void)dbg_chunk;
-    const int warp = tid >> 5, lane = tid & 31;
-    // 1. diagonal 16 x 16 blocks in fp32 on the CUDA cores (as above)
-    if (tid < 64) {
-        const int b = tid >> 4, col = tid & 15;
-        const float *Ab = A + (16 * b) * TP + 16 * b;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-            for (int m = 0; m + 1 < r; m += 2) {
-                acc0 = fmaf(Ab[r * TP + m], x[m], acc0);
-                acc1 = fmaf(Ab[r * TP + m + 1], x[m + 1], acc1);
-            }
-            if (r & 1) acc0 = fmaf(Ab[r * TP + r - 1], x[r - 1], acc0);
-            x[r] = (r == col) ? 1.f : ((r < col) ? 0.f : -(acc0 + acc1));
-        }
-        float *Tb = T + (16 * b) * TP + 16 * b;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Tb[r * TP + col] = x[r];
-    }
-    GDN_TRI_MARK(22);
-    __syncthreads();
-    GDN_TRI_MARK(23);
-    // 2. 16 -> 32: warp p merges blocks (2p, 2p+1); scratch in A's upper block (lo, hi)
-    if (warp < 2) {
-        const int lo = 32 * warp, hi = lo + 16;
-        warp_gemm_16x16<TP, 16>(A + hi * TP + lo, T + lo * TP + lo, A + lo * TP + hi, 1.f, lane);
-        __syncwarp();
-        warp_gemm_16x16<TP, 16>(T + hi * TP + hi, A + lo * TP + hi, T + hi * TP + lo, -1.f, lane);
-    }
-    GDN_TRI_MARK(24);
-    __syncthreads();
-    GDN_TRI_MARK(25);
-    // 3. 32 -> 64: warp w < 4 owns the 16 x 16 quadrant (w >> 1, w & 1) of the 32 x 32 result;
-    //    scratch X = A_HL D_L in rows 0..31, columns 32..63 of A
-    if (warp < 4) {
-        const int mb = (warp >> 1) * 16, nb = (warp & 1) * 16;
-        warp_gemm_16x16<TP, 32>(A + (32 + mb) * TP, T + nb, A + mb * TP + 32 + nb, 1.f, lane);
-    }
-    __syncthreads();
-    if (warp < 4) {
-        const int mb = (warp >> 1) * 16, nb = (warp & 1) * 16;
-        warp_gemm_16x16<TP, 32>(T + (32 + mb) * TP + 32, A + 32 + nb, T + (32 + mb) * TP + nb, -1.f, lane);
-    }
-}
-
-// Warpgroup version: the same algorithm run by 128 threads (t = 0..127) that
-// synchronise with `sync()` (a named barrier over exactly those threads).
+// Blocked inverse with tf32 tensor-core merges, run by one warpgroup (t = 0..127) that
+// synchronises with `sync()` (a named barrier over exactly those threads):
+//   1. the four diagonal 16 x 16 blocks by forward substitution in fp32 (one thread per
+//      column of a block);
+//   2. 16 -> 32: warp p merges blocks (2p, 2p+1), T_HL = -T_HH A_HL T_LL, with the
+//      product A_HL T_LL kept in A's upper block (lo, hi) as scratch;
+//   3. 32 -> 64: warp w < 4 owns quadrant (w >> 1, w & 1) of the lower-left 32 x 32 block,
+//      with A_HL T_LL kept in rows 0..31, columns 32..63 of A.
 template <int TP, typename Sync>
 __device__ __forceinline__ void invert_unit_lower_64_tf32_wg(float *A, float *T, int t, Sync sync)
 {
