@@ -66,6 +66,18 @@ def decode_bytes_per_step(w) -> int:
             + N * w.H_v * 8)
 
 
+VERIFY_T = 4      # tokens per gdn_decode_multi call (e.g. three drafted tokens + one)
+
+
+def decode_multi_bytes_per_call(w, T: int) -> int:
+    """Algorithmic bytes of one multi-token call: the state read and written once, and T
+    tokens' q, k, v, out, g, beta."""
+    e = torch.tensor([], dtype=w.dtype).element_size()
+    N = w.decode_seqs
+    return (N * w.H_v * w.dk * w.dv * 4 * 2
+            + T * (N * (2 * w.H_qk * w.dk + 2 * w.H_v * w.dv) * e + N * w.H_v * 8))
+
+
 def decode_flops_per_step(w) -> int:
     # a = S^T k, b = S^T q, S <- alpha S + k u^T: 3 MACs per state element
     return 2 * 3 * w.decode_seqs * w.H_v * w.dk * w.dv
@@ -239,6 +251,35 @@ def time_decode(gdn, w, passes, warmup, stream, device):
     return [a.elapsed_time(b) for a, b in evs]
 
 
+def time_decode_multi(gdn, w, T, passes, warmup, stream, device):
+    """The decode workload's token stream, T consecutive tokens per gdn_decode_multi call
+    (decode_steps / T calls per pass, every token committed)."""
+    S = inputs.decode_state(w, device)
+    steps = [inputs.decode_step_inputs(w, s, device) for s in range(w.decode_steps)]
+    xs = [{n: torch.stack([steps[j * T + t][n] for t in range(T)], dim=1).contiguous()
+           for n in ("q", "k", "v", "g", "beta")} for j in range(w.decode_steps // T)]
+    del steps
+    outs = [torch.empty_like(x["v"]) for x in xs]
+
+    def one_pass():
+        for x, o in zip(xs, outs):
+            gdn.gdn_decode_multi(x["q"], x["k"], x["v"], x["g"], x["beta"], S, out=o, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one_pass()
+    stream.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(passes)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            a.record(stream)
+            one_pass()
+            b.record(stream)
+    stream.synchronize()
+    return [a.elapsed_time(b) for a, b in evs], len(xs)
+
+
 def cpu_baseline_prefill(w, max_tokens=None):
     """The oracle (float variant, all host cores) on the prefill workload, timed."""
     import oracle
@@ -332,6 +373,9 @@ def run_ours(args):
         dec_passes = max(1, min(args.steps, 5))
         dtimes = time_decode(gdn, wd, dec_passes, max(1, min(args.warmup, 3)), stream, device)
         barrier(world)
+        vtimes, v_calls = time_decode_multi(gdn, wd, VERIFY_T, dec_passes, max(1, min(args.warmup, 3)),
+                                            stream, device)
+        barrier(world)
     clocks = clk.summary()
     if status != 0:
         raise RuntimeError(f"device error after prefill: {gdn.gdn_status_string(status)}")
@@ -349,6 +393,10 @@ def run_ours(args):
     dec_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode.cu")
     ms_dec_step = ms_decode_pass / wd.decode_steps
     dec_bytes = decode_bytes_per_step(wd)
+    ms_verify_pass = max_over_ranks(sum(vtimes) / len(vtimes), world)
+    ver_bytes = decode_multi_bytes_per_call(wd, VERIFY_T)
+    ver_gbs = ver_bytes / (ms_verify_pass / v_calls * 1e-3) / 1e9
+    ver_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode_multi.cu")
     dec_gbs = dec_bytes / (ms_dec_step * 1e-3) / 1e9
 
     line = {
@@ -385,11 +433,21 @@ def run_ours(args):
                          "peak_source": f"{peaks['source']} copy bandwidth",
                          "algorithmic_bytes_per_launch": dec_bytes},
         },
+        "decode_multi": {
+            "workload": f"{wd.name} as {VERIFY_T}-token calls", "tokens_per_call": VERIFY_T,
+            "value": world * wd.decode_seqs * wd.decode_steps / (ms_verify_pass * 1e-3),
+            "unit": "tokens/s", "ms_per_call": ms_verify_pass / v_calls, "passes": dec_passes,
+            "roofline": {"bound": "hbm", "achieved": ver_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": ver_gbs / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic("decode_multi", ver_src),
+                         "peak_source": f"{peaks['source']} copy bandwidth",
+                         "algorithmic_bytes_per_launch": ver_bytes},
+        },
         "e2e": {"value": world * tok / (ms_e2e * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "gdn_prefill via the C ABI; pinned host inputs copied in and outputs + "
                         "final state copied out inside the timed region"},
-        "gpu_launches": args.steps + dec_passes * wd.decode_steps,
+        "gpu_launches": args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

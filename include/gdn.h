@@ -108,6 +108,29 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const fl
                            int32_t H_qk, int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype,
                            float scale, uint32_t flags, cudaStream_t stream);
 
+/* Multi-token decode / draft verification: T consecutive tokens (1 <= T <= 8) of
+ * every (sequence, value head) applied in one call, Eq. (1) once per token in order,
+ * with the state read once and written at most once.  This is the sequential
+ * recurrence over a short segment (the same rule as gdn_decode_step, applied T times);
+ * it serves speculative decoding, where several drafted tokens (for instance from a
+ * multi-token-prediction head) are checked at once and only an accepted prefix is
+ * kept.
+ *
+ *   q, k     : [N, T, H_qk, dk] dtype;  v, out : [N, T, H_v, dv] dtype
+ *   g, beta  : [N, T, H_v] fp32
+ *   S_inout  : [N, H_v, dk, dv] fp32
+ *   n_commit : device [N] int32 or NULL.  out[n, t] is o_t for every t < T (each token
+ *              sees the state after all tokens before it).  S_inout[n] is replaced by
+ *              the state after the first c = n_commit[n] tokens (clamped to [0, T];
+ *              c = 0 leaves it unchanged); NULL means c = T for every sequence.
+ * dk, dv in {64, 128}; H_v % H_qk == 0; q, k, v, out, S_inout 16-byte aligned.
+ * GDN_ERR_UNSUPPORTED for T outside [1, 8].  N == 0 is a no-op (pointers may be NULL). */
+gdn_status gdn_decode_multi(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float *S_inout, void *out,
+                            const int32_t *n_commit, int32_t N, int32_t T, int32_t H_qk,
+                            int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype, float scale,
+                            uint32_t flags, cudaStream_t stream);
+
 /* gdn_prefill for callers that cannot allocate device memory: the same computation
  * and arguments, minus the workspace.  The paper has no counterpart; this is a
  * deployment convenience.  Some callers cannot call cudaMalloc (for instance code

@@ -23,7 +23,8 @@ GDN_FLAG_FORCE_CUDA_CORE = 2
 
 # every symbol include/gdn.h declares
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
-            "gdn_get_device_error", "gdn_status_string", "gdn_prefill_static_scratch")
+            "gdn_get_device_error", "gdn_status_string", "gdn_prefill_static_scratch",
+            "gdn_decode_multi")
 
 _lib = None
 
@@ -55,6 +56,9 @@ def lib():
         L.gdn_decode_step.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, I32, I32, ctypes.c_int,
                                       F, U32, P]
         L.gdn_decode_step.restype = ctypes.c_int
+        L.gdn_decode_multi.argtypes = [P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
+                                       ctypes.c_int, F, U32, P]
+        L.gdn_decode_multi.restype = ctypes.c_int
         L.gdn_get_device_error.argtypes = [P, P]
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -182,6 +186,25 @@ def gdn_decode_step(q, k, v, g, beta, S_inout, *, out=None, scale: float = 1.0, 
         _dev(S_inout, "S_inout"), _dev(out, "out"), N, H_qk, H_v, dk, dv, _dtype_code(q),
         float(scale), int(flags), _stream(stream))
     _check(st, "gdn_decode_step")
+    return out
+
+
+def gdn_decode_multi(q, k, v, g, beta, S_inout, *, n_commit=None, out=None, scale: float = 1.0,
+                     flags: int = 0, stream=None):
+    """T consecutive tokens per (sequence, head) in one call: q,k [N, T, H_qk, dk];
+    v [N, T, H_v, dv]; g, beta [N, T, H_v].  S_inout [N, H_v, dk, dv] becomes the state
+    after n_commit[n] tokens (int32 [N] on the device; None = all T).  Returns out."""
+    N, T, H_qk, dk = q.shape
+    H_v, dv = v.shape[-2:]
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    if n_commit is not None and n_commit.dtype != torch.int32:
+        raise ValueError("n_commit must be int32")
+    st = lib().gdn_decode_multi(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+        _dev(S_inout, "S_inout"), _dev(out, "out"), _dev(n_commit, "n_commit"), N, T, H_qk, H_v,
+        dk, dv, _dtype_code(q), float(scale), int(flags), _stream(stream))
+    _check(st, "gdn_decode_multi")
     return out
 
 

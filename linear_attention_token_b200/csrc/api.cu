@@ -23,6 +23,10 @@ cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *
                                       const int32_t *cu, int N, long long T_dense, long long T_total,
                                       int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
                                       cudaStream_t stream);
+cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, float *S, void *out, const int32_t *n_commit,
+                                int N, int T, int H_qk, int H_v, int dk, int dv, gdn_dtype dtype,
+                                float scale, int l2norm, cudaStream_t stream);
 size_t static_scratch_capacity();
 cudaError_t static_scratch_ptr(void **out);
 }  // namespace gdn
@@ -128,6 +132,26 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v, 
     const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
     cudaError_t e = gdn::launch_decode(q, k, v, g, beta, S_inout, out, N, H_qk, H_v, dk, dv,
                                        dtype, scale, l2, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API gdn_status gdn_decode_multi(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, float *S_inout, void *out,
+                                    const int32_t *n_commit, int32_t N, int32_t T, int32_t H_qk,
+                                    int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype,
+                                    float scale, uint32_t flags, cudaStream_t stream)
+{
+    if (N < 0) return GDN_ERR_INVALID_ARG;
+    if (T < 1 || T > 8) return GDN_ERR_UNSUPPORTED;
+    gdn_status st = common_checks(q, k, v, g, beta, out, H_qk, H_v, dk, dv, dtype, flags, N > 0);
+    if (st != GDN_OK) return st;
+    if ((N > 0 && !S_inout) || !aligned(S_inout, 16) || !aligned(n_commit, 4))
+        return GDN_ERR_INVALID_ARG;
+    if ((long long)N * H_v > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (N == 0) return GDN_OK;
+    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    cudaError_t e = gdn::launch_decode_multi(q, k, v, g, beta, S_inout, out, n_commit, N, T,
+                                             H_qk, H_v, dk, dv, dtype, scale, l2, stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -145,3 +145,31 @@ def decode_step(q, k, v, g, beta, S, scale: float = 1.0, l2norm: bool = False,
     cu = np.arange(N + 1, dtype=np.int64)
     return recurrent(q, k, v, g, beta, S0=S, cu_seqlens=cu, scale=scale, l2norm=l2norm,
                      threads=threads)
+
+
+def decode_multi(q, k, v, g, beta, S, n_commit=None, scale: float = 1.0, l2norm: bool = False,
+                 threads: int = 0):
+    """T consecutive tokens per sequence: q,k [N,T,H_qk,dk], v [N,T,H_v,dv], g,beta [N,T,H_v],
+    S [N,H_v,dk,dv], n_commit [N] or None.
+
+    Eq. (1) applied to each sequence's T tokens in order: the outputs are the
+    recurrence's over all T tokens, and the returned state is the recurrence's state
+    after the first n_commit[n] tokens (clamped to [0, T]; all T when None).  Returns
+    (out [N,T,H_v,dv], S_new) as numpy.
+    """
+    N, T = q.shape[0], q.shape[1]
+    flat = lambda x: _arr(x, np.float64).reshape((N * T,) + tuple(x.shape[2:]))
+    cu = np.arange(0, N * T + 1, T, dtype=np.int64)
+    out, S_all = recurrent(flat(q), flat(k), flat(v), flat(g), flat(beta), S0=S, cu_seqlens=cu,
+                           scale=scale, l2norm=l2norm, threads=threads)
+    out = out.reshape((N, T) + out.shape[1:])
+    if n_commit is None:
+        return out, S_all
+    c = np.clip(np.asarray(n_commit.cpu() if hasattr(n_commit, "cpu") else n_commit).astype(np.int64), 0, T)
+    # the first c[n] tokens of sequence n, packed
+    idx = np.concatenate([n * T + np.arange(c[n]) for n in range(N)]).astype(np.int64)
+    cu_c = np.concatenate([[0], np.cumsum(c)]).astype(np.int64)
+    pick = lambda x: flat(x)[idx]
+    _, S_c = recurrent(pick(q), pick(k), pick(v), pick(g), pick(beta), S0=S, cu_seqlens=cu_c,
+                       scale=scale, l2norm=l2norm, threads=threads)
+    return out, S_c

@@ -119,6 +119,34 @@ def test_decode_with_no_sequences_is_a_no_op(L):
     assert _decode(L, N=0) == gdn.GDN_OK
 
 
+def _decode_multi(L, **over):
+    a = dict(q=A, k=A + 0x1000, v=A + 0x2000, g=A + 0x3000, beta=A + 0x4000, S=A + 0x5000,
+             out=A + 0x6000, commit=None, N=4, T=4, H_qk=2, H_v=4, dk=128, dv=128, dtype=1,
+             scale=1.0, flags=0)
+    a.update(over)
+    return L.gdn_decode_multi(P(a["q"]), P(a["k"]), P(a["v"]), P(a["g"]), P(a["beta"]),
+                              P(a["S"]), P(a["out"]), P(a["commit"]), a["N"], a["T"], a["H_qk"],
+                              a["H_v"], a["dk"], a["dv"], a["dtype"], a["scale"], a["flags"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(T=0), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(T=9), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(S=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(commit=A + 0x7002), gdn.GDN_ERR_INVALID_ARG),     # int32 array, 2-byte aligned
+    (dict(v=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=-2), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H_v=3), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dv=96), gdn.GDN_ERR_UNSUPPORTED),
+])
+def test_decode_multi_rejects_on_host(L, over, expect):
+    assert _decode_multi(L, **over) == expect
+
+
+def test_decode_multi_with_no_sequences_is_a_no_op(L):
+    assert _decode_multi(L, N=0) == gdn.GDN_OK
+
+
 def test_get_device_error_rejects_null(L):
     assert L.gdn_get_device_error(None, None) == gdn.GDN_ERR_INVALID_ARG
 

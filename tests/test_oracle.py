@@ -342,6 +342,36 @@ def test_decode_step_is_one_token_recurrence():
     assert np.array_equal(o, o2) and np.array_equal(S, S2)
 
 
+def test_decode_multi_against_brute_force():
+    """Multi-token decode: outputs over all T tokens and the state committed after c of
+    them, against the exact brute force (two sequences, one head, c = 2 and c = 0)."""
+    rng = np.random.default_rng(43)
+    T, dk, dv = 4, 3, 2
+    seqs, commits = [], [2, 0]
+    for _ in range(2):
+        k = [[_rand_frac(rng, -1, 1) for _ in range(dk)] for _ in range(T)]
+        v = [[_rand_frac(rng, -2, 2) for _ in range(dv)] for _ in range(T)]
+        q = [[_rand_frac(rng, -1, 1) for _ in range(dk)] for _ in range(T)]
+        alpha = [F(int(rng.integers(1, 16)), 16) for _ in range(T)]
+        beta = [F(int(rng.integers(1, 16)), 16) for _ in range(T)]
+        S0 = [[_rand_frac(rng, -1, 1) for _ in range(dv)] for _ in range(dk)]
+        seqs.append((q, k, v, alpha, beta, S0))
+    fl = lambda x: np.array(x, dtype=np.float64)
+    Q = np.stack([fl(s[0]) for s in seqs])[:, :, None]          # [N, T, 1, dk]
+    K = np.stack([fl(s[1]) for s in seqs])[:, :, None]
+    V = np.stack([fl(s[2]) for s in seqs])[:, :, None]
+    G = np.log(np.stack([fl(s[3]) for s in seqs]))[:, :, None]
+    B = np.stack([fl(s[4]) for s in seqs])[:, :, None]
+    S0 = np.stack([fl(s[5]) for s in seqs])[:, None]            # [N, 1, dk, dv]
+    out, S = oracle.decode_multi(Q, K, V, G, B, S0, n_commit=np.array(commits))
+    for n, (q, k, v, alpha, beta, s0) in enumerate(seqs):
+        outs, states = brute.step_matrices(q, k, v, alpha, beta, s0)
+        ref_o = np.array([[float(x) for x in o] for o in outs])
+        assert rel_err(out[n, :, 0], ref_o) < 1e-12
+        ref_S = states[commits[n] - 1] if commits[n] > 0 else s0
+        assert rel_err(S[n, 0], np.array([[float(x) for x in r] for r in ref_S])) < 1e-12
+
+
 def test_rejects_bad_sizes():
     c = rand_case(np.random.default_rng(42), 5, 2, 3, 4, 4)      # H_v not a multiple of H_qk
     with pytest.raises(ValueError):
