@@ -56,6 +56,10 @@ typedef enum {
 #define GDN_FLAG_QK_L2NORM 1u
 /* Prefill: use the CUDA-core chunked kernel even where the tensor-core one applies. */
 #define GDN_FLAG_FORCE_CUDA_CORE 2u
+/* g and beta hold unconstrained logits a, b instead of the gates themselves: the
+ * kernels form g = -softplus(a) (so alpha = exp(g) lies in (0, 1)) and
+ * beta = sigmoid(b) (in (0, 1)) as they load them, in fp32. */
+#define GDN_FLAG_GATE_LOGITS 4u
 
 /* Bytes of device workspace gdn_prefill needs for these sizes (at least 256).
  * The workspace holds the device error word; it must be zero-filled before its

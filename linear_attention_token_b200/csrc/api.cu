@@ -10,23 +10,23 @@
 namespace gdn {
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *S, void *out, int N, int H_qk, int H_v,
-                          int dk, int dv, gdn_dtype dtype, float scale, int l2norm,
+                          int dk, int dv, gdn_dtype dtype, float scale, int opts,
                           cudaStream_t stream);
 cudaError_t launch_prefill_cc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *S0, void *out, float *S_final,
                               const int32_t *cu, int N, long long T, int H_qk, int H_v, int dk,
-                              int dv, gdn_dtype dtype, float scale, int l2norm,
+                              int dv, gdn_dtype dtype, float scale, int opts,
                               cudaStream_t stream);
 bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype);
 cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *v, const float *g,
                                       const float *beta, const float *S0, void *out, float *S_final,
                                       const int32_t *cu, int N, long long T_dense, long long T_total,
-                                      int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
+                                      int H_qk, int H_v, float scale, int opts, DeviceError *err,
                                       cudaStream_t stream);
 cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, float *S, void *out, const int32_t *n_commit,
                                 int N, int T, int H_qk, int H_v, int dk, int dv, gdn_dtype dtype,
-                                float scale, int l2norm, cudaStream_t stream);
+                                float scale, int opts, cudaStream_t stream);
 size_t static_scratch_capacity();
 cudaError_t static_scratch_ptr(void **out);
 }  // namespace gdn
@@ -35,6 +35,12 @@ namespace {
 
 constexpr size_t kWorkspaceBytes = 256;
 
+// per-call options for the kernels (common.cuh)
+int options_of(uint32_t flags)
+{
+    return ((flags & GDN_FLAG_QK_L2NORM) ? gdn::kOptL2Norm : 0) |
+           ((flags & GDN_FLAG_GATE_LOGITS) ? gdn::kOptGateLogits : 0);
+}
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool head_dim_ok(int32_t d) { return d == 64 || d == 128; }
 
@@ -49,7 +55,8 @@ gdn_status common_checks(const void *q, const void *k, const void *v, const floa
     if (H_qk <= 0 || H_v <= 0 || H_v % H_qk != 0) return GDN_ERR_INVALID_ARG;
     if (dk <= 0 || dv <= 0) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
-    if (flags & ~(GDN_FLAG_QK_L2NORM | GDN_FLAG_FORCE_CUDA_CORE)) return GDN_ERR_INVALID_ARG;
+    if (flags & ~(GDN_FLAG_QK_L2NORM | GDN_FLAG_FORCE_CUDA_CORE | GDN_FLAG_GATE_LOGITS))
+        return GDN_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
         return GDN_ERR_INVALID_ARG;
     if (!aligned(g, 4) || !aligned(beta, 4)) return GDN_ERR_INVALID_ARG;
@@ -102,7 +109,7 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, cons
         }
         return GDN_OK;
     }
-    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    const int l2 = options_of(flags);
     cudaError_t e;
     if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
         e = gdn::launch_prefill_tc_cluster(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
@@ -129,7 +136,7 @@ GDN_API gdn_status gdn_decode_step(const void *q, const void *k, const void *v, 
     if ((N > 0 && !S_inout) || !aligned(S_inout, 16)) return GDN_ERR_INVALID_ARG;
     if ((long long)N * H_v > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     if (N == 0) return GDN_OK;
-    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    const int l2 = options_of(flags);
     cudaError_t e = gdn::launch_decode(q, k, v, g, beta, S_inout, out, N, H_qk, H_v, dk, dv,
                                        dtype, scale, l2, stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
@@ -149,7 +156,7 @@ GDN_API gdn_status gdn_decode_multi(const void *q, const void *k, const void *v,
         return GDN_ERR_INVALID_ARG;
     if ((long long)N * H_v > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     if (N == 0) return GDN_OK;
-    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    const int l2 = options_of(flags);
     cudaError_t e = gdn::launch_decode_multi(q, k, v, g, beta, S_inout, out, n_commit, N, T,
                                              H_qk, H_v, dk, dv, dtype, scale, l2, stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
@@ -199,7 +206,7 @@ GDN_API gdn_status gdn_prefill_static_scratch(const void *q, const void *k, cons
     // the error word must start at zero; earlier calls may have left one behind
     if (cudaMemsetAsync(scratch, 0, sizeof(gdn::DeviceError), stream) != cudaSuccess)
         return GDN_ERR_CUDA;
-    const int l2 = (flags & GDN_FLAG_QK_L2NORM) ? 1 : 0;
+    const int l2 = options_of(flags);
     cudaError_t e;
     if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
         e = gdn::launch_prefill_tc_cluster(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,

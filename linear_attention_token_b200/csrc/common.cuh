@@ -29,6 +29,22 @@ __device__ __forceinline__ void record_error(DeviceError *err, int status, int w
     }
 }
 
+// Per-call options the host packs into one int for every kernel.
+constexpr int kOptL2Norm = 1;       // L2-normalise q and k per (token, head) in the kernel
+constexpr int kOptGateLogits = 2;   // g and beta hold logits: g = -softplus(a), beta = sigmoid(b)
+
+// Gate prologue (GDN_FLAG_GATE_LOGITS): the decay gate alpha = exp(g) must lie in (0, 1)
+// and the write strength beta in (0, 1) ("論文解説: Qwen3.8-Next の設計", section "GDNの中身",
+// the text under Eq. (1)); from unconstrained logits, g = -softplus(a) and beta = sigmoid(b).
+// softplus is evaluated as max(a, 0) + log1p(exp(-|a|)), which neither overflows nor loses
+// the small values.
+__device__ __forceinline__ float gate_log_decay(float x, int opts) {
+    return (opts & kOptGateLogits) ? -(fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)))) : x;
+}
+__device__ __forceinline__ float gate_strength(float x, int opts) {
+    return (opts & kOptGateLogits) ? 1.f / (1.f + expf(-x)) : x;
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -22,7 +22,7 @@ template <int DK, int DV, typename TIn>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                    const float *__restrict__ g, const float *__restrict__ beta, float *S,
-                   TIn *__restrict__ out, int H_qk, int H_v, float scale, int l2norm)
+                   TIn *__restrict__ out, int H_qk, int H_v, float scale, int opts)
 {
     constexpr int NT = 256;
     constexpr int TPR = DV / 4;        // threads per state row
@@ -62,7 +62,7 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
 #pragma unroll
     for (int w = 0; w < DK / 32; ++w) { skk += dots[0][w]; sqq += dots[1][w]; skq += dots[2][w]; }
     float rk = 1.f, rq = 1.f;
-    if (l2norm) {
+    if (opts & kOptL2Norm) {
         rk = rsqrtf(skk + 1e-6f);
         rq = rsqrtf(sqq + 1e-6f);
         skq *= rk * rq;
@@ -82,8 +82,8 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     __syncthreads();
 
     // 4. per value column: u, o
-    const float alpha = expf(g[nh]);
-    const float bt = beta[nh];
+    const float alpha = expf(gate_log_decay(g[nh], opts));
+    const float bt = gate_strength(beta[nh], opts);
     if (tid < DV) {
         float a = 0.f, b = 0.f;
 #pragma unroll
@@ -113,28 +113,28 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
 template <int DK, int DV, typename TIn>
 static cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const float *g,
                                    const float *beta, float *S, void *out, int N, int H_qk,
-                                   int H_v, float scale, int l2norm, cudaStream_t stream)
+                                   int H_v, float scale, int opts, cudaStream_t stream)
 {
     const long long blocks = (long long)N * H_v;
     if (blocks == 0) return cudaSuccess;
     decode_step_kernel<DK, DV, TIn><<<(unsigned)blocks, 256, 0, stream>>>(
         (const TIn *)q, (const TIn *)k, (const TIn *)v, g, beta, S, (TIn *)out, H_qk, H_v,
-        scale, l2norm);
+        scale, opts);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *S, void *out, int N, int H_qk, int H_v,
-                          int dk, int dv, gdn_dtype dtype, float scale, int l2norm,
+                          int dk, int dv, gdn_dtype dtype, float scale, int opts,
                           cudaStream_t stream)
 {
 #define GDN_DECODE_CASE(DK, DV)                                                                \
     if (dk == DK && dv == DV) {                                                                \
         return dtype == GDN_BF16                                                               \
                    ? launch_decode_t<DK, DV, __nv_bfloat16>(q, k, v, g, beta, S, out, N, H_qk, \
-                                                            H_v, scale, l2norm, stream)        \
+                                                            H_v, scale, opts, stream)        \
                    : launch_decode_t<DK, DV, float>(q, k, v, g, beta, S, out, N, H_qk, H_v,    \
-                                                    scale, l2norm, stream);                    \
+                                                    scale, opts, stream);                    \
     }
     GDN_DECODE_CASE(128, 128)
     GDN_DECODE_CASE(64, 64)

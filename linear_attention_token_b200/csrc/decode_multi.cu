@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(256, 2)
 decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                     const float *__restrict__ g, const float *__restrict__ beta, float *S,
                     TIn *__restrict__ out, const int32_t *__restrict__ n_commit, int T, int H_qk,
-                    int H_v, int num_heads, float scale, int l2norm)
+                    int H_v, int num_heads, float scale, int opts)
 {
     constexpr int NT = 256;
     constexpr int TPR = DV / 4;
@@ -130,13 +130,14 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const 
             }
             if (lane == 0) {
                 float rk = 1.f, rq = 1.f;
-                if (l2norm) {
+                if (opts & kOptL2Norm) {
                     rk = rsqrtf(skk + 1e-6f);
                     rq = rsqrtf(sqq + 1e-6f);
                     skq *= rk * rq;
                 }
                 tok_s[t][0] = rk; tok_s[t][1] = rq; tok_s[t][2] = skq;
-                tok_s[t][3] = expf(tg[buf * MT + t]); tok_s[t][4] = tb[buf * MT + t];
+                tok_s[t][3] = expf(gate_log_decay(tg[buf * MT + t], opts));
+                tok_s[t][4] = gate_strength(tb[buf * MT + t], opts);
             }
         }
         // every thread has its slice of the state: the buffer takes the next head's
@@ -199,7 +200,7 @@ template <int DK, int DV, typename TIn>
 static cudaError_t launch_decode_multi_t(const void *q, const void *k, const void *v,
                                          const float *g, const float *beta, float *S, void *out,
                                          const int32_t *n_commit, int N, int T, int H_qk,
-                                         int H_v, float scale, int l2norm, cudaStream_t stream)
+                                         int H_v, float scale, int opts, cudaStream_t stream)
 {
     const long long heads = (long long)N * H_v;
     if (heads == 0) return cudaSuccess;
@@ -219,14 +220,14 @@ static cudaError_t launch_decode_multi_t(const void *q, const void *k, const voi
     const long long grid = heads < 2LL * sms ? heads : 2LL * sms;
     decode_multi_kernel<DK, DV, TIn><<<(unsigned)grid, 256, smem, stream>>>(
         (const TIn *)q, (const TIn *)k, (const TIn *)v, g, beta, S, (TIn *)out, n_commit, T,
-        H_qk, H_v, (int)heads, scale, l2norm);
+        H_qk, H_v, (int)heads, scale, opts);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, float *S, void *out, const int32_t *n_commit,
                                 int N, int T, int H_qk, int H_v, int dk, int dv, gdn_dtype dtype,
-                                float scale, int l2norm, cudaStream_t stream)
+                                float scale, int opts, cudaStream_t stream)
 {
     if (T < 1 || T > kMaxDecodeTokens) return cudaErrorInvalidValue;
 #define GDN_DECODE_MULTI_CASE(DK, DV)                                                         \
@@ -234,9 +235,9 @@ cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, con
         return dtype == GDN_BF16                                                              \
                    ? launch_decode_multi_t<DK, DV, __nv_bfloat16>(q, k, v, g, beta, S, out,   \
                                                                   n_commit, N, T, H_qk, H_v,  \
-                                                                  scale, l2norm, stream)      \
+                                                                  scale, opts, stream)      \
                    : launch_decode_multi_t<DK, DV, float>(q, k, v, g, beta, S, out, n_commit, \
-                                                          N, T, H_qk, H_v, scale, l2norm,     \
+                                                          N, T, H_qk, H_v, scale, opts,     \
                                                           stream);                            \
     }
     GDN_DECODE_MULTI_CASE(128, 128)

@@ -48,7 +48,7 @@ prefill_cc_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
                   const float *__restrict__ g, const float *__restrict__ beta,
                   const float *S0, TIn *__restrict__ out, float *S_final,
                   const int32_t *__restrict__ cu_seqlens, long long T_dense, int H_qk, int H_v,
-                  int DV, float scale, int l2norm)
+                  int DV, float scale, int opts)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     CcSmem<DK> &sm = *reinterpret_cast<CcSmem<DK> *>(smem_raw);
@@ -90,7 +90,7 @@ prefill_cc_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
                 ss_k += kv * kv;
                 ss_q += qv * qv;
             }
-            if (l2norm) {
+            if (opts & kOptL2Norm) {
                 const float rk = rsqrtf(warp_sum(ss_k) + 1e-6f), rq = rsqrtf(warp_sum(ss_q) + 1e-6f);
                 for (int d = lane; d < DK; d += 32) { sm.K[i][d] *= rk; sm.Q[i][d] *= rq; }
             }
@@ -98,8 +98,8 @@ prefill_cc_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TI
         }
         if (tid < CC_C) {
             const bool valid = tid < L;
-            sm.g[tid] = valid ? g[(size_t)(c0 + tid) * H_v + h] : 0.f;
-            sm.b[tid] = valid ? beta[(size_t)(c0 + tid) * H_v + h] : 0.f;
+            sm.g[tid] = valid ? gate_log_decay(g[(size_t)(c0 + tid) * H_v + h], opts) : 0.f;
+            sm.b[tid] = valid ? gate_strength(beta[(size_t)(c0 + tid) * H_v + h], opts) : 0.f;
         }
         __syncthreads();
 
@@ -255,7 +255,7 @@ template <int DK, typename TIn>
 static cudaError_t launch_cc_t(const void *q, const void *k, const void *v, const float *g,
                                const float *beta, const float *S0, void *out, float *S_final,
                                const int32_t *cu, int N, long long T, int H_qk, int H_v, int dv,
-                               float scale, int l2norm, cudaStream_t stream)
+                               float scale, int opts, cudaStream_t stream)
 {
     const size_t smem = sizeof(CcSmem<DK>);
     cudaError_t e = cudaFuncSetAttribute(prefill_cc_kernel<DK, TIn>,
@@ -264,25 +264,25 @@ static cudaError_t launch_cc_t(const void *q, const void *k, const void *v, cons
     dim3 grid((unsigned)N, (unsigned)H_v, (unsigned)(dv / CC_BV));
     prefill_cc_kernel<DK, TIn><<<grid, CC_NT, smem, stream>>>(
         (const TIn *)q, (const TIn *)k, (const TIn *)v, g, beta, S0, (TIn *)out, S_final, cu, T,
-        H_qk, H_v, dv, scale, l2norm);
+        H_qk, H_v, dv, scale, opts);
     return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_cc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *S0, void *out, float *S_final,
                               const int32_t *cu, int N, long long T, int H_qk, int H_v, int dk,
-                              int dv, gdn_dtype dtype, float scale, int l2norm,
+                              int dv, gdn_dtype dtype, float scale, int opts,
                               cudaStream_t stream)
 {
     if (N == 0) return cudaSuccess;
     if (dk == 128)
         return dtype == GDN_BF16
-                   ? launch_cc_t<128, __nv_bfloat16>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, l2norm, stream)
-                   : launch_cc_t<128, float>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, l2norm, stream);
+                   ? launch_cc_t<128, __nv_bfloat16>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, opts, stream)
+                   : launch_cc_t<128, float>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, opts, stream);
     if (dk == 64)
         return dtype == GDN_BF16
-                   ? launch_cc_t<64, __nv_bfloat16>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, l2norm, stream)
-                   : launch_cc_t<64, float>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, l2norm, stream);
+                   ? launch_cc_t<64, __nv_bfloat16>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, opts, stream)
+                   : launch_cc_t<64, float>(q, k, v, g, beta, S0, out, S_final, cu, N, T, H_qk, H_v, dv, scale, opts, stream);
     return cudaErrorInvalidValue;
 }
 

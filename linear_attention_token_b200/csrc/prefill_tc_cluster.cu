@@ -200,7 +200,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const float *__restrict__ beta, const float *S0,
                           __nv_bfloat16 *__restrict__ out, float *S_final,
                           const int32_t *__restrict__ cu_seqlens, long long T_dense, int H_qk,
-                          int H_v, float scale, DeviceError *err, uint32_t budget)
+                          int H_v, float scale, int opts, DeviceError *err, uint32_t budget)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -458,8 +458,8 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         auto fetch_vectors = [&](int c) {                // g, beta of chunk c into registers
             const long long t0 = t_begin + (long long)c * K4_C;
             const int L = (int)min((long long)K4_C, t_end - t0);
-            pre_g = (t < L) ? g[(size_t)(t0 + t) * H_v + h] : 0.f;
-            pre_b = (t < L) ? beta[(size_t)(t0 + t) * H_v + h] : 0.f;
+            pre_g = (t < L) ? gate_log_decay(g[(size_t)(t0 + t) * H_v + h], opts) : 0.f;
+            pre_b = (t < L) ? gate_strength(beta[(size_t)(t0 + t) * H_v + h], opts) : 0.f;
         };
         auto finish_vectors = [&](int c) {               // G, gamma, decay-to-end; then signal
             float *cv = cvec0 + (c & 1) * 320;
@@ -605,8 +605,8 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         auto fetch_gb = [&](int pp) {
             const long long tt = t_begin + (long long)pp * K4_C;
             const int LL = (int)min((long long)K4_C, t_end - tt);
-            nxt_g = (t < LL) ? g[(size_t)(tt + t) * H_v + h] : 0.f;
-            nxt_b = (t < LL) ? beta[(size_t)(tt + t) * H_v + h] : 0.f;
+            nxt_g = (t < LL) ? gate_log_decay(g[(size_t)(tt + t) * H_v + h], opts) : 0.f;
+            nxt_b = (t < LL) ? gate_strength(beta[(size_t)(tt + t) * H_v + h], opts) : 0.f;
         };
         if ((int)r < nch && t < K4_C) fetch_gb((int)r);
 #pragma unroll 1
@@ -1070,7 +1070,7 @@ bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype)
 cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *v, const float *g,
                                       const float *beta, const float *S0, void *out, float *S_final,
                                       const int32_t *cu, int N, long long T_dense, long long T_total,
-                                      int H_qk, int H_v, float scale, int l2norm, DeviceError *err,
+                                      int H_qk, int H_v, float scale, int opts, DeviceError *err,
                                       cudaStream_t stream)
 {
     if (T_total >= (1LL << 31) || (long long)N * 4 > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -1089,10 +1089,10 @@ cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *
         attr_set = true;
     }
     dim3 grid((unsigned)(4 * N), (unsigned)H_v);
-    auto kern = l2norm ? prefill_tc_cluster_kernel<true> : prefill_tc_cluster_kernel<false>;
+    auto kern = (opts & kOptL2Norm) ? prefill_tc_cluster_kernel<true> : prefill_tc_cluster_kernel<false>;
     kern<<<grid, K4_THREADS, K4_SMEM, stream>>>(
         mq, mk, mv, g, beta, S0, (__nv_bfloat16 *)out, S_final, cu, T_dense, H_qk, H_v, scale,
-        err, wait_budget4());
+        opts, err, wait_budget4());
     return cudaGetLastError();
 }
 

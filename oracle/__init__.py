@@ -173,3 +173,14 @@ def decode_multi(q, k, v, g, beta, S, n_commit=None, scale: float = 1.0, l2norm:
     _, S_c = recurrent(pick(q), pick(k), pick(v), pick(g), pick(beta), S0=S, cu_seqlens=cu_c,
                        scale=scale, l2norm=l2norm, threads=threads)
     return out, S_c
+
+
+def gates_from_logits(a, b):
+    """Gate prologue: from unconstrained logits, the decay gate's log g = -softplus(a)
+    (so alpha = exp(g) lies in (0, 1)) and the write strength beta = sigmoid(b) (in
+    (0, 1)) -- the ranges stated under Eq. (1) of "論文解説: Qwen3.8-Next の設計",
+    section "GDNの中身".  fp64; returns numpy (g, beta)."""
+    a = _arr(a, np.float64)
+    b = _arr(b, np.float64)
+    e = np.exp(-np.abs(b))                      # in (0, 1]: no overflow on either side
+    return -np.logaddexp(0.0, a), np.where(b >= 0, 1.0 / (1.0 + e), e / (1.0 + e))

@@ -372,6 +372,40 @@ def test_decode_multi_against_brute_force():
         assert rel_err(S[n, 0], np.array([[float(x) for x in r] for r in ref_S])) < 1e-12
 
 
+def test_gates_from_logits_closed_forms():
+    """softplus(0) = ln 2 and sigmoid(0) = 1/2; softplus(a) -> a for large a and -> e^a
+    for very negative a (no overflow, no loss of the small value); both gates inside
+    (0, 1) over the whole range."""
+    a = np.array([0.0, 40.0, -40.0, 800.0, -800.0, 1.5])
+    g, beta = oracle.gates_from_logits(a, a)
+    assert g[0] == -np.log(2.0) and beta[0] == 0.5
+    assert abs(g[1] + 40.0) < 1e-15 and abs(g[2] + np.exp(-40.0)) < 1e-30
+    assert g[3] == -800.0 and abs(g[4]) < 1e-300
+    assert abs(g[5] + np.log1p(np.exp(1.5))) < 1e-15
+    assert abs(beta[5] - 1.0 / (1.0 + np.exp(-1.5))) < 1e-15
+    alpha = np.exp(g)
+    assert np.all((alpha > 0) | (g < -700)) and np.all(alpha <= 1) and np.all((beta >= 0) & (beta <= 1))
+
+
+def test_gate_logits_zero_is_half_against_brute_force():
+    """Zero logits give alpha = beta = 1/2 exactly; the recurrence fed through the gate
+    prologue then matches the exact brute force with alpha = beta = 1/2."""
+    rng = np.random.default_rng(47)
+    T, dk, dv = 6, 3, 2
+    k = [[_rand_frac(rng, -1, 1) for _ in range(dk)] for _ in range(T)]
+    v = [[_rand_frac(rng, -2, 2) for _ in range(dv)] for _ in range(T)]
+    q = [[_rand_frac(rng, -1, 1) for _ in range(dk)] for _ in range(T)]
+    S0 = [[_rand_frac(rng, -1, 1) for _ in range(dv)] for _ in range(dk)]
+    half = [F(1, 2)] * T
+    outs, states = brute.step_matrices(q, k, v, half, half, S0)
+    g, beta = oracle.gates_from_logits(np.zeros((T, 1)), np.zeros((T, 1)))
+    fl = lambda x: np.array(x, dtype=np.float64)
+    out, S = oracle.recurrent(fl(q)[:, None], fl(k)[:, None], fl(v)[:, None], g, beta,
+                              S0=fl(S0)[None, None])
+    assert rel_err(out[:, 0], np.array([[float(x) for x in o] for o in outs])) < 1e-12
+    assert rel_err(S[0, 0], np.array([[float(x) for x in r] for r in states[-1]])) < 1e-12
+
+
 def test_rejects_bad_sizes():
     c = rand_case(np.random.default_rng(42), 5, 2, 3, 4, 4)      # H_v not a multiple of H_qk
     with pytest.raises(ValueError):
