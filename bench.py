@@ -280,6 +280,30 @@ def time_decode_multi(gdn, w, T, passes, warmup, stream, device):
     return [a.elapsed_time(b) for a, b in evs], len(xs)
 
 
+def time_backward(gdn, x, w, steps, warmup, stream):
+    """gdn_backward on the prefill workload (d_out random, no dS_final), device-timed."""
+    B, T = len(w.seq_lens), w.seq_lens[0]
+    view = lambda t: t.view(B, T, *t.shape[1:])
+    gen = torch.Generator(device="cpu").manual_seed(inputs.BASE_SEED + 99)
+    d_out = torch.randn(x["v"].shape, generator=gen).to(w.dtype).to(x["v"].device)
+    args = [view(x[n]) for n in ("q", "k", "v", "g", "beta")] + [view(d_out)]
+    ws = torch.empty(int(gdn.lib().gdn_backward_workspace_size(B, B * T, w.H_v, w.dk, w.dv)),
+                     dtype=torch.uint8, device=d_out.device)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            gdn.gdn_backward(*args, workspace=ws, stream=stream)
+    stream.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            a.record(stream)
+            gdn.gdn_backward(*args, workspace=ws, stream=stream)
+            b.record(stream)
+    stream.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
 def cpu_baseline_prefill(w, max_tokens=None):
     """The oracle (float variant, all host cores) on the prefill workload, timed."""
     import oracle
@@ -376,6 +400,9 @@ def run_ours(args):
         vtimes, v_calls = time_decode_multi(gdn, wd, VERIFY_T, dec_passes, max(1, min(args.warmup, 3)),
                                             stream, device)
         barrier(world)
+        bw_steps = max(1, min(args.steps, 3))
+        btimes = time_backward(gdn, x, wp, bw_steps, 1, stream)
+        barrier(world)
     clocks = clk.summary()
     if status != 0:
         raise RuntimeError(f"device error after prefill: {gdn.gdn_status_string(status)}")
@@ -394,6 +421,7 @@ def run_ours(args):
     ms_dec_step = ms_decode_pass / wd.decode_steps
     dec_bytes = decode_bytes_per_step(wd)
     ms_verify_pass = max_over_ranks(sum(vtimes) / len(vtimes), world)
+    ms_bw = max_over_ranks(sum(btimes) / len(btimes), world)
     ver_bytes = decode_multi_bytes_per_call(wd, VERIFY_T)
     ver_gbs = ver_bytes / (ms_verify_pass / v_calls * 1e-3) / 1e9
     ver_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode_multi.cu")
@@ -443,11 +471,17 @@ def run_ours(args):
                          "peak_source": f"{peaks['source']} copy bandwidth",
                          "algorithmic_bytes_per_launch": ver_bytes},
         },
+        "backward": {
+            "workload": wp.name, "value": world * tok / (ms_bw * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms_bw, "steps": bw_steps,
+            "kernel": "backward_kernel: exact sequential reverse pass, checkpoint every 64 "
+                      "tokens, CUDA cores; bound by the per-head token chain",
+        },
         "e2e": {"value": world * tok / (ms_e2e * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "gdn_prefill via the C ABI; pinned host inputs copied in and outputs + "
                         "final state copied out inside the timed region"},
-        "gpu_launches": args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls,
+        "gpu_launches": args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls + bw_steps,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

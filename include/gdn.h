@@ -135,6 +135,36 @@ gdn_status gdn_decode_multi(const void *q, const void *k, const void *v, const f
                             int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype, float scale,
                             uint32_t flags, cudaStream_t stream);
 
+/* Backward pass: gradients of a loss L with respect to q, k, v, g, beta and S0, given
+ * d_out = dL/d out and dS_final = dL/d S_final, for the computation gdn_prefill performs
+ * (same inputs, layouts, varlen and GVA rules, scale and flags).
+ * Reverse-mode differentiation of Eq. (1) token by token; exact (no chunked
+ * re-association), with the state checkpointed every 64 tokens in the workspace and each
+ * chunk recomputed from its checkpoint.
+ *
+ *   d_out            : like out ([.., T, H_v, dv], dtype)
+ *   dS_final         : [N, H_v, dk, dv] fp32 or NULL (= 0)
+ *   dq, dk           : [.., T, H_qk, dk] fp32 (value heads sharing a q/k head are summed)
+ *   dv               : [.., T, H_v, dv] fp32
+ *   dg, dbeta        : [.., T, H_v] fp32; with GDN_FLAG_GATE_LOGITS the gradients with
+ *                      respect to the logits passed in g and beta
+ *   dS0              : [N, H_v, dk, dv] fp32 or NULL (not computed)
+ *   workspace        : device scratch of at least gdn_backward_workspace_size bytes,
+ *                      16-byte aligned, no initial contents required
+ * The library zero-fills dq, dk, dg, dbeta itself (they are accumulated with atomic adds;
+ * their summation order, and so their last bits, may vary from run to run).  dv % 32 == 0.
+ * GDN_ERR_UNSUPPORTED with GDN_FLAG_QK_L2NORM.  Nothing to do when T_total == 0 except
+ * dS0 = dS_final. */
+size_t gdn_backward_workspace_size(int32_t num_seqs, int64_t T_total, int32_t H_v, int32_t dk,
+                                   int32_t dv);
+gdn_status gdn_backward(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *S0, const void *d_out,
+                        const float *dS_final, float *dq, float *dk, float *dv, float *dg,
+                        float *dbeta, float *dS0, const int32_t *cu_seqlens, int32_t num_seqs,
+                        int32_t B, int64_t T, int32_t H_qk, int32_t H_v, int32_t dk_dim,
+                        int32_t dv_dim, gdn_dtype dtype, float scale, uint32_t flags,
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* gdn_prefill for callers that cannot allocate device memory: the same computation
  * and arguments, minus the workspace.  The paper has no counterpart; this is a
  * deployment convenience.  Some callers cannot call cudaMalloc (for instance code

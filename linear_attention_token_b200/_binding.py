@@ -25,7 +25,7 @@ GDN_FLAG_GATE_LOGITS = 4
 # every symbol include/gdn.h declares
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
             "gdn_get_device_error", "gdn_status_string", "gdn_prefill_static_scratch",
-            "gdn_decode_multi")
+            "gdn_decode_multi", "gdn_backward", "gdn_backward_workspace_size")
 
 _lib = None
 
@@ -60,6 +60,11 @@ def lib():
         L.gdn_decode_multi.argtypes = [P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32, I32,
                                        ctypes.c_int, F, U32, P]
         L.gdn_decode_multi.restype = ctypes.c_int
+        L.gdn_backward_workspace_size.argtypes = [I32, I64, I32, I32, I32]
+        L.gdn_backward_workspace_size.restype = SZ
+        L.gdn_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, I32, I32, I64, I32,
+                                   I32, I32, I32, ctypes.c_int, F, U32, P, SZ, P]
+        L.gdn_backward.restype = ctypes.c_int
         L.gdn_get_device_error.argtypes = [P, P]
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -207,6 +212,47 @@ def gdn_decode_multi(q, k, v, g, beta, S_inout, *, n_commit=None, out=None, scal
         dk, dv, _dtype_code(q), float(scale), int(flags), _stream(stream))
     _check(st, "gdn_decode_multi")
     return out
+
+
+def gdn_backward(q, k, v, g, beta, d_out, S0=None, dS_final=None, cu_seqlens=None, *,
+                 scale: float = 1.0, flags: int = 0, want_dS0: bool = True, workspace=None,
+                 stream=None):
+    """Gradients of a loss with respect to q, k, v, g, beta (and S0), given d_out (like out)
+    and dS_final (fp32 [N, H_v, dk, dv] or None).  Shapes and varlen form as gdn_prefill.
+
+    Returns a dict of fp32 tensors dq, dk (like q), dv (like v), dg, dbeta (like g) and
+    dS0 ([N, H_v, dk, dv], None when want_dS0 is False).
+    """
+    if cu_seqlens is not None:
+        T_total, H_qk, dk = q.shape[-3:]
+        B, T, N = 1, T_total, cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+    else:
+        if q.dim() == 4:
+            B, T, H_qk, dk = q.shape
+        else:
+            B, (T, H_qk, dk) = 1, q.shape
+        T_total, N = B * T, B
+    H_v, dv = v.shape[-2:]
+    f32 = dict(dtype=torch.float32, device=v.device)
+    grads = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32),
+             "dv": torch.empty(v.shape, **f32), "dg": torch.empty(g.shape, **f32),
+             "dbeta": torch.empty(beta.shape, **f32),
+             "dS0": torch.empty(N, H_v, dk, dv, **f32) if want_dS0 else None}
+    if workspace is None:
+        n = int(lib().gdn_backward_workspace_size(N, T_total, H_v, dk, dv))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=v.device)
+    st = lib().gdn_backward(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+        _dev(S0, "S0"), _dev(d_out, "d_out"), _dev(dS_final, "dS_final"),
+        _dev(grads["dq"], "dq"), _dev(grads["dk"], "dk"), _dev(grads["dv"], "dv"),
+        _dev(grads["dg"], "dg"), _dev(grads["dbeta"], "dbeta"), _dev(grads["dS0"], "dS0"),
+        _dev(cu_seqlens, "cu_seqlens"), N if cu_seqlens is not None else 0, B, T, H_qk, H_v,
+        dk, dv, _dtype_code(q), float(scale), int(flags), _dev(workspace, "workspace"),
+        workspace.numel(), _stream(stream))
+    _check(st, "gdn_backward")
+    return grads
 
 
 def gdn_get_device_error(workspace: torch.Tensor, stream=None) -> int:

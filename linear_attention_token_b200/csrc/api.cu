@@ -27,6 +27,13 @@ cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, con
                                 const float *beta, float *S, void *out, const int32_t *n_commit,
                                 int N, int T, int H_qk, int H_v, int dk, int dv, gdn_dtype dtype,
                                 float scale, int opts, cudaStream_t stream);
+size_t backward_workspace_bytes(int N, long long T_total, int H_v, int dk, int dv);
+cudaError_t launch_backward(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const float *S0, const void *d_out,
+                            const float *dS_final, float *dq, float *dk, float *dv, float *dg,
+                            float *dbeta, float *dS0, const int32_t *cu, int N, long long T_dense,
+                            long long T_total, int H_qk, int H_v, int dkk, int dvv,
+                            gdn_dtype dtype, float scale, int opts, void *ws, cudaStream_t stream);
 size_t static_scratch_capacity();
 cudaError_t static_scratch_ptr(void **out);
 }  // namespace gdn
@@ -159,6 +166,69 @@ GDN_API gdn_status gdn_decode_multi(const void *q, const void *k, const void *v,
     const int l2 = options_of(flags);
     cudaError_t e = gdn::launch_decode_multi(q, k, v, g, beta, S_inout, out, n_commit, N, T,
                                              H_qk, H_v, dk, dv, dtype, scale, l2, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API size_t gdn_backward_workspace_size(int32_t num_seqs, int64_t T_total, int32_t H_v,
+                                           int32_t dk, int32_t dv)
+{
+    if (num_seqs < 0 || T_total < 0 || H_v < 0 || !head_dim_ok(dk) || !head_dim_ok(dv)) return 0;
+    return gdn::backward_workspace_bytes(num_seqs, T_total, H_v, dk, dv);
+}
+
+GDN_API gdn_status gdn_backward(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const float *S0, const void *d_out,
+                                const float *dS_final, float *dq, float *dk, float *dv,
+                                float *dg, float *dbeta, float *dS0,
+                                const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
+                                int64_t T, int32_t H_qk, int32_t H_v, int32_t dk_dim,
+                                int32_t dv_dim, gdn_dtype dtype, float scale, uint32_t flags,
+                                void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    const bool has_tokens = (cu_seqlens ? (long long)T : (long long)B * T) > 0;
+    gdn_status st = common_checks(q, k, v, g, beta, d_out, H_qk, H_v, dk_dim, dv_dim, dtype,
+                                  flags, has_tokens);
+    if (st != GDN_OK) return st;
+    if (flags & GDN_FLAG_QK_L2NORM) return GDN_ERR_UNSUPPORTED;
+    if (has_tokens && (!dq || !dk || !dv || !dg || !dbeta)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(dg, 4) ||
+        !aligned(dbeta, 4))
+        return GDN_ERR_INVALID_ARG;
+    int N;
+    if (cu_seqlens) {
+        if (B != 1 || num_seqs < 0 || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+        N = num_seqs;
+    } else {
+        N = B;
+    }
+    if ((S0 && !aligned(S0, 16)) || (dS_final && !aligned(dS_final, 16)) || (dS0 && !aligned(dS0, 16)))
+        return GDN_ERR_INVALID_ARG;
+    const long long T_total = cu_seqlens ? (long long)T : (long long)B * T;
+    if ((long long)N * H_v * (dv_dim / 32) > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    const size_t need = gdn_backward_workspace_size(N, T_total, H_v, dk_dim, dv_dim);
+    if (N > 0 && T_total > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
+        return GDN_ERR_INVALID_ARG;
+    if (N == 0) return GDN_OK;
+    if (T_total == 0) {
+        if (dS0) {
+            const size_t bytes = (size_t)N * H_v * dk_dim * dv_dim * sizeof(float);
+            cudaError_t e = dS_final ? cudaMemcpyAsync(dS0, dS_final, bytes,
+                                                       cudaMemcpyDeviceToDevice, stream)
+                                     : cudaMemsetAsync(dS0, 0, bytes, stream);
+            if (e != cudaSuccess) return GDN_ERR_CUDA;
+        }
+        return GDN_OK;
+    }
+    // accumulated with atomic adds
+    cudaError_t e = cudaMemsetAsync(dq, 0, (size_t)T_total * H_qk * dk_dim * sizeof(float), stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, (size_t)T_total * H_qk * dk_dim * sizeof(float), stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dg, 0, (size_t)T_total * H_v * sizeof(float), stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, (size_t)T_total * H_v * sizeof(float), stream);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    e = gdn::launch_backward(q, k, v, g, beta, S0, d_out, dS_final, dq, dk, dv, dg, dbeta, dS0,
+                             cu_seqlens, N, cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v,
+                             dk_dim, dv_dim, dtype, scale, options_of(flags), workspace, stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -147,6 +147,41 @@ def test_decode_multi_with_no_sequences_is_a_no_op(L):
     assert _decode_multi(L, N=0) == gdn.GDN_OK
 
 
+def _backward(L, **over):
+    a = dict(q=A, k=A + 0x1000, v=A + 0x2000, g=A + 0x3000, beta=A + 0x4000, S0=None,
+             d_out=A + 0x5000, dSf=None, dq=A + 0x6000, dk=A + 0x7000, dv=A + 0x8000,
+             dg=A + 0x9000, db=A + 0xa000, dS0=None, cu=None, num_seqs=0, B=1, T=64, H_qk=2,
+             H_v=4, dk_dim=128, dv_dim=128, dtype=1, scale=1.0, flags=0, ws=A + 0xb000,
+             ws_bytes=1 << 40)
+    a.update(over)
+    return L.gdn_backward(P(a["q"]), P(a["k"]), P(a["v"]), P(a["g"]), P(a["beta"]), P(a["S0"]),
+                          P(a["d_out"]), P(a["dSf"]), P(a["dq"]), P(a["dk"]), P(a["dv"]),
+                          P(a["dg"]), P(a["db"]), P(a["dS0"]), P(a["cu"]), a["num_seqs"], a["B"],
+                          a["T"], a["H_qk"], a["H_v"], a["dk_dim"], a["dv_dim"], a["dtype"],
+                          a["scale"], a["flags"], P(a["ws"]), a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(flags=gdn.GDN_FLAG_QK_L2NORM), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dq=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(db=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(d_out=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ws=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dv=A + 0x8004), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dS0=A + 0xc008), gdn.GDN_ERR_INVALID_ARG),
+    (dict(dk_dim=96), gdn.GDN_ERR_UNSUPPORTED),
+])
+def test_backward_rejects_on_host(L, over, expect):
+    assert _backward(L, **over) == expect
+
+
+def test_backward_workspace_size(L):
+    # checkpoints every 64 tokens plus one recomputed chunk, per (sequence, head, 32 columns)
+    n = gdn._binding.lib().gdn_backward_workspace_size(2, 8192, 16, 128, 128)
+    assert n == 2 * 16 * 4 * (8192 // 64 + 1 + 65) * 128 * 32 * 4
+
+
 def test_get_device_error_rejects_null(L):
     assert L.gdn_get_device_error(None, None) == gdn.GDN_ERR_INVALID_ARG
 

@@ -406,6 +406,69 @@ def test_gate_logits_zero_is_half_against_brute_force():
     assert rel_err(S[0, 0], np.array([[float(x) for x in r] for r in states[-1]])) < 1e-12
 
 
+def _fd_case(seed):
+    rng = np.random.default_rng(seed)
+    T, Hq, Hv, dk, dv = 7, 1, 2, 3, 2
+    c = dict(q=rng.normal(size=(T, Hq, dk)), k=rng.normal(size=(T, Hq, dk)) * 0.5,
+             v=rng.normal(size=(T, Hv, dv)), g=-np.abs(rng.normal(size=(T, Hv))) * 0.5,
+             beta=1 / (1 + np.exp(-rng.normal(size=(T, Hv)))),
+             S0=rng.normal(size=(2, Hv, dk, dv)) * 0.3)
+    dO = rng.normal(size=(T, Hv, dv))
+    dSf = rng.normal(size=(2, Hv, dk, dv))
+    return c, dO, dSf, np.array([0, 3, 7])
+
+
+def _fd_errors(backward_fn, seed=0, scale=0.7):
+    """Worst relative gap, per gradient, between backward_fn and central differences of
+    L = <out, dO> + <S_final, dS_final> through the forward oracle."""
+    c, dO, dSf, cu = _fd_case(seed)
+    names = ["q", "k", "v", "g", "beta", "S0"]
+
+    def L(vals):
+        o, S = oracle.recurrent(vals["q"], vals["k"], vals["v"], vals["g"], vals["beta"],
+                                S0=vals["S0"], cu_seqlens=cu, scale=scale)
+        return np.sum(o * dO) + np.sum(S * dSf)
+
+    grads = backward_fn(c["q"], c["k"], c["v"], c["g"], c["beta"], c["S0"], dO, dSf, cu,
+                        scale=scale)
+    out = []
+    for name, G in zip(names, grads):
+        A = c[name]
+        num = np.zeros_like(A)
+        for idx in np.ndindex(A.shape):
+            hi = dict(c); lo = dict(c)
+            hi[name] = A.copy(); hi[name][idx] += 1e-6
+            lo[name] = A.copy(); lo[name][idx] -= 1e-6
+            num[idx] = (L(hi) - L(lo)) / 2e-6
+        out.append(np.abs(num - G).max() / max(np.abs(num).max(), 1e-12))
+    return out
+
+
+def test_backward_matches_finite_differences():
+    """Every gradient of the backward oracle (q, k, v, g, beta, S0; two ragged sequences,
+    two value heads on one q/k head, a given S0 and dS_final) against central
+    differences of the forward oracle."""
+    from oracle.backward import backward
+    assert max(_fd_errors(backward)) < 1e-7
+
+
+@pytest.mark.parametrize("old,new", [
+    ("dal += -bt * (du @ a)", "dal += bt * (du @ a)"),            # sign of the erase term
+    ("da = -al * bt * du", "da = -bt * du"),                      # alpha dropped in da
+    ("dq[t, hq] += scale * S_t @ d_out[t, h]", "dq[t, hq] += scale * S_p @ d_out[t, h]"),
+    ("dS = dS + scale * np.outer(qt, d_out[t, h])", "dS = dS + np.outer(qt, d_out[t, h])"),
+])
+def test_backward_pins_catch_plausible_mistakes(old, new):
+    """The finite-difference pin fails for each planted mistake in the backward oracle."""
+    import inspect
+    import oracle.backward as ob
+    src = inspect.getsource(ob)
+    assert old in src
+    ns = {}
+    exec(compile(src.replace(old, new), "mutant", "exec"), ns)
+    assert max(_fd_errors(ns["backward"])) > 1e-3
+
+
 def test_rejects_bad_sizes():
     c = rand_case(np.random.default_rng(42), 5, 2, 3, 4, 4)      # H_v not a multiple of H_qk
     with pytest.raises(ValueError):
