@@ -11,8 +11,8 @@
 //   dv = beta du;  dg = alpha dalpha;  dS <- alpha dS + k da^T;  dS0 = dS at the end.
 //
 // Exact and sequential (no chunked re-association): one CTA per (sequence, value head,
-// 32-column slice of the value dimension), one thread per state row, so a thread holds
-// its row of S (and of dS) in registers.  The value columns of S evolve independently, so
+// 16-column slice of the value dimension), one thread per state row, so a thread holds
+// its row of S (and of dS) in registers; two CTAs share an SM.  The value columns of S evolve independently, so
 // the slices need no exchange; the gradients that sum over value columns (dq, dk, dalpha,
 // dbeta) are accumulated across slices and grouped value heads with atomic adds.
 //   Phase 1: the state is run forward over the sequence and stored at every chunk start
@@ -26,13 +26,14 @@ namespace gdn {
 namespace {
 
 constexpr int BW_C = 64;     // chunk (checkpoint interval)
-constexpr int BW_BV = 32;    // value columns per CTA
+constexpr int BW_BV = 16;    // value columns per CTA
 
-// 32 values per lane -> lane l holds the sum over the warp's lanes of value l (31 shuffles)
-__device__ __forceinline__ float warp_transpose_sum(float (&x)[32], int lane)
+// BW_BV values per lane -> lane l holds the sum over the warp's 32 lanes of value
+// (l mod BW_BV): halving exchanges (BW_BV - 1 shuffles), then the remaining lane halves
+__device__ __forceinline__ float warp_transpose_sum(float (&x)[BW_BV], int lane)
 {
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) {
+    for (int m = BW_BV / 2; m >= 1; m >>= 1) {
         const bool upper = (lane & m) != 0;
 #pragma unroll
         for (int i = 0; i < m; ++i) {
@@ -41,6 +42,8 @@ __device__ __forceinline__ float warp_transpose_sum(float (&x)[32], int lane)
             x[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
         }
     }
+#pragma unroll
+    for (int m = BW_BV; m < 32; m <<= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], m);
     return x[0];
 }
 
@@ -58,7 +61,7 @@ struct BwShared {
 }  // namespace
 
 template <int DK, typename TIn>
-__global__ void __launch_bounds__(DK, 1)
+__global__ void __launch_bounds__(DK, 2)
 backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                 const float *__restrict__ g, const float *__restrict__ beta, const float *S0,
                 const TIn *__restrict__ d_out, const float *dS_final, float *dq, float *dk,
@@ -113,11 +116,11 @@ backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
     // one token forward on the row in registers: returns nothing, leaves a, u in sm
     auto step_forward = [&](float (&s)[BW_BV], int i) {
         const float kr = sm.k[i][r];
-        float x[32];
+        float x[BW_BV];
 #pragma unroll
         for (int j = 0; j < BW_BV; ++j) x[j] = s[j] * kr;
         const float part = warp_transpose_sum(x, lane);
-        sm.red[warp][lane] = part;
+        if (lane < BW_BV) sm.red[warp][lane] = part;
         __syncthreads();
         if (r < BW_BV) {
             float a = 0.f;
@@ -204,10 +207,13 @@ backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             }
             atomicAdd(dq + ((size_t)t * H_qk + hq) * DK + r, dq_part);
             // du = dS^T k (over rows)
-            float x[32];
+            float x[BW_BV];
 #pragma unroll
             for (int j = 0; j < BW_BV; ++j) x[j] = dS[j] * kr;
-            sm.red[warp][lane] = warp_transpose_sum(x, lane);
+            {
+                const float part = warp_transpose_sum(x, lane);
+                if (lane < BW_BV) sm.red[warp][lane] = part;
+            }
             // this row's share of <dS, S_{t-1}>
             float dal_part = 0.f;
 #pragma unroll
@@ -233,8 +239,9 @@ backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             atomicAdd(dk + ((size_t)t * H_qk + hq) * DK + r, dk_part);
             if (warp == 0) {
                 // dbeta (slice share) = <du, v - alpha a>;  -beta <du, a> joins dalpha
-                const float du = sm.col[lane], a = sm.a[i][lane];
-                const float db = warp_sum(du * (sm.v[i][lane] - al * a));
+                const bool on = lane < BW_BV;
+                const float du = on ? sm.col[lane] : 0.f, a = on ? sm.a[i][lane] : 0.f;
+                const float db = warp_sum(on ? du * (sm.v[i][lane] - al * a) : 0.f);
                 const float da_dot = warp_sum(du * a);
                 if (lane == 0) {
                     float dal = 0.f;

@@ -177,9 +177,9 @@ def test_backward_rejects_on_host(L, over, expect):
 
 
 def test_backward_workspace_size(L):
-    # checkpoints every 64 tokens plus one recomputed chunk, per (sequence, head, 32 columns)
+    # checkpoints every 64 tokens plus one recomputed chunk, per (sequence, head, 16 columns)
     n = gdn._binding.lib().gdn_backward_workspace_size(2, 8192, 16, 128, 128)
-    assert n == 2 * 16 * 4 * (8192 // 64 + 1 + 65) * 128 * 32 * 4
+    assert n == 2 * 16 * 8 * (8192 // 64 + 1 + 65) * 128 * 16 * 4
 
 
 def test_get_device_error_rejects_null(L):
