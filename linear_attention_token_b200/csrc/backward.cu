@@ -189,12 +189,17 @@ backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             step_forward(s, i);
             store_row(my_scr + (size_t)(i + 1) * DK * BW_BV, s);
         }
-        // backward over the chunk's tokens; s holds S_t (after token i)
+        // backward over the chunk's tokens; s holds S_t (after token i).  S_{t-1} of the
+        // next (earlier) token is loaded one step ahead, so its latency hides behind a step.
+        float sp_next[BW_BV];
+        if (L > 0) load_row(my_scr + (size_t)(L - 1) * DK * BW_BV, sp_next);
 #pragma unroll 1
         for (int i = L - 1; i >= 0; --i) {
             const long long t = t0 + i;
-            float sp[BW_BV];
-            load_row(my_scr + (size_t)i * DK * BW_BV, sp);    // S_{t-1}
+            float sp[BW_BV];                                   // S_{t-1}
+#pragma unroll
+            for (int j = 0; j < BW_BV; ++j) sp[j] = sp_next[j];
+            if (i > 0) load_row(my_scr + (size_t)(i - 1) * DK * BW_BV, sp_next);
             const float al = expf(sm.g[i]), bt = sm.beta[i];
             const float qr = sm.q[i][r], kr = sm.k[i][r];
             // dS += scale q do^T ; dq_t (this slice's columns) = scale S_t do
