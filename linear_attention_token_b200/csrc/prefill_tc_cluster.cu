@@ -16,19 +16,22 @@
 //     WS = W S_r -> U_r = U~_r - WS -> S_r <- gamma_end S_r + K~^T U_r -> next chunk,
 // with Q S_r and P U_r for the outputs off that chain.  The per-chunk quantities that
 // do not depend on the value columns (P, the inverse T, W, U~) are computed once per
-// chunk, by CTA (chunk mod 4), and copied into all four CTAs' shared memory with
-// bulk DSMEM copies that complete on the receivers' mbarriers.  Each CTA therefore
-// prepares every fourth chunk, several chunks ahead of the state chain.
+// chunk, by CTA (chunk mod 4), several chunks ahead of the state chain.  They travel
+// through L2: the producer bulk-stores W, P and all four U~ slices (already in the
+// shared-memory tile layout) into the chunk's slot of a small global ring, signals the
+// four CTAs, and each bulk-loads W, P and its own slice into its two-slot ring.  (DSMEM
+// copies from one SM run at about 20 B/cycle, which capped the producer; L2 does not.)
 //
 // Roles inside a CTA (448 threads):
 //   warps 0-3    chain group:  U epilogue and state epilogue; its first thread issues
 //                              the chain's MMAs WS = W S_r and S2 = K~^T U_r; thread 32
 //                              issues PU = P U_r
 //   warps 4-7    prep group:   inputs fix-up, A/P epilogue, triangular inverse, T'/T'',
-//                              W/U~ epilogue into the send staging
-//   warp 8       chain issuer: TMA for Q, MMA QS = Q S_r (queued behind WS), ring
-//                              bookkeeping
-//   warp 9       prep issuer:  TMA for the prepared chunk, MMAs P1 ([K;Q]K^T), W, U~, sends
+//                              W/U~ epilogue into the store staging
+//   warp 8       chain issuer: TMA for Q, MMA QS = Q S_r (queued behind WS), the ring
+//                              (bulk loads of ready chunks, receipts to the producers)
+//   warp 9       prep issuer:  TMA for the prepared chunk, MMAs P1 ([K;Q]K^T), W, U~,
+//                              bulk stores into the L2 ring, ready signals
 //   warps 10-13  aux group:    per-chunk vectors, K~ build, output epilogue
 // Accumulators live in TMEM; the state slice S_r (128 x 32 fp32) stays in TMEM for the
 // whole sequence.  Every wait is bounded; a CTA whose wait runs out records

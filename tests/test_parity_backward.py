@@ -59,6 +59,7 @@ def _check(x, d_out, dSf, scale=1.0, flags=0, g=None, beta=None):
     ([150], 1, 1, 64, 64),
     ([70, 129], 2, 2, 128, 64),
     ([65, 3], 1, 2, 64, 128),
+    ([70, 0, 5, 1], 2, 2, 128, 128),          # an empty sequence passes dS_final to dS0
 ])
 def test_backward_matches_oracle(dtype, lens, H_qk, H_v, dk, dv):
     x, d_out, dSf = _case(lens, H_qk, H_v, dk, dv, dtype, seed=sum(lens) + dk + dv)
@@ -93,3 +94,17 @@ def test_backward_dense_batch_layout():
     torch.cuda.synchronize()
     for n in ("dq", "dk", "dv", "dg", "dbeta", "dS0"):
         assert err(dense[n].reshape(packed[n].shape), packed[n].double().cpu()) < 1e-6, n
+
+
+def test_backward_is_repeatable_up_to_atomics():
+    """Two calls agree to rounding: dv and dS0 bit for bit (each element has one writer),
+    the atomically accumulated dq, dk, dg, dbeta within float rounding."""
+    x, d_out, dSf = _case([150, 40], 2, 4, 128, 128, torch.bfloat16, seed=31)
+    a = gdn.gdn_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d_out, x["S0"], dSf,
+                         x["cu_seqlens"])
+    b = gdn.gdn_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d_out, x["S0"], dSf,
+                         x["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert torch.equal(a["dv"], b["dv"]) and torch.equal(a["dS0"], b["dS0"])
+    for n in ("dq", "dk", "dg", "dbeta"):
+        assert err(a[n], b[n].double().cpu()) < 1e-5, n
