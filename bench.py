@@ -453,10 +453,7 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded; q,k ~ N(0,1) L2-normalised, v ~ N(0,1), g = -softplus(N(0,1)), "
                 "beta = sigmoid(N(0,1)))",
-        "config": {"workload": wp.name, "B": len(wp.seq_lens), "T": wp.seq_lens[0],
-                   "H_qk": wp.H_qk, "H_v": wp.H_v, "dk": wp.dk, "dv": wp.dv, "chunk": CHUNK,
-                   "state": "fp32", "parallelism": f"replicas x{world}" if world > 1 else "single",
-                   "l2": "256 MB buffer written between timed prefill steps (outside the events)"},
+        "config": prefill_config(wp, world),
         "roofline": {"bound": "tensor", "achieved": pf_tflops,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": pf_tflops / peaks["bf16_tflops"],
@@ -507,6 +504,13 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+def prefill_config(wp, world):
+    return {"workload": wp.name, "B": len(wp.seq_lens), "T": wp.seq_lens[0],
+            "H_qk": wp.H_qk, "H_v": wp.H_v, "dk": wp.dk, "dv": wp.dv, "chunk": CHUNK,
+            "state": "fp32", "parallelism": f"replicas x{world}" if world > 1 else "single",
+            "l2": "256 MB buffer written between timed prefill steps (outside the events)"}
+
+
 def run_reference(args):
     """The oracle as it stands, on the host cores, on our arm's workload and metric."""
     rank = int(os.environ.get("RANK", "0"))
@@ -522,11 +526,11 @@ def run_reference(args):
     base = dict(runs[0])
     base["value"] = v
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 0,
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "device": "host cores (the oracle; no GPU work)",
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wp.name, "B": len(wp.seq_lens), "T": wp.seq_lens[0],
-                   "H_qk": wp.H_qk, "H_v": wp.H_v, "dk": wp.dk, "dv": wp.dv},
+        "config": prefill_config(wp, args.gpus),
         "cpu_baseline": base,
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
