@@ -360,7 +360,11 @@ def cpu_baseline_decode(w, steps=2):
                       f"{w.H_v} heads of {w.name}"}
 
 
-def dist_init():
+def dist_init(backend=None, timeout_s: float = 120.0):
+    """One process per GPU under torchrun (RANK / WORLD_SIZE / MASTER_* from the env):
+    NCCL on GPUs; gloo when there is no GPU (the CPU tests of this plumbing).  The
+    ranks are replicas: nothing but the barrier and the max-over-ranks timing crosses
+    between them."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world <= 1:
         return 0, 1, 0
@@ -368,26 +372,42 @@ def dist_init():
     import torch.distributed as dist
     rank = int(os.environ["RANK"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+    kwargs = {}
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+        kwargs["device_id"] = torch.device("cuda", local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kwargs)
     return rank, world, local
+
+
+def _device_sync():
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        torch.cuda.synchronize()
 
 
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    _device_sync()
 
 
 def max_over_ranks(x: float, world: int) -> float:
     if world <= 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, ms_max: float) -> float:
+    """Whole-job throughput of `world` replicas: every rank's tokens over the slowest
+    rank's time."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
 
 
 def run_ours(args):
@@ -441,7 +461,7 @@ def run_ours(args):
 
     line = {
         "metric": METRIC,
-        "value": world * tok / (ms_prefill * 1e-3),
+        "value": job_tokens_per_s(world, tok, ms_prefill),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
