@@ -837,11 +837,14 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             auto poll_ring = [&]() {
                 const int a = next_load;
                 if (a <= load_limit && a < nch &&
-                    mbar_try_wait_cluster(bars + B_READY + (a & 7), (uint32_t)((a >> 3) & 1))) {
+                    mbar_try_wait(bars + B_READY + (a & 7), (uint32_t)((a >> 3) & 1))) {
                     const int sa = a & 1;
                     const unsigned char *src = gring + (size_t)(a & 7) * K4_GCHUNK;
                     unsigned char *dst = sm + S4_RING + sa * K4_RING_BYTES;
                     uint64_t *fb = bars + (sa ? B_FULL1 : B_FULL0);
+                    // polled at CTA scope (cheap); the cluster-scope acquire that pairs with
+                    // the producer's release is this one fence, taken once the phase is seen
+                    fence_release_cluster();
                     fence_proxy_async_global();
                     mbar_arrive_expect_tx(fb, K4_RING_BYTES);
                     bulk_load_global(dst, src, 24576, fb);                          // W | P
