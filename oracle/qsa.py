@@ -106,7 +106,10 @@ def block_scores(q, q_pos: int, k_hat, rope_dims: int = ROPE_DIMS, base: float =
     k_hat = np.asarray(k_hat, np.float64)
     s = np.zeros(k_hat.shape[0], np.float64)
     for h in range(qh.shape[0]):
-        s += k_hat @ qh[h]
+        # each row's dot product by the same elementwise reduction, so that equal rows
+        # score exactly equal (a matrix-vector library call may round rows differently by
+        # position, which would break exact ties by noise)
+        s += (k_hat * qh[h]).sum(axis=1)
     return s
 
 

@@ -198,6 +198,18 @@ def check_heads_sum(Q):
     assert np.allclose(s, parts, rtol=0, atol=1e-12 * np.abs(s).max())
 
 
+def check_equal_rows_score_equal(Q):
+    """Ties are decided by block order only if equal rows score exactly equal, wherever
+    they sit in the cache."""
+    rng = np.random.default_rng(7)
+    v = rng.standard_normal(128)
+    kh = rng.standard_normal((5003, 128))
+    pos = rng.choice(5003, 700, replace=False)
+    kh[pos] = v
+    s = Q.block_scores(rng.standard_normal((4, 128)), 123457, kh)
+    assert np.unique(s[pos]).size == 1
+
+
 BATTERY = [
     ("rope_hand", check_rope_hand_values),
     ("rope_complex", check_rope_complex_form),
@@ -207,6 +219,7 @@ BATTERY = [
     ("causality", check_causality_boundary),
     ("relative_scores", check_scores_relative_form),
     ("heads_sum", check_heads_sum),
+    ("equal_rows", check_equal_rows_score_equal),
 ]
 
 
