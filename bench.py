@@ -9,7 +9,9 @@ workload (B=2, T=4096, H=16, dk=dv=128, bf16 q/k/v, fp32 g/beta/state, S0=0);
 carries the decode workload (256 sequences x 128 single-token steps, H=32,
 dk=dv=128, bf16 q/k/v, fp32 state ~ N(0, 0.02)) under "decode", the roofline of
 each kernel, the end-to-end figure through the C ABI with host buffers ("e2e"),
-and the CPU oracle timed on this host ("cpu_baseline").
+and the CPU oracle timed on this host ("cpu_baseline").  "qsa_indexer" carries the QSA
+compressed indexer: one query per sequence against 8 caches of 262,144 blocks (1,048,576
+tokens each, budget 512 blocks), and the compression of those 8,388,608 keys.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
 the launching stream; a 256 MB buffer is written between prefill steps (outside
@@ -76,6 +78,14 @@ def decode_multi_bytes_per_call(w, T: int) -> int:
     N = w.decode_seqs
     return (N * w.H_v * w.dk * w.dv * 4 * 2
             + T * (N * (2 * w.H_qk * w.dk + 2 * w.H_v * w.dv) * e + N * w.H_v * 8))
+
+
+def qsa_index_bytes(wq, blocks: int) -> int:
+    """Algorithmic bytes of one indexer call: every cached block row read once (128 bf16),
+    the queries (4 x 128 bf16 per sequence) and positions read once, the kept blocks, their
+    scores and tokens written once."""
+    N, K = wq.num_seqs, wq.budget_blocks
+    return blocks * 256 + N * (4 * 128 * 2 + 4) + N * K * (4 + 4 + 4 * 4)
 
 
 def decode_flops_per_step(w) -> int:
@@ -316,6 +326,66 @@ def time_backward(gdn, x, w, steps, warmup, stream):
     return [a.elapsed_time(b) for a, b in evs]
 
 
+def time_qsa(gdn, wq, steps, warmup, stream, device):
+    """The QSA indexer on its decode workload (8 sequences x 1,048,576 cached tokens =
+    262,144 blocks each, budget 512 blocks): each timed call is one gdn_qsa_index_decode
+    (score, threshold, collect and finish kernels).  The 512 MB block cache is larger than
+    L2, so no flush is needed between calls.  Then gdn_qsa_compress over the same
+    sequences' 8,388,608 raw keys (2.1 GB in, 0.5 GB out)."""
+    x = inputs.qsa_decode_inputs(wq, device)
+    N, nb = wq.num_seqs, x["k_hat"].shape[0]
+    ws = gdn.qsa_index_workspace(N, nb, device)
+    bi = torch.empty(N, wq.budget_blocks, dtype=torch.int32, device=device)
+    bs = torch.empty(N, wq.budget_blocks, dtype=torch.float32, device=device)
+    ti = torch.empty(N, 4 * wq.budget_blocks, dtype=torch.int32, device=device)
+
+    def call():
+        gdn.gdn_qsa_index_decode(x["q"], x["q_pos"], x["k_hat"], x["cu_blocks"],
+                                 wq.budget_blocks, workspace=ws, block_idx=bi, block_score=bs,
+                                 token_idx=ti, stream=stream)
+
+    def timed(fn, n, warm):
+        with torch.cuda.stream(stream):
+            for _ in range(warm):
+                fn()
+        stream.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for a, b in evs:
+                a.record(stream)
+                fn()
+                b.record(stream)
+        stream.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    itimes = timed(call, steps, warmup)
+    T = sum(wq.ctx_lens)
+    k = inputs.qsa_keys(T, inputs.QSA_SEED + 50, device)
+    cu = inputs.qsa_offsets(wq.ctx_lens, device)
+    k_hat = torch.empty(nb, 128, dtype=torch.bfloat16, device=device)
+    ctimes = timed(lambda: gdn.gdn_qsa_compress(k, cu, x["cu_blocks"], k_hat=k_hat,
+                                                stream=stream), max(1, min(steps, 5)), 1)
+    del k, k_hat
+    return itimes, ctimes, nb, T
+
+
+def cpu_baseline_qsa(wq, seqs=2):
+    """The oracle's indexer (float64 numpy, Python ranking) on `seqs` of the workload's
+    queries, timed on this host."""
+    from oracle import qsa as oq
+    x = inputs.qsa_decode_inputs(wq, "cpu")
+    cb = x["cu_blocks"].numpy()
+    q = x["q"][:seqs].float().numpy()
+    kh = x["k_hat"][:int(cb[seqs])].float().numpy()
+    t0 = time.perf_counter()
+    oq.index_decode(q, x["q_pos"][:seqs].numpy(), kh, cb[:seqs + 1], wq.budget_blocks)
+    dt = time.perf_counter() - t0
+    return {"value": seqs / dt, "unit": "queries/s", "cores": 1, "kind": "oracle",
+            "sample": f"{seqs} of the {wq.num_seqs} queries (262,144 blocks each), float64 "
+                      f"numpy scores and Python ranking, one thread"}
+
+
 def cpu_baseline_prefill(w, max_tokens=None):
     """The oracle (float variant, all host cores) on the prefill workload, timed."""
     import oracle
@@ -435,6 +505,10 @@ def run_ours(args):
         bw_steps = max(1, min(args.steps, 3))
         btimes = time_backward(gdn, x, wp, bw_steps, 1, stream)
         barrier(world)
+        wq = inputs.qsa_workloads()[0]
+        q_steps = max(3, min(args.steps, 20))
+        qtimes, ctimes, q_blocks, q_tokens = time_qsa(gdn, wq, q_steps, 3, stream, device)
+        barrier(world)
     clocks = clk.summary()
     if status != 0:
         raise RuntimeError(f"device error after prefill: {gdn.gdn_status_string(status)}")
@@ -458,6 +532,13 @@ def run_ours(args):
     ver_gbs = ver_bytes / (ms_verify_pass / v_calls * 1e-3) / 1e9
     ver_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode_multi.cu")
     dec_gbs = dec_bytes / (ms_dec_step * 1e-3) / 1e9
+    ms_qsa = max_over_ranks(sum(qtimes) / len(qtimes), world)
+    ms_cmp = max_over_ranks(sum(ctimes) / len(ctimes), world)
+    qsa_bytes = qsa_index_bytes(wq, q_blocks)
+    qsa_gbs = qsa_bytes / (ms_qsa * 1e-3) / 1e9
+    cmp_bytes = q_tokens * 256 + q_blocks * 256
+    cmp_gbs = cmp_bytes / (ms_cmp * 1e-3) / 1e9
+    qsa_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "qsa.cu")
 
     line = {
         "metric": METRIC,
@@ -506,17 +587,39 @@ def run_ours(args):
             "kernel": "backward_kernel: exact sequential reverse pass, checkpoint every 64 "
                       "tokens, CUDA cores; bound by the per-head token chain",
         },
+        "qsa_indexer": {
+            "workload": wq.name, "value": world * wq.num_seqs / (ms_qsa * 1e-3),
+            "unit": "queries/s", "ms_per_call": ms_qsa, "calls": len(qtimes),
+            "budget_blocks": wq.budget_blocks, "cached_blocks": q_blocks,
+            "roofline": {"bound": "hbm", "achieved": qsa_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": qsa_gbs / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic("qsa_score", qsa_src),
+                         "peak_source": f"{peaks['source']} copy bandwidth",
+                         "algorithmic_bytes_per_launch": qsa_bytes,
+                         "timed": "the whole gdn_qsa_index_decode call (4 kernels); the score "
+                                  "kernel is the dominant one"},
+            "compress": {
+                "workload": f"{wq.num_seqs} x {wq.ctx_lens[0]} raw keys -> {q_blocks} blocks",
+                "value": world * q_tokens / (ms_cmp * 1e-3), "unit": "tokens/s",
+                "ms_per_call": ms_cmp, "calls": len(ctimes),
+                "roofline": {"bound": "hbm", "achieved": cmp_gbs, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": cmp_gbs / peaks["hbm_gbs"],
+                             "traffic": profiled_traffic("qsa_compress", qsa_src),
+                             "algorithmic_bytes_per_launch": cmp_bytes}},
+        },
         "e2e": {"value": world * tok / (ms_e2e * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "gdn_prefill via the C ABI; every step's pinned host inputs copied in and "
                         "outputs + final state copied out inside the timed region; consecutive "
                         "steps alternate two streams so copies overlap"},
-        "gpu_launches": args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls + bw_steps,
+        "gpu_launches": (args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls + bw_steps
+                         + 4 * len(qtimes) + len(ctimes)),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_prefill(wp)
         line["decode"]["cpu_baseline"] = cpu_baseline_decode(wd)
+        line["qsa_indexer"]["cpu_baseline"] = cpu_baseline_qsa(wq)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

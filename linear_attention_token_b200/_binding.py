@@ -1,4 +1,4 @@
-"""ctypes binding of libgdn (include/gdn.h): argument marshalling only.
+"""ctypes binding of libgdn (include/gdn.h, include/qsa.h): argument marshalling only.
 
 Every step of the gated delta rule runs in libgdn's CUDA kernels; this module
 passes torch device pointers, sizes and the current CUDA stream through the C ABI
@@ -22,10 +22,15 @@ GDN_FLAG_QK_L2NORM = 1
 GDN_FLAG_FORCE_CUDA_CORE = 2
 GDN_FLAG_GATE_LOGITS = 4
 
-# every symbol include/gdn.h declares
+# QSA indexer constants (include/qsa.h)
+GDN_QSA_R, GDN_QSA_DIM, GDN_QSA_ROPE_DIMS, GDN_QSA_HEADS = 4, 128, 64, 4
+GDN_QSA_MAX_BUDGET, GDN_QSA_MAX_SEQS = 4096, 4096
+
+# every symbol include/gdn.h and include/qsa.h declare
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
             "gdn_get_device_error", "gdn_status_string", "gdn_prefill_static_scratch",
-            "gdn_decode_multi", "gdn_backward", "gdn_backward_workspace_size")
+            "gdn_decode_multi", "gdn_backward", "gdn_backward_workspace_size",
+            "gdn_qsa_compress", "gdn_qsa_index_workspace_size", "gdn_qsa_index_decode")
 
 _lib = None
 
@@ -65,6 +70,12 @@ def lib():
         L.gdn_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, I32, I32, I64, I32,
                                    I32, I32, I32, ctypes.c_int, F, U32, P, SZ, P]
         L.gdn_backward.restype = ctypes.c_int
+        L.gdn_qsa_compress.argtypes = [P, P, P, P, P, I32, I64, F, P]
+        L.gdn_qsa_compress.restype = ctypes.c_int
+        L.gdn_qsa_index_workspace_size.argtypes = [I32, I64]
+        L.gdn_qsa_index_workspace_size.restype = SZ
+        L.gdn_qsa_index_decode.argtypes = [P, P, P, P, I32, I64, I32, F, P, P, P, P, SZ, P]
+        L.gdn_qsa_index_decode.restype = ctypes.c_int
         L.gdn_get_device_error.argtypes = [P, P]
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -258,3 +269,53 @@ def gdn_backward(q, k, v, g, beta, d_out, S0=None, dS_final=None, cu_seqlens=Non
 def gdn_get_device_error(workspace: torch.Tensor, stream=None) -> int:
     """Synchronise the stream; return (and clear) the device error status in the workspace."""
     return int(lib().gdn_get_device_error(_dev(workspace, "workspace"), _stream(stream)))
+
+
+# ------------------------------------------------------------------ QSA indexer
+def gdn_qsa_compress(k, cu_seqlens, cu_blocks, *, k_hat, pos0=None, rope_base: float = 10000.0,
+                     stream=None):
+    """Block cache from indexer keys: k [T_total, 128] bf16 -> k_hat [total_blocks, 128] bf16
+    (written in place and returned); cu_seqlens, cu_blocks int32 [N + 1], pos0 int32 [N]."""
+    N = cu_seqlens.numel() - 1
+    st = lib().gdn_qsa_compress(
+        _dev(k, "k"), _dev(cu_seqlens, "cu_seqlens"), _dev(cu_blocks, "cu_blocks"),
+        _dev(pos0, "pos0"), _dev(k_hat, "k_hat"), N, k_hat.shape[0], float(rope_base),
+        _stream(stream))
+    _check(st, "gdn_qsa_compress")
+    return k_hat
+
+
+def gdn_qsa_index_workspace_size(num_seqs: int, total_blocks: int) -> int:
+    return int(lib().gdn_qsa_index_workspace_size(num_seqs, total_blocks))
+
+
+def qsa_index_workspace(num_seqs: int, total_blocks: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size gdn_qsa_index_decode needs."""
+    n = gdn_qsa_index_workspace_size(num_seqs, total_blocks)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def gdn_qsa_index_decode(q, q_pos, k_hat, cu_blocks, budget_blocks: int = 512, *,
+                         rope_base: float = 10000.0, workspace=None, block_idx=None,
+                         block_score=None, token_idx=None, want_scores: bool = True,
+                         want_tokens: bool = True, stream=None):
+    """Indexer for one new token per sequence: q [N, 4, 128] bf16, q_pos int32 [N],
+    k_hat [total_blocks, 128] bf16, cu_blocks int32 [N + 1].  Returns (block_idx [N, budget],
+    block_score [N, budget] or None, token_idx [N, 4 budget] or None)."""
+    N = q.shape[0]
+    dev = q.device
+    if workspace is None:
+        workspace = qsa_index_workspace(N, k_hat.shape[0], dev)
+    if block_idx is None:
+        block_idx = torch.empty(N, budget_blocks, dtype=torch.int32, device=dev)
+    if block_score is None and want_scores:
+        block_score = torch.empty(N, budget_blocks, dtype=torch.float32, device=dev)
+    if token_idx is None and want_tokens:
+        token_idx = torch.empty(N, GDN_QSA_R * budget_blocks, dtype=torch.int32, device=dev)
+    st = lib().gdn_qsa_index_decode(
+        _dev(q, "q"), _dev(q_pos, "q_pos"), _dev(k_hat, "k_hat"), _dev(cu_blocks, "cu_blocks"),
+        N, k_hat.shape[0], int(budget_blocks), float(rope_base), _dev(block_idx, "block_idx"),
+        _dev(block_score, "block_score"), _dev(token_idx, "token_idx"),
+        _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "gdn_qsa_index_decode")
+    return block_idx, block_score, token_idx

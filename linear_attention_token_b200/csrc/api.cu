@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "../../include/qsa.h"
 
 #define GDN_API extern "C" __attribute__((visibility("default")))
 
@@ -34,6 +35,15 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const f
                             float *dbeta, float *dS0, const int32_t *cu, int N, long long T_dense,
                             long long T_total, int H_qk, int H_v, int dkk, int dvv,
                             gdn_dtype dtype, float scale, int opts, void *ws, cudaStream_t stream);
+size_t qsa_index_workspace_bytes(int N, long long total_blocks);
+cudaError_t launch_qsa_compress(const void *k, const int32_t *cu_seqlens, const int32_t *cu_blocks,
+                                const int32_t *pos0, void *k_hat, int N, long long total_blocks,
+                                float rope_base, cudaStream_t stream);
+cudaError_t launch_qsa_index_decode(const void *q, const int32_t *q_pos, const void *k_hat,
+                                    const int32_t *cu_blocks, int N, long long total_blocks,
+                                    int budget, float rope_base, int32_t *block_idx,
+                                    float *block_score, int32_t *token_idx, void *workspace,
+                                    cudaStream_t stream);
 size_t static_scratch_capacity();
 cudaError_t static_scratch_ptr(void **out);
 }  // namespace gdn
@@ -304,6 +314,63 @@ GDN_API gdn_status gdn_get_device_error(void *workspace, cudaStream_t stream)
             return GDN_ERR_CUDA;
     }
     return static_cast<gdn_status>(h.status);
+}
+
+// ------------------------------------------------------------ QSA indexer (qsa.h)
+namespace {
+bool rope_base_ok(float base) { return base > 0.f && base < INFINITY; }
+}  // namespace
+
+GDN_API gdn_status gdn_qsa_compress(const void *k, const int32_t *cu_seqlens,
+                                    const int32_t *cu_blocks, const int32_t *pos0, void *k_hat,
+                                    int32_t num_seqs, int64_t total_blocks, float rope_base,
+                                    cudaStream_t stream)
+{
+    if (num_seqs < 0 || total_blocks < 0 || total_blocks > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (!rope_base_ok(rope_base)) return GDN_ERR_INVALID_ARG;
+    if (total_blocks == 0) return GDN_OK;
+    if (num_seqs == 0) return GDN_ERR_INVALID_ARG;
+    if (!k || !cu_seqlens || !cu_blocks || !k_hat) return GDN_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(k_hat, 16) || !aligned(cu_seqlens, 4) ||
+        !aligned(cu_blocks, 4) || !aligned(pos0, 4))
+        return GDN_ERR_INVALID_ARG;
+    const cudaError_t e = gdn::launch_qsa_compress(k, cu_seqlens, cu_blocks, pos0, k_hat, num_seqs,
+                                                   total_blocks, rope_base, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+GDN_API size_t gdn_qsa_index_workspace_size(int32_t num_seqs, int64_t total_blocks)
+{
+    if (num_seqs < 0 || total_blocks < 0) return 0;
+    return gdn::qsa_index_workspace_bytes(num_seqs, total_blocks);
+}
+
+GDN_API gdn_status gdn_qsa_index_decode(const void *q, const int32_t *q_pos, const void *k_hat,
+                                        const int32_t *cu_blocks, int32_t num_seqs,
+                                        int64_t total_blocks, int32_t budget_blocks,
+                                        float rope_base, int32_t *block_idx, float *block_score,
+                                        int32_t *token_idx, void *workspace,
+                                        size_t workspace_bytes, cudaStream_t stream)
+{
+    if (num_seqs < 0 || num_seqs > GDN_QSA_MAX_SEQS) return num_seqs < 0 ? GDN_ERR_INVALID_ARG
+                                                                          : GDN_ERR_UNSUPPORTED;
+    if (total_blocks < 0 || total_blocks > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (budget_blocks < 1 || budget_blocks > GDN_QSA_MAX_BUDGET) return GDN_ERR_INVALID_ARG;
+    if (!rope_base_ok(rope_base)) return GDN_ERR_INVALID_ARG;
+    if (num_seqs == 0) return GDN_OK;
+    if (!q || !q_pos || !cu_blocks || !block_idx || !workspace) return GDN_ERR_INVALID_ARG;
+    if (total_blocks > 0 && !k_hat) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_hat, 16) || !aligned(workspace, 16) || !aligned(q_pos, 4) ||
+        !aligned(cu_blocks, 4) || !aligned(block_idx, 4) || !aligned(block_score, 4) ||
+        !aligned(token_idx, 4))
+        return GDN_ERR_INVALID_ARG;
+    if (workspace_bytes < gdn::qsa_index_workspace_bytes(num_seqs, total_blocks))
+        return GDN_ERR_INVALID_ARG;
+    const cudaError_t e = gdn::launch_qsa_index_decode(q, q_pos, k_hat, cu_blocks, num_seqs,
+                                                       total_blocks, budget_blocks, rope_base,
+                                                       block_idx, block_score, token_idx,
+                                                       workspace, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 GDN_API const char *gdn_status_string(gdn_status status)

@@ -1,0 +1,583 @@
+// QSA compressed indexer on sm_100a: the block cache (mean-pooled, rotary-encoded keys)
+// and the decode-time indexer (multi-query block scores, budgeted selection, expansion
+// to tokens).  Operation and contract: include/qsa.h ("論文解説: Qwen3.8-Next の設計",
+// section "部品②: QSA").
+//
+//   qsa_compress_kernel   stream of 4 token keys in, one encoded block key out (HBM-bound).
+//   qsa_score_kernel      stream over the block cache: one fp32 score per eligible block
+//                         and a 4096-bin histogram of the scores' top 12 order bits per
+//                         sequence (HBM-bound; the dominant kernel of the indexer).
+//   qsa_threshold_kernel  per sequence: the histogram bin that holds the budget-th score.
+//   qsa_collect_kernel    pass over the scores (L2-resident): blocks above that bin are
+//                         kept, blocks inside it become candidates.
+//   qsa_finish_kernel     per sequence: exact selection among the candidates (two radix
+//                         passes over the low score bits, then the block index for ties),
+//                         sort by block, write blocks / scores / tokens, re-zero the
+//                         sequence's workspace record.
+//
+// Scores are reduced to one query vector per sequence: the four heads share the key and
+// the logits are summed, so sum_h q_h . k = (sum_h q_h) . k.  Ranking compares 32-bit
+// order keys of the fp32 scores (a monotone map of the float's bits), and ties fall to
+// the smaller block index, which makes the kept set unique.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "../../include/qsa.h"
+
+namespace gdn {
+namespace {
+
+constexpr int QR = GDN_QSA_R, QD = GDN_QSA_DIM, QROPE = GDN_QSA_ROPE_DIMS;
+constexpr int QHALF = QROPE / 2, QHEADS = GDN_QSA_HEADS;
+constexpr int HBITS = 12, HBINS = 1 << HBITS;        // first radix digit (score kernel)
+constexpr int SURE_CAP = GDN_QSA_MAX_BUDGET;          // blocks kept above the threshold bin
+constexpr int CAND_CAP = 8192;                        // candidates listed from that bin
+constexpr int SCORE_TILE = 512;                       // cache rows per scoring work item
+constexpr int COLLECT_TILE = 4096;                    // score entries per collect work item
+constexpr int kScoreThreads = 256, kFinishThreads = 1024;
+
+// One sequence's record in the indexer workspace (zero between calls except thr/rank).
+struct SeqWork {
+    uint32_t hist[HBINS];     // scores per top-12-bit bin, filled by the score kernel
+    uint32_t n_sure, n_cand;  // list lengths (n_cand counts past CAND_CAP too)
+    int32_t thr_bin, rank;    // threshold bin (-1: keep every eligible block), rank inside it
+    uint2 sure[SURE_CAP];     // (order key, block) kept outright
+    uint2 cand[CAND_CAP];     // (order key, block) inside the threshold bin
+};
+static_assert(sizeof(SeqWork) % 16 == 0, "workspace records stay 16-byte aligned");
+
+constexpr double kTwoPiHi = 6.283185307179586;        // 2 pi rounded to double
+constexpr double kTwoPiLo = 2.4492935982947064e-16;   // 2 pi - kTwoPiHi
+constexpr double kInvTwoPi = 0.15915494309189535;
+
+// Rotation angle p * w, reduced into [-pi, pi] in double precision by subtracting the
+// nearest multiple of a two-part 2 pi (Cody and Waite's additive reduction).  Positions
+// reach 2^31, where a float angle would be off by whole hundredths of a radian.
+__device__ __forceinline__ float reduced_angle(double p, double w) {
+    const double x = p * w;
+    const double n = rint(x * kInvTwoPi);
+    return (float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, x));
+}
+
+__device__ __forceinline__ double rotary_freq(double base, int i) {   // base^(-i / 32)
+    return pow(base, -(double)i / (double)QHALF);
+}
+
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Monotone map float -> uint32 (larger score, larger key); -0 is taken as +0 so that equal
+// scores always get equal keys.
+__device__ __forceinline__ uint32_t order_key(float x) {
+    if (x == 0.f) x = 0.f;
+    const uint32_t u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Blocks of sequence n the query may score: whole blocks at or before its position (and
+// inside the cache's total_blocks rows, whatever the offsets say).
+__device__ __forceinline__ int eligible(const int32_t *cu_blocks, const int32_t *q_pos, int n,
+                                        int total_blocks) {
+    const long long end = cu_blocks[n + 1] < total_blocks ? cu_blocks[n + 1] : total_blocks;
+    const long long cached = end - cu_blocks[n];
+    const long long seen = ((long long)q_pos[n] + 1) / QR;
+    const long long e = cached < seen ? cached : seen;
+    return e > 0 ? (int)e : 0;
+}
+
+// Exclusive prefix sum of one int per thread over the CTA (blockDim.x multiple of 32,
+// at most 1024); `total` gets the sum.  Uses 33 ints of shared scratch.
+__device__ int block_exclusive_scan(int v, int *scratch, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < nw) scratch[lane] = w;          // inclusive warp totals
+        if (lane == 31) scratch[32] = w;
+    }
+    __syncthreads();
+    const int before = (warp > 0 ? scratch[warp - 1] : 0) + x - v;
+    total = scratch[32];
+    __syncthreads();                                // scratch may be reused at once
+    return before;
+}
+
+// item0[n] = first work item of sequence n, item0[N] = item count; a sequence gets
+// ceil(eligible / tile) items.  N <= GDN_QSA_MAX_SEQS.
+__device__ void build_items(int *item0, int *scratch, int N, const int32_t *cu_blocks,
+                            const int32_t *q_pos, int total_blocks, int tile) {
+    const int per = (N + blockDim.x - 1) / blockDim.x;
+    const int m0 = threadIdx.x * per;
+    int local = 0;
+    for (int m = m0; m < m0 + per && m < N; ++m)
+        local += (eligible(cu_blocks, q_pos, m, total_blocks) + tile - 1) / tile;
+    int total;
+    int acc = block_exclusive_scan(local, scratch, total);
+    for (int m = m0; m < m0 + per && m < N; ++m) {
+        item0[m] = acc;
+        acc += (eligible(cu_blocks, q_pos, m, total_blocks) + tile - 1) / tile;
+    }
+    if (threadIdx.x == 0) item0[N] = total;
+    __syncthreads();
+}
+
+// Largest n < N with item0[n] <= it (sequences without items are skipped).
+__device__ __forceinline__ int seq_of_item(const int *item0, int N, int it) {
+    int lo = 0, hi = N;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (item0[mid] <= it) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Among nbins counts in h (shared), the highest bin b with
+//   count(bins above b) < r <= count(bins at or above b)       (1 <= r <= total)
+// -> out[0] = b, out[1] = count(bins above b), out[2] = h[b].  nbins is a multiple of
+// blockDim.x; every thread of the CTA calls this.
+__device__ void find_from_top(const uint32_t *h, int nbins, int r, int *scratch, int *out) {
+    const int per = nbins / blockDim.x;
+    const int top = nbins - per * threadIdx.x;      // this thread owns bins [top - per, top)
+    if (threadIdx.x == 0) { out[0] = 0; out[1] = 0; out[2] = 0; }   // (r outside 1..total)
+    int local = 0;
+    for (int b = top - 1; b >= top - per; --b) local += (int)h[b];
+    int total;
+    const int above = block_exclusive_scan(local, scratch, total);
+    if (above < r && r <= above + local) {
+        int acc = above;
+        for (int b = top - 1; b >= top - per; --b) {
+            if (acc + (int)h[b] >= r) { out[0] = b; out[1] = acc; out[2] = (int)h[b]; break; }
+            acc += (int)h[b];
+        }
+    }
+    __syncthreads();
+}
+
+// ------------------------------------------------------------------ compress
+// A half-warp per cache row: lane l (0..15) owns dims 8 l .. 8 l + 7 of the row.  Lanes
+// 0-3 hold the first rotary halves (dims 0..31), lanes 4-7 their partners (32..63), lanes
+// 8-15 the pass-through dims.
+__global__ void __launch_bounds__(256) qsa_compress_kernel(
+    const __nv_bfloat16 *__restrict__ k, const int32_t *__restrict__ cu_seqlens,
+    const int32_t *__restrict__ cu_blocks, const int32_t *__restrict__ pos0,
+    __nv_bfloat16 *__restrict__ k_hat, int N, int total_blocks, double base)
+{
+    __shared__ double w_s[QHALF];
+    if (threadIdx.x < QHALF) w_s[threadIdx.x] = rotary_freq(base, threadIdx.x);
+    __syncthreads();
+    const int lane = threadIdx.x & 31, hl = lane & 15;
+    const unsigned hmask = 0xffffu << (lane & 16);
+    const int half_id = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 4);
+    const int n_halves = (int)((gridDim.x * blockDim.x) >> 4);
+    for (int row = half_id; row < total_blocks; row += n_halves) {
+        int lo = 0, hi = N;                          // largest n with cu_blocks[n] <= row
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(cu_blocks + mid) <= row) lo = mid; else hi = mid;
+        }
+        const int n = lo;
+        const int b = row - __ldg(cu_blocks + n);
+        const int t0 = __ldg(cu_seqlens + n), len = __ldg(cu_seqlens + n + 1) - t0;
+        const int nb = __ldg(cu_blocks + n + 1) - __ldg(cu_blocks + n);
+        if (b < 0 || b >= nb || b >= len / QR) continue;    // uniform over the half-warp
+        const __nv_bfloat16 *src = k + (size_t)(t0 + QR * b) * QD + 8 * hl;
+        uint4 tok[QR];
+#pragma unroll
+        for (int j = 0; j < QR; ++j) tok[j] = ld_stream(src + (size_t)j * QD);
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = 0.f;
+#pragma unroll
+        for (int j = 0; j < QR; ++j) {
+            const uint32_t wv[4] = {tok[j].x, tok[j].y, tok[j].z, tok[j].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) { x[2 * e] += bf_lo(wv[e]); x[2 * e + 1] += bf_hi(wv[e]); }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] *= 1.f / QR;
+        float y[8];                                  // the rotation partner's pooled value
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = __shfl_xor_sync(hmask, x[e], 4, 16);
+        if (hl < 8) {
+            const double p = (double)(pos0 ? __ldg(pos0 + n) : 0) + (double)QR * b;
+            const bool first = hl < 4;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float s, c;
+                __sincosf(reduced_angle(p, w_s[8 * (hl & 3) + e]), &s, &c);
+                x[e] = first ? fmaf(x[e], c, -y[e] * s) : fmaf(x[e], c, y[e] * s);
+            }
+        }
+        uint4 o;
+        o.x = pack_bf2(x[0], x[1]); o.y = pack_bf2(x[2], x[3]);
+        o.z = pack_bf2(x[4], x[5]); o.w = pack_bf2(x[6], x[7]);
+        *reinterpret_cast<uint4 *>(k_hat + (size_t)row * QD + 8 * hl) = o;
+    }
+}
+
+// --------------------------------------------------------------------- score
+// Persistent CTAs walk work items (sequence, tile of SCORE_TILE rows).  A group of 8
+// lanes owns a row (lane g owns dims 16 g .. 16 g + 15, 32 bytes), a warp 4 rows per
+// step, unrolled U steps deep so that 4 KB per warp are in flight.
+constexpr int kScoreUnroll = 4;
+
+__global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
+    const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ q_pos,
+    const __nv_bfloat16 *__restrict__ k_hat, const int32_t *__restrict__ cu_blocks, int N,
+    int total_blocks, double base, SeqWork *__restrict__ ws, float *__restrict__ scores)
+{
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);
+    float *qbar = reinterpret_cast<float *>(hist + HBINS);
+    int *scratch = reinterpret_cast<int *>(qbar + QD);
+    int *item0 = scratch + 36;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 3, gl = lane & 7;
+    for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = 0;
+    build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, SCORE_TILE);
+    const int n_items = item0[N];
+    int cur = -1;
+    float qv[16];
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+        const int n = seq_of_item(item0, N, it);
+        if (n != cur) {
+            __syncthreads();
+            if (cur >= 0) {                         // hand the finished sequence's counts on
+                for (int i = tid; i < HBINS; i += blockDim.x) {
+                    const uint32_t v = hist[i];
+                    if (v) { atomicAdd(&ws[cur].hist[i], v); hist[i] = 0; }
+                }
+            }
+            if (tid < QD) {                         // sum over heads of RoPE(q_h, q_pos)
+                const __nv_bfloat16 *qn = q + (size_t)n * QHEADS * QD;
+                const int d = tid;
+                float acc = 0.f;
+                if (d < QROPE) {
+                    float s, c;
+                    sincosf(reduced_angle((double)q_pos[n], rotary_freq(base, d & (QHALF - 1))), &s, &c);
+                    const int pd = d ^ QHALF;       // rotation partner
+                    const float sg = d < QHALF ? -s : s;
+#pragma unroll
+                    for (int h = 0; h < QHEADS; ++h)
+                        acc += fmaf(__bfloat162float(qn[h * QD + d]), c,
+                                    sg * __bfloat162float(qn[h * QD + pd]));
+                } else {
+#pragma unroll
+                    for (int h = 0; h < QHEADS; ++h) acc += __bfloat162float(qn[h * QD + d]);
+                }
+                qbar[d] = acc;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) qv[e] = qbar[16 * gl + e];
+            cur = n;
+        }
+        const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
+        const int r0 = (it - item0[n]) * SCORE_TILE;
+        const int r1 = min(elig, r0 + SCORE_TILE);
+        const __nv_bfloat16 *kb = k_hat + (size_t)cu_blocks[n] * QD + 16 * gl;
+        float *sc = scores + cu_blocks[n];
+        for (int base_row = r0 + 4 * warp; base_row < r1; base_row += 32 * kScoreUnroll) {
+            uint4 a[kScoreUnroll][2];
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) {
+                const int row = base_row + g + 32 * u;
+                if (row < r1) {
+                    a[u][0] = ld_stream(kb + (size_t)row * QD);
+                    a[u][1] = ld_stream(kb + (size_t)row * QD + 8);
+                } else {
+                    a[u][0] = make_uint4(0, 0, 0, 0);
+                    a[u][1] = make_uint4(0, 0, 0, 0);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kScoreUnroll; ++u) {
+                const uint32_t wv[8] = {a[u][0].x, a[u][0].y, a[u][0].z, a[u][0].w,
+                                        a[u][1].x, a[u][1].y, a[u][1].z, a[u][1].w};
+                float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    s0 = fmaf(qv[2 * e], bf_lo(wv[e]), s0);
+                    s1 = fmaf(qv[2 * e + 1], bf_hi(wv[e]), s1);
+                }
+                float s = s0 + s1;
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                const int row = base_row + g + 32 * u;
+                if (gl == 0 && row < r1) {
+                    sc[row] = s;
+                    atomicAdd(&hist[order_key(s) >> (32 - HBITS)], 1u);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (cur >= 0) {
+        for (int i = tid; i < HBINS; i += blockDim.x) {
+            const uint32_t v = hist[i];
+            if (v) atomicAdd(&ws[cur].hist[i], v);
+        }
+    }
+}
+
+// ----------------------------------------------------------------- threshold
+__global__ void __launch_bounds__(kFinishThreads) qsa_threshold_kernel(
+    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int total_blocks,
+    int budget, SeqWork *__restrict__ ws)
+{
+    __shared__ uint32_t h[HBINS];
+    __shared__ int scratch[36], res[3];
+    const int n = blockIdx.x;
+    SeqWork &w = ws[n];
+    const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
+    if (elig <= budget) {
+        if (threadIdx.x == 0) { w.thr_bin = -1; w.rank = elig; }
+        return;
+    }
+    for (int i = threadIdx.x; i < HBINS; i += blockDim.x) h[i] = w.hist[i];
+    __syncthreads();
+    find_from_top(h, HBINS, budget, scratch, res);
+    if (threadIdx.x == 0) { w.thr_bin = res[0]; w.rank = budget - res[1]; }
+}
+
+// ------------------------------------------------------------------- collect
+__global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
+    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int N,
+    int total_blocks, const float *__restrict__ scores, SeqWork *__restrict__ ws)
+{
+    extern __shared__ __align__(16) unsigned char smem[];
+    int *scratch = reinterpret_cast<int *>(smem);
+    int *item0 = scratch + 36;
+    build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, COLLECT_TILE);
+    const int n_items = item0[N];
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+        const int n = seq_of_item(item0, N, it);
+        SeqWork &w = ws[n];
+        const int thr = w.thr_bin;
+        const int r0 = (it - item0[n]) * COLLECT_TILE;
+        const int r1 = min(eligible(cu_blocks, q_pos, n, total_blocks), r0 + COLLECT_TILE);
+        const float *sc = scores + cu_blocks[n];
+        for (int row = r0 + threadIdx.x; row < r1; row += blockDim.x) {
+            const uint32_t key = order_key(sc[row]);
+            const int bin = (int)(key >> (32 - HBITS));
+            if (thr < 0 || bin > thr) {
+                const uint32_t slot = atomicAdd(&w.n_sure, 1u);
+                if (slot < SURE_CAP) w.sure[slot] = make_uint2(key, (uint32_t)row);
+            } else if (bin == thr) {
+                const uint32_t slot = atomicAdd(&w.n_cand, 1u);
+                if (slot < CAND_CAP) w.cand[slot] = make_uint2(key, (uint32_t)row);
+            }
+        }
+    }
+}
+
+// -------------------------------------------------------------------- finish
+__global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
+    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int total_blocks,
+    int budget, const float *__restrict__ scores, SeqWork *__restrict__ ws,
+    int32_t *__restrict__ block_idx,
+    float *__restrict__ block_score, int32_t *__restrict__ token_idx)
+{
+    __shared__ uint2 sel[SURE_CAP];
+    __shared__ uint32_t h[2048];
+    __shared__ int scratch[36], res[3], s_count;
+    const int n = blockIdx.x, tid = threadIdx.x;
+    SeqWork &w = ws[n];
+    const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
+    const int thr = w.thr_bin;
+    const int n_sure = min((int)w.n_sure, SURE_CAP);
+    const uint32_t n_cand = w.n_cand;
+    if (tid == 0) s_count = 0;
+    for (int i = tid; i < n_sure; i += blockDim.x) sel[i] = w.sure[i];
+    __syncthreads();
+
+    if (thr >= 0 && elig > 0) {
+        const bool listed = n_cand <= (uint32_t)CAND_CAP;
+        const float *sc = scores + cu_blocks[n];
+        // every candidate (order key, block) of the threshold bin, from the list or, when
+        // the bin overflowed it, from the scores themselves
+        auto for_cand = [&](auto &&f) {
+            if (listed) {
+                for (uint32_t i = tid; i < n_cand; i += blockDim.x) {
+                    const uint2 c = w.cand[i];
+                    f(c.x, c.y);
+                }
+            } else {
+                for (int i = tid; i < elig; i += blockDim.x) {
+                    const uint32_t key = order_key(sc[i]);
+                    if ((int)(key >> (32 - HBITS)) == thr) f(key, (uint32_t)i);
+                }
+            }
+        };
+        int r = w.rank;                             // 1-based rank inside the bin
+        uint32_t kmask = 0xffffffffu << (32 - HBITS), kval = (uint32_t)thr << (32 - HBITS);
+        int eq = 0;
+        for (int shift = 32 - HBITS - 10; shift >= 0; shift -= 10) {   // bits 19..10, 9..0
+            for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0;
+            __syncthreads();
+            for_cand([&](uint32_t key, uint32_t) {
+                if ((key & kmask) == kval) atomicAdd(&h[(key >> shift) & 1023u], 1u);
+            });
+            __syncthreads();
+            find_from_top(h, 1024, r, scratch, res);
+            kval |= (uint32_t)res[0] << shift;
+            kmask |= 1023u << shift;
+            r -= res[1];
+            eq = res[2];
+            __syncthreads();
+        }
+        const uint32_t tau = kval;                  // order key of the budget-th best block
+        uint32_t iota = 0xffffffffu;                // blocks of key tau kept up to this index
+        if (eq > r) {
+            // the r smallest block indices among key == tau: radix over the index bits,
+            // smallest first (bin nb - 1 - digit, so that "from the top" means smallest)
+            uint32_t imask = 0, ival = 0;
+            const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
+            for (int p = 0; p < 3; ++p) {
+                const int nb = 1 << widths[p], sh = shifts[p];
+                for (int i = tid; i < nb; i += blockDim.x) h[i] = 0;
+                __syncthreads();
+                for_cand([&](uint32_t key, uint32_t idx) {
+                    if (key == tau && (idx & imask) == ival)
+                        atomicAdd(&h[nb - 1 - ((idx >> sh) & (uint32_t)(nb - 1))], 1u);
+                });
+                __syncthreads();
+                find_from_top(h, nb, r, scratch, res);
+                ival |= (uint32_t)(nb - 1 - res[0]) << sh;
+                imask |= (uint32_t)(nb - 1) << sh;
+                r -= res[1];
+                __syncthreads();
+            }
+            iota = ival;
+        }
+        for_cand([&](uint32_t key, uint32_t idx) {
+            if (key > tau || (key == tau && idx <= iota)) {
+                const int slot = n_sure + atomicAdd(&s_count, 1);
+                if (slot < SURE_CAP) sel[slot] = make_uint2(key, idx);
+            }
+        });
+    }
+    __syncthreads();
+    const int count = min(thr >= 0 ? n_sure + s_count : n_sure, min(budget, SURE_CAP));
+
+    // sort the kept blocks by index (bitonic over the next power of two)
+    int P = 1;
+    while (P < count) P <<= 1;
+    for (int i = count + tid; i < P; i += blockDim.x) sel[i] = make_uint2(0u, 0xffffffffu);
+    __syncthreads();
+    for (int kk = 2; kk <= P; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += blockDim.x) {
+                const int ij = i ^ j;
+                if (ij > i) {
+                    const uint2 a = sel[i], b = sel[ij];
+                    const bool up = (i & kk) == 0;
+                    if ((a.y > b.y) == up) { sel[i] = b; sel[ij] = a; }
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    int32_t *bi = block_idx + (size_t)n * budget;
+    for (int i = tid; i < budget; i += blockDim.x) bi[i] = i < count ? (int32_t)sel[i].y : -1;
+    if (block_score) {
+        float *bs = block_score + (size_t)n * budget;
+        for (int i = tid; i < budget; i += blockDim.x) bs[i] = i < count ? key_value(sel[i].x) : -INFINITY;
+    }
+    if (token_idx) {
+        int32_t *ti = token_idx + (size_t)n * budget * QR;
+        for (int t = tid; t < budget * QR; t += blockDim.x) {
+            const int i = t / QR;
+            ti[t] = i < count ? (int32_t)(QR * sel[i].y + (uint32_t)(t % QR)) : -1;
+        }
+    }
+    // leave the record zeroed for the next call
+    for (int i = tid; i < HBINS; i += blockDim.x) w.hist[i] = 0;
+    if (tid == 0) { w.n_sure = 0; w.n_cand = 0; }
+}
+
+int sm_count() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+}  // namespace
+
+size_t qsa_index_workspace_bytes(int N, long long total_blocks) {
+    const size_t rec = (size_t)N * sizeof(SeqWork);
+    return rec + (((size_t)total_blocks * sizeof(float) + 255) / 256) * 256;
+}
+
+cudaError_t launch_qsa_compress(const void *k, const int32_t *cu_seqlens, const int32_t *cu_blocks,
+                                const int32_t *pos0, void *k_hat, int N, long long total_blocks,
+                                float rope_base, cudaStream_t stream) {
+    const int rows_per_cta = 256 / 16;
+    long long want = (total_blocks + rows_per_cta - 1) / rows_per_cta;
+    const long long cap = (long long)sm_count() * 8;
+    const int grid = (int)(want < cap ? want : cap);
+    qsa_compress_kernel<<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(k), cu_seqlens, cu_blocks, pos0,
+        static_cast<__nv_bfloat16 *>(k_hat), N, (int)total_blocks, (double)rope_base);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qsa_index_decode(const void *q, const int32_t *q_pos, const void *k_hat,
+                                    const int32_t *cu_blocks, int N, long long total_blocks,
+                                    int budget, float rope_base, int32_t *block_idx,
+                                    float *block_score, int32_t *token_idx, void *workspace,
+                                    cudaStream_t stream) {
+    SeqWork *ws = static_cast<SeqWork *>(workspace);
+    float *scores = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) +
+                                              (size_t)N * sizeof(SeqWork));
+    const int persistent = sm_count() * 4;
+    const size_t items_smem = (size_t)(36 + N + 1) * sizeof(int);
+    const size_t score_smem = HBINS * sizeof(uint32_t) + QD * sizeof(float) + items_smem;
+    qsa_score_kernel<<<persistent, kScoreThreads, score_smem, stream>>>(
+        static_cast<const __nv_bfloat16 *>(q), q_pos, static_cast<const __nv_bfloat16 *>(k_hat),
+        cu_blocks, N, (int)total_blocks, (double)rope_base, ws, scores);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    qsa_threshold_kernel<<<N, kFinishThreads, 0, stream>>>(q_pos, cu_blocks, (int)total_blocks,
+                                                           budget, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    qsa_collect_kernel<<<persistent, kScoreThreads, items_smem, stream>>>(
+        q_pos, cu_blocks, N, (int)total_blocks, scores, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    qsa_finish_kernel<<<N, kFinishThreads, 0, stream>>>(q_pos, cu_blocks, (int)total_blocks,
+                                                        budget, scores, ws, block_idx,
+                                                        block_score, token_idx);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -157,3 +157,79 @@ def decode_step_inputs(w: Workload, step: int, device="cpu", seed: Optional[int]
     assert w.kind == "decode"
     s = (BASE_SEED + w.index if seed is None else seed) + 1000 * step
     return draw(w.decode_seqs, w.H_qk, w.H_v, w.dk, w.dv, w.dtype, s, device, w.g_mult)
+
+
+# ------------------------------------------------------------------ QSA indexer
+# Recipe: indexer keys and query heads ~ N(0, 1), cast to bf16.  A block-cache row stands
+# for the mean of 4 such keys after a rotation, i.e. an isotropic normal with standard
+# deviation 1/2; caches drawn directly take that distribution.  Palette caches (tests of
+# exact ties) repeat a few rows c * v (c = 1, 2, ...) for one drawn vector v.
+QSA_DIM, QSA_HEADS, QSA_R = 128, 4, 4
+QSA_SEED = BASE_SEED + 40
+
+
+@dataclasses.dataclass(frozen=True)
+class QsaWorkload:
+    name: str
+    ctx_lens: tuple           # tokens per sequence so far; the query is the last of them
+    budget_blocks: int = 512  # 2048 tokens at 4 tokens per block
+    index: int = 0
+
+    @property
+    def num_seqs(self) -> int:
+        return len(self.ctx_lens)
+
+    @property
+    def blocks(self) -> tuple:
+        return tuple(int(L) // QSA_R for L in self.ctx_lens)
+
+
+def qsa_workloads() -> list:
+    return [
+        QsaWorkload("qsa_decode_n8_ctx1m_budget2048", (1 << 20,) * 8, 512, index=0),
+        QsaWorkload("qsa_decode_n5_ragged_budget2048", (70001, 8191, 4096, 3, 2052), 512,
+                    index=1),
+    ]
+
+
+def qsa_keys(T: int, seed: int, device="cpu") -> torch.Tensor:
+    gen = torch.Generator(device=torch.device(device)).manual_seed(seed)
+    return torch.randn(T, QSA_DIM, generator=gen, device=device).to(torch.bfloat16).contiguous()
+
+
+def qsa_queries(N: int, seed: int, device="cpu") -> torch.Tensor:
+    gen = torch.Generator(device=torch.device(device)).manual_seed(seed)
+    return (torch.randn(N, QSA_HEADS, QSA_DIM, generator=gen, device=device)
+            .to(torch.bfloat16).contiguous())
+
+
+def qsa_cache(total_blocks: int, seed: int, device="cpu") -> torch.Tensor:
+    gen = torch.Generator(device=torch.device(device)).manual_seed(seed)
+    return ((torch.randn(total_blocks, QSA_DIM, generator=gen, device=device) * 0.5)
+            .to(torch.bfloat16).contiguous())
+
+
+def qsa_palette_cache(total_blocks: int, n_distinct: int, seed: int, device="cpu") -> torch.Tensor:
+    """Rows c * v with c drawn from 1..n_distinct per row (exact ties inside each c)."""
+    gen = torch.Generator(device=torch.device(device)).manual_seed(seed)
+    v = torch.randn(QSA_DIM, generator=gen, device=device) * 0.5
+    c = torch.randint(1, n_distinct + 1, (total_blocks, 1), generator=gen, device=device)
+    return (c.to(torch.float32) * v).to(torch.bfloat16).contiguous()
+
+
+def qsa_offsets(counts, device="cpu") -> torch.Tensor:
+    return cu_seqlens_of(counts).to(device)
+
+
+def qsa_decode_inputs(w: QsaWorkload, device="cpu", seed: Optional[int] = None) -> dict:
+    """q [N, 4, 128], q_pos [N] (the last token of each sequence), the block cache and its
+    row offsets."""
+    s = QSA_SEED + w.index if seed is None else seed
+    blocks = w.blocks
+    return {
+        "q": qsa_queries(w.num_seqs, s, device),
+        "q_pos": torch.tensor([max(0, L - 1) for L in w.ctx_lens], dtype=torch.int32,
+                              device=device),
+        "k_hat": qsa_cache(int(sum(blocks)), s + 1, device),
+        "cu_blocks": qsa_offsets(blocks, device),
+    }

@@ -1,8 +1,9 @@
 """Host-side checks of the C ABI that need no GPU: the library loads, exports
-every symbol include/gdn.h declares, and rejects bad arguments before launching."""
+every symbol include/*.h declares, and rejects bad arguments before launching."""
 from __future__ import annotations
 
 import ctypes
+import glob
 import os
 import re
 
@@ -12,7 +13,7 @@ import linear_attention_token_b200 as gdn
 from linear_attention_token_b200 import build as gdn_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "gdn.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 @pytest.fixture(scope="module")
@@ -22,7 +23,7 @@ def L():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(gdn_[a-z_]+)\s*\(", text)))
 
@@ -192,3 +193,84 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(ValueError):
         gdn.gdn_decode_step(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2),
                             torch.zeros(4, 2, 128, 128))
+
+
+# ------------------------------------------------------------------ QSA indexer
+def _qsa_compress(L, **over):
+    a = dict(k=A, cu=A + 0x1000, cub=A + 0x2000, pos0=None, k_hat=A + 0x3000, N=2, nb=64,
+             base=10000.0)
+    a.update(over)
+    return L.gdn_qsa_compress(P(a["k"]), P(a["cu"]), P(a["cub"]), P(a["pos0"]), P(a["k_hat"]),
+                              a["N"], a["nb"], a["base"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(k=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(cub=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(k_hat=A + 0x3008), gdn.GDN_ERR_INVALID_ARG),      # bf16 rows need 16-byte alignment
+    (dict(pos0=A + 0x4002), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=0), gdn.GDN_ERR_INVALID_ARG),                   # blocks but no sequence
+    (dict(nb=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(nb=1 << 31), gdn.GDN_ERR_INVALID_ARG),
+    (dict(base=0.0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(base=float("inf")), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_qsa_compress_rejects_on_host(L, over, expect):
+    assert _qsa_compress(L, **over) == expect
+
+
+def test_qsa_compress_without_blocks_is_a_no_op(L):
+    assert _qsa_compress(L, nb=0, k=None, k_hat=None) == gdn.GDN_OK
+
+
+def _qsa_index(L, **over):
+    a = dict(q=A, qpos=A + 0x1000, k_hat=A + 0x2000, cub=A + 0x3000, N=2, nb=64, budget=512,
+             base=10000.0, bi=A + 0x4000, bs=None, ti=None, ws=A + 0x5000, ws_bytes=1 << 40)
+    a.update(over)
+    return L.gdn_qsa_index_decode(P(a["q"]), P(a["qpos"]), P(a["k_hat"]), P(a["cub"]), a["N"],
+                                  a["nb"], a["budget"], a["base"], P(a["bi"]), P(a["bs"]),
+                                  P(a["ti"]), P(a["ws"]), a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(qpos=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(bi=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ws=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(k_hat=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(q=A + 8), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ti=A + 0x6002), gdn.GDN_ERR_INVALID_ARG),
+    (dict(budget=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(budget=4097), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=4097), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(ws_bytes=1024), gdn.GDN_ERR_INVALID_ARG),
+    (dict(base=-1.0), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_qsa_index_rejects_on_host(L, over, expect):
+    assert _qsa_index(L, **over) == expect
+
+
+def test_qsa_index_with_no_sequences_is_a_no_op(L):
+    assert _qsa_index(L, N=0, q=None, qpos=None, bi=None, ws=None) == gdn.GDN_OK
+
+
+def test_qsa_workspace_size(L):
+    # per sequence: 4096-bin histogram, two counters, threshold and rank, 4096 kept and
+    # 8192 candidate (key, block) pairs; then one fp32 score per cached block (256-byte
+    # rounded)
+    rec = 4096 * 4 + 4 * 4 + 4096 * 8 + 8192 * 8
+    assert L.gdn_qsa_index_workspace_size(3, 1000) == 3 * rec + 4096
+    assert L.gdn_qsa_index_workspace_size(-1, 10) == 0
+
+
+def test_qsa_constants_match_the_header():
+    text = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    vals = dict(re.findall(r"#define (GDN_QSA_[A-Z_]+) (\d+)", text))
+    b = gdn._binding
+    assert int(vals["GDN_QSA_R"]) == b.GDN_QSA_R == 4
+    assert int(vals["GDN_QSA_DIM"]) == b.GDN_QSA_DIM == 128
+    assert int(vals["GDN_QSA_ROPE_DIMS"]) == b.GDN_QSA_ROPE_DIMS == 64
+    assert int(vals["GDN_QSA_HEADS"]) == b.GDN_QSA_HEADS == 4
+    assert int(vals["GDN_QSA_MAX_BUDGET"]) == b.GDN_QSA_MAX_BUDGET
+    assert int(vals["GDN_QSA_MAX_SEQS"]) == b.GDN_QSA_MAX_SEQS
