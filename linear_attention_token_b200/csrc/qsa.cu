@@ -7,9 +7,9 @@
 //   qsa_score_kernel      stream over the block cache: one fp32 score per eligible block
 //                         and a 4096-bin histogram of the scores' top 12 order bits per
 //                         sequence (HBM-bound; the dominant kernel of the indexer).
-//   qsa_threshold_kernel  per sequence: the histogram bin that holds the budget-th score.
-//   qsa_collect_kernel    pass over the scores (L2-resident): blocks above that bin are
-//                         kept, blocks inside it become candidates.
+//   qsa_collect_kernel    pass over the scores (L2-resident): from the histogram, the bin
+//                         that holds the budget-th score; blocks above it are kept, blocks
+//                         inside it become candidates.
 //   qsa_finish_kernel     per sequence: exact selection among the candidates (two radix
 //                         passes over the low score bits, then the block index for ties),
 //                         sort by block, write blocks / scores / tokens, re-zero the
@@ -42,6 +42,8 @@ struct SeqWork {
     uint32_t hist[HBINS];     // scores per top-12-bit bin, filled by the score kernel
     uint32_t n_sure, n_cand;  // list lengths (n_cand counts past CAND_CAP too)
     int32_t thr_bin, rank;    // threshold bin (-1: keep every eligible block), rank inside it
+    uint32_t items_done;      // score work items finished (the last one sets thr_bin, rank)
+    uint32_t pad[3];
     uint2 sure[SURE_CAP];     // (order key, block) kept outright
     uint2 cand[CAND_CAP];     // (order key, block) inside the threshold bin
 };
@@ -69,6 +71,16 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
+}
+
+// Programmatic dependent launch: the next kernel of the call may start its prologue while
+// this one drains; it waits for this grid's completion (and its memory) before it reads
+// anything this grid wrote.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_primary() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
@@ -243,16 +255,31 @@ __global__ void __launch_bounds__(256) qsa_compress_kernel(
     }
 }
 
+// The threshold of sequence n from its finished histogram (h: HBINS counts in shared
+// memory, loaded by the caller): the bin holding the budget-th best score and that
+// score's rank inside the bin; bin -1 when every eligible block is kept.
+__device__ void threshold_of(const uint32_t *h, int elig, int budget, int *scratch, int *res,
+                             int &bin, int &rank) {
+    if (elig <= budget) { bin = -1; rank = elig; return; }
+    find_from_top(h, HBINS, budget, scratch, res);
+    bin = res[0];
+    rank = budget - res[1];
+    __syncthreads();
+}
+
 // --------------------------------------------------------------------- score
-// Persistent CTAs walk work items (sequence, tile of SCORE_TILE rows).  A group of 8
-// lanes owns a row (lane g owns dims 16 g .. 16 g + 15, 32 bytes), a warp 4 rows per
-// step, unrolled U steps deep so that 4 KB per warp are in flight.
+// Persistent CTAs; CTA c takes the contiguous run of work items [c per, (c + 1) per), so
+// it stays on one sequence for long stretches (one summed query and one histogram hand-off
+// per sequence it touches).  A group of 8 lanes owns a row (lane g owns dims
+// 16 g .. 16 g + 15, 32 bytes), a warp 4 rows per step, unrolled U steps deep so that
+// 4 KB per warp are in flight.
 constexpr int kScoreUnroll = 4;
 
 __global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ q_pos,
     const __nv_bfloat16 *__restrict__ k_hat, const int32_t *__restrict__ cu_blocks, int N,
-    int total_blocks, double base, SeqWork *__restrict__ ws, float *__restrict__ scores)
+    int total_blocks, int budget, double base, SeqWork *__restrict__ ws,
+    float *__restrict__ scores)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem);
@@ -263,47 +290,41 @@ __global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
     for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = 0;
     build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, SCORE_TILE);
     const int n_items = item0[N];
-    int cur = -1;
-    float qv[16];
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const int per = (n_items + gridDim.x - 1) / gridDim.x;
+    int it = blockIdx.x * per;
+    const int it_end = min(n_items, it + per);
+    while (it < it_end) {
         const int n = seq_of_item(item0, N, it);
-        if (n != cur) {
-            __syncthreads();
-            if (cur >= 0) {                         // hand the finished sequence's counts on
-                for (int i = tid; i < HBINS; i += blockDim.x) {
-                    const uint32_t v = hist[i];
-                    if (v) { atomicAdd(&ws[cur].hist[i], v); hist[i] = 0; }
-                }
-            }
-            if (tid < QD) {                         // sum over heads of RoPE(q_h, q_pos)
-                const __nv_bfloat16 *qn = q + (size_t)n * QHEADS * QD;
-                const int d = tid;
-                float acc = 0.f;
-                if (d < QROPE) {
-                    float s, c;
-                    sincosf(reduced_angle((double)q_pos[n], rotary_freq(base, d & (QHALF - 1))), &s, &c);
-                    const int pd = d ^ QHALF;       // rotation partner
-                    const float sg = d < QHALF ? -s : s;
-#pragma unroll
-                    for (int h = 0; h < QHEADS; ++h)
-                        acc += fmaf(__bfloat162float(qn[h * QD + d]), c,
-                                    sg * __bfloat162float(qn[h * QD + pd]));
-                } else {
-#pragma unroll
-                    for (int h = 0; h < QHEADS; ++h) acc += __bfloat162float(qn[h * QD + d]);
-                }
-                qbar[d] = acc;
-            }
-            __syncthreads();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) qv[e] = qbar[16 * gl + e];
-            cur = n;
-        }
+        const int seg_end = min(it_end, item0[n + 1]);
         const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
         const int r0 = (it - item0[n]) * SCORE_TILE;
-        const int r1 = min(elig, r0 + SCORE_TILE);
-        const __nv_bfloat16 *kb = k_hat + (size_t)cu_blocks[n] * QD + 16 * gl;
-        float *sc = scores + cu_blocks[n];
+        const int r1 = min(elig, (seg_end - item0[n]) * SCORE_TILE);
+        const long long row0 = cu_blocks[n];
+        if (tid < QD) {                             // sum over heads of RoPE(q_h, q_pos)
+            const __nv_bfloat16 *qn = q + (size_t)n * QHEADS * QD;
+            const int d = tid;
+            float acc = 0.f;
+            if (d < QROPE) {
+                float sn, cs;
+                sincosf(reduced_angle((double)q_pos[n], rotary_freq(base, d & (QHALF - 1))), &sn, &cs);
+                const int pd = d ^ QHALF;           // rotation partner
+                const float sg = d < QHALF ? -sn : sn;
+#pragma unroll
+                for (int h = 0; h < QHEADS; ++h)
+                    acc += fmaf(__bfloat162float(qn[h * QD + d]), cs,
+                                sg * __bfloat162float(qn[h * QD + pd]));
+            } else {
+#pragma unroll
+                for (int h = 0; h < QHEADS; ++h) acc += __bfloat162float(qn[h * QD + d]);
+            }
+            qbar[d] = acc;
+        }
+        __syncthreads();
+        float qv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) qv[e] = qbar[16 * gl + e];
+        const __nv_bfloat16 *kb = k_hat + (size_t)row0 * QD + 16 * gl;
+        float *sc = scores + row0;
         for (int base_row = r0 + 4 * warp; base_row < r1; base_row += 32 * kScoreUnroll) {
             uint4 a[kScoreUnroll][2];
 #pragma unroll
@@ -327,48 +348,68 @@ __global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
                     s0 = fmaf(qv[2 * e], bf_lo(wv[e]), s0);
                     s1 = fmaf(qv[2 * e + 1], bf_hi(wv[e]), s1);
                 }
-                float s = s0 + s1;
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                float sum = s0 + s1;
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
                 const int row = base_row + g + 32 * u;
                 if (gl == 0 && row < r1) {
-                    sc[row] = s;
-                    atomicAdd(&hist[order_key(s) >> (32 - HBITS)], 1u);
+                    sc[row] = sum;
+                    atomicAdd(&hist[order_key(sum) >> (32 - HBITS)], 1u);
                 }
             }
         }
-    }
-    __syncthreads();
-    if (cur >= 0) {
+        __syncthreads();                            // hand this sequence's counts on
         for (int i = tid; i < HBINS; i += blockDim.x) {
             const uint32_t v = hist[i];
-            if (v) atomicAdd(&ws[cur].hist[i], v);
+            if (v) { atomicAdd(&ws[n].hist[i], v); hist[i] = 0; }
         }
+        // the CTA that completes the sequence's last work item derives its threshold
+        // (every thread fences its own counts before the one arrival on the item counter)
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const uint32_t mine = (uint32_t)(seg_end - it);
+            const uint32_t all = (uint32_t)(item0[n + 1] - item0[n]);
+            scratch[35] = (atomicAdd(&ws[n].items_done, mine) + mine == all) ? 1 : 0;
+            __threadfence();
+        }
+        __syncthreads();
+        if (scratch[35]) {
+            for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = __ldcg(&ws[n].hist[i]);
+            __syncthreads();
+            int thr, rank;
+            threshold_of(hist, elig, budget, scratch, scratch + 32, thr, rank);
+            if (tid == 0) { ws[n].thr_bin = thr; ws[n].rank = rank; }
+            __syncthreads();
+            for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = 0;
+            __syncthreads();
+        }
+        it = seg_end;
     }
-}
-
-// ----------------------------------------------------------------- threshold
-__global__ void __launch_bounds__(kFinishThreads) qsa_threshold_kernel(
-    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int total_blocks,
-    int budget, SeqWork *__restrict__ ws)
-{
-    __shared__ uint32_t h[HBINS];
-    __shared__ int scratch[36], res[3];
-    const int n = blockIdx.x;
-    SeqWork &w = ws[n];
-    const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
-    if (elig <= budget) {
-        if (threadIdx.x == 0) { w.thr_bin = -1; w.rank = elig; }
-        return;
-    }
-    for (int i = threadIdx.x; i < HBINS; i += blockDim.x) h[i] = w.hist[i];
-    __syncthreads();
-    find_from_top(h, HBINS, budget, scratch, res);
-    if (threadIdx.x == 0) { w.thr_bin = res[0]; w.rank = budget - res[1]; }
+    pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------- collect
+// Same contiguous work split as the score kernel (COLLECT_TILE scores per item); each
+// CTA derives the threshold of every sequence it touches from that sequence's histogram.
+constexpr int kCollectPer = COLLECT_TILE / kScoreThreads;      // scores per thread per item
+
+__device__ __forceinline__ void warp_append(bool pred, uint32_t key, uint32_t idx,
+                                            uint32_t *count, uint2 *list, uint32_t cap) {
+    const unsigned m = __ballot_sync(0xffffffffu, pred);
+    if (!m) return;
+    const int lane = threadIdx.x & 31;
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0;
+    if (lane == leader) base = atomicAdd(count, (uint32_t)__popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (pred) {
+        const uint32_t slot = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+        if (slot < cap) list[slot] = make_uint2(key, idx);
+    }
+}
+
 __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int N,
     int total_blocks, const float *__restrict__ scores, SeqWork *__restrict__ ws)
@@ -378,56 +419,104 @@ __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
     int *item0 = scratch + 36;
     build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, COLLECT_TILE);
     const int n_items = item0[N];
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const int per = (n_items + gridDim.x - 1) / gridDim.x;
+    int it = blockIdx.x * per;
+    const int it_end = min(n_items, it + per);
+    pdl_wait_primary();                             // scores and thresholds are complete
+    while (it < it_end) {
         const int n = seq_of_item(item0, N, it);
+        const int seg_end = min(it_end, item0[n + 1]);
+        const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
+        const int r0 = (it - item0[n]) * COLLECT_TILE;
+        const int r1 = min(elig, (seg_end - item0[n]) * COLLECT_TILE);
         SeqWork &w = ws[n];
         const int thr = w.thr_bin;
-        const int r0 = (it - item0[n]) * COLLECT_TILE;
-        const int r1 = min(eligible(cu_blocks, q_pos, n, total_blocks), r0 + COLLECT_TILE);
         const float *sc = scores + cu_blocks[n];
-        for (int row = r0 + threadIdx.x; row < r1; row += blockDim.x) {
-            const uint32_t key = order_key(sc[row]);
-            const int bin = (int)(key >> (32 - HBITS));
-            if (thr < 0 || bin > thr) {
-                const uint32_t slot = atomicAdd(&w.n_sure, 1u);
-                if (slot < SURE_CAP) w.sure[slot] = make_uint2(key, (uint32_t)row);
-            } else if (bin == thr) {
-                const uint32_t slot = atomicAdd(&w.n_cand, 1u);
-                if (slot < CAND_CAP) w.cand[slot] = make_uint2(key, (uint32_t)row);
+        // rows r0 + threadIdx.x + 256 j, all loads of a step issued before any is used;
+        // the loop bound is uniform over the CTA so the warp ballots see every lane
+        for (int b = r0; b < r1; b += COLLECT_TILE) {
+            float v[kCollectPer];
+#pragma unroll
+            for (int j = 0; j < kCollectPer; ++j) {
+                const int row = b + threadIdx.x + kScoreThreads * j;
+                v[j] = row < r1 ? __ldcg(sc + row) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < kCollectPer; ++j) {
+                const int row = b + threadIdx.x + kScoreThreads * j;
+                const uint32_t key = order_key(v[j]);
+                const int bin = (int)(key >> (32 - HBITS));
+                const bool in = row < r1;
+                warp_append(in && (thr < 0 || bin > thr), key, (uint32_t)row, &w.n_sure, w.sure,
+                            SURE_CAP);
+                warp_append(in && bin == thr, key, (uint32_t)row, &w.n_cand, w.cand, CAND_CAP);
             }
         }
+        it = seg_end;
     }
+    pdl_launch_dependents();
 }
 
 // -------------------------------------------------------------------- finish
+// One CTA per sequence.  Dynamic shared memory: the radix-pass histogram (2048 words), the
+// kept list (SURE_CAP pairs), the candidates (CAND_CAP pairs) and a bitmap of kept blocks
+// (kBitmapBlocks bits).  With at most kBitmapBlocks eligible blocks the kept set is marked
+// in the bitmap and written out in block order by one ordered compaction; longer caches
+// sort the kept list instead.
+constexpr int kPassBins = 2048;
+constexpr int kBitmapBlocks = 1 << 18;
+constexpr int kBitmapWords = kBitmapBlocks / 32;
+constexpr size_t kFinishSmem = kPassBins * 4 + SURE_CAP * 8 + CAND_CAP * 8 + kBitmapWords * 4;
+
 __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int total_blocks,
     int budget, const float *__restrict__ scores, SeqWork *__restrict__ ws,
-    int32_t *__restrict__ block_idx,
-    float *__restrict__ block_score, int32_t *__restrict__ token_idx)
+    int32_t *__restrict__ block_idx, float *__restrict__ block_score,
+    int32_t *__restrict__ token_idx)
 {
-    __shared__ uint2 sel[SURE_CAP];
-    __shared__ uint32_t h[2048];
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *h = reinterpret_cast<uint32_t *>(smem);
+    uint2 *sel = reinterpret_cast<uint2 *>(h + kPassBins);
+    uint2 *cand = sel + SURE_CAP;
+    uint32_t *bm = reinterpret_cast<uint32_t *>(cand + CAND_CAP);
     __shared__ int scratch[36], res[3], s_count;
     const int n = blockIdx.x, tid = threadIdx.x;
     SeqWork &w = ws[n];
     const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
-    const int thr = w.thr_bin;
-    const int n_sure = min((int)w.n_sure, SURE_CAP);
-    const uint32_t n_cand = w.n_cand;
+    const bool use_bitmap = elig <= kBitmapBlocks;
+    const int n_words = (elig + 31) / 32;
+    if (use_bitmap)
+        for (int i = tid; i < n_words; i += blockDim.x) bm[i] = 0u;
+    pdl_wait_primary();                             // the lists are complete
+    const int n_sure = elig > 0 ? min((int)w.n_sure, SURE_CAP) : 0;
+    const uint32_t n_cand = elig > 0 ? w.n_cand : 0u;
+    const bool listed = n_cand <= (uint32_t)CAND_CAP;
+    const int thr = elig > 0 ? w.thr_bin : -1;
+    int r = w.rank;
     if (tid == 0) s_count = 0;
-    for (int i = tid; i < n_sure; i += blockDim.x) sel[i] = w.sure[i];
+    // all list loads of a thread issued before any is stored
+#pragma unroll
+    for (int j = 0; j < SURE_CAP / kFinishThreads; ++j) {
+        const int i = tid + j * kFinishThreads;
+        if (i < n_sure) sel[i] = __ldcg(&w.sure[i]);
+    }
+    if (listed) {
+#pragma unroll
+        for (int j = 0; j < CAND_CAP / kFinishThreads; ++j) {
+            const uint32_t i = tid + j * kFinishThreads;
+            if (i < n_cand) cand[i] = __ldcg(&w.cand[i]);
+        }
+    }
     __syncthreads();
 
-    if (thr >= 0 && elig > 0) {
-        const bool listed = n_cand <= (uint32_t)CAND_CAP;
+    if (thr >= 0) {
         const float *sc = scores + cu_blocks[n];
-        // every candidate (order key, block) of the threshold bin, from the list or, when
-        // the bin overflowed it, from the scores themselves
+        // every candidate (order key, block) of the threshold bin: from shared memory, or,
+        // when the bin overflowed the list, from the scores themselves
         auto for_cand = [&](auto &&f) {
             if (listed) {
                 for (uint32_t i = tid; i < n_cand; i += blockDim.x) {
-                    const uint2 c = w.cand[i];
+                    const uint2 c = cand[i];
                     f(c.x, c.y);
                 }
             } else {
@@ -437,7 +526,6 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
                 }
             }
         };
-        int r = w.rank;                             // 1-based rank inside the bin
         uint32_t kmask = 0xffffffffu << (32 - HBITS), kval = (uint32_t)thr << (32 - HBITS);
         int eq = 0;
         for (int shift = 32 - HBITS - 10; shift >= 0; shift -= 10) {   // bits 19..10, 9..0
@@ -480,49 +568,82 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
         }
         for_cand([&](uint32_t key, uint32_t idx) {
             if (key > tau || (key == tau && idx <= iota)) {
-                const int slot = n_sure + atomicAdd(&s_count, 1);
-                if (slot < SURE_CAP) sel[slot] = make_uint2(key, idx);
+                if (use_bitmap) {
+                    atomicOr(&bm[idx >> 5], 1u << (idx & 31));
+                } else {
+                    const int slot = n_sure + atomicAdd(&s_count, 1);
+                    if (slot < SURE_CAP) sel[slot] = make_uint2(key, idx);
+                }
             }
         });
     }
+    if (use_bitmap)
+        for (int i = tid; i < n_sure; i += blockDim.x) atomicOr(&bm[sel[i].y >> 5], 1u << (sel[i].y & 31));
     __syncthreads();
-    const int count = min(thr >= 0 ? n_sure + s_count : n_sure, min(budget, SURE_CAP));
-
-    // sort the kept blocks by index (bitonic over the next power of two)
-    int P = 1;
-    while (P < count) P <<= 1;
-    for (int i = count + tid; i < P; i += blockDim.x) sel[i] = make_uint2(0u, 0xffffffffu);
-    __syncthreads();
-    for (int kk = 2; kk <= P; kk <<= 1) {
-        for (int j = kk >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < P; i += blockDim.x) {
-                const int ij = i ^ j;
-                if (ij > i) {
-                    const uint2 a = sel[i], b = sel[ij];
-                    const bool up = (i & kk) == 0;
-                    if ((a.y > b.y) == up) { sel[i] = b; sel[ij] = a; }
-                }
-            }
-            __syncthreads();
-        }
-    }
+    int count = min(thr >= 0 ? n_sure + s_count : n_sure, min(budget, SURE_CAP));
 
     int32_t *bi = block_idx + (size_t)n * budget;
-    for (int i = tid; i < budget; i += blockDim.x) bi[i] = i < count ? (int32_t)sel[i].y : -1;
-    if (block_score) {
-        float *bs = block_score + (size_t)n * budget;
-        for (int i = tid; i < budget; i += blockDim.x) bs[i] = i < count ? key_value(sel[i].x) : -INFINITY;
+    float *bs = block_score ? block_score + (size_t)n * budget : nullptr;
+    int32_t *ti = token_idx ? token_idx + (size_t)n * budget * QR : nullptr;
+    auto put = [&](int pos, uint2 e) {             // kept block e at output position pos
+        bi[pos] = (int32_t)e.y;
+        if (bs) bs[pos] = key_value(e.x);
+        if (ti) {
+#pragma unroll
+            for (int j = 0; j < QR; ++j) ti[pos * QR + j] = (int32_t)(QR * e.y + (uint32_t)j);
+        }
+    };
+    if (use_bitmap) {
+        // ordered compaction: thread t owns bitmap words [t per, (t + 1) per)
+        const float *sc = scores + cu_blocks[n];
+        const int per = (n_words + blockDim.x - 1) / blockDim.x;
+        const int w0 = tid * per, w1 = min(n_words, w0 + per);
+        int local = 0;
+        for (int i = w0; i < w1; ++i) local += __popc(bm[i]);
+        int total;
+        int pos = block_exclusive_scan(local, scratch, total);
+        count = min(total, min(budget, SURE_CAP));   // the bitmap holds the kept set
+        for (int i = w0; i < w1; ++i) {
+            uint32_t m = bm[i];
+            while (m) {
+                const int b = __ffs(m) - 1;
+                m &= m - 1;
+                const uint32_t idx = 32u * (uint32_t)i + (uint32_t)b;
+                if (pos < count) put(pos, make_uint2(order_key(__ldcg(sc + idx)), idx));
+                ++pos;
+            }
+        }
+    } else {
+        int P = 1;
+        while (P < count) P <<= 1;
+        for (int i = count + tid; i < P; i += blockDim.x) sel[i] = make_uint2(0u, 0xffffffffu);
+        __syncthreads();
+        for (int kk = 2; kk <= P; kk <<= 1) {
+            for (int j = kk >> 1; j > 0; j >>= 1) {
+                for (int i = tid; i < P; i += blockDim.x) {
+                    const int ij = i ^ j;
+                    if (ij > i) {
+                        const uint2 a = sel[i], b = sel[ij];
+                        const bool up = (i & kk) == 0;
+                        if ((a.y > b.y) == up) { sel[i] = b; sel[ij] = a; }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        for (int i = tid; i < count; i += blockDim.x) put(i, sel[i]);
     }
-    if (token_idx) {
-        int32_t *ti = token_idx + (size_t)n * budget * QR;
-        for (int t = tid; t < budget * QR; t += blockDim.x) {
-            const int i = t / QR;
-            ti[t] = i < count ? (int32_t)(QR * sel[i].y + (uint32_t)(t % QR)) : -1;
+    for (int i = count + tid; i < budget; i += blockDim.x) {
+        bi[i] = -1;
+        if (bs) bs[i] = -INFINITY;
+        if (ti) {
+#pragma unroll
+            for (int j = 0; j < QR; ++j) ti[i * QR + j] = -1;
         }
     }
     // leave the record zeroed for the next call
     for (int i = tid; i < HBINS; i += blockDim.x) w.hist[i] = 0;
-    if (tid == 0) { w.n_sure = 0; w.n_cand = 0; }
+    if (tid == 0) { w.n_sure = 0; w.n_cand = 0; w.items_done = 0; }
 }
 
 int sm_count() {
@@ -565,19 +686,38 @@ cudaError_t launch_qsa_index_decode(const void *q, const int32_t *q_pos, const v
     const size_t score_smem = HBINS * sizeof(uint32_t) + QD * sizeof(float) + items_smem;
     qsa_score_kernel<<<persistent, kScoreThreads, score_smem, stream>>>(
         static_cast<const __nv_bfloat16 *>(q), q_pos, static_cast<const __nv_bfloat16 *>(k_hat),
-        cu_blocks, N, (int)total_blocks, (double)rope_base, ws, scores);
+        cu_blocks, N, (int)total_blocks, budget, (double)rope_base, ws, scores);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    qsa_threshold_kernel<<<N, kFinishThreads, 0, stream>>>(q_pos, cu_blocks, (int)total_blocks,
-                                                           budget, ws);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    qsa_collect_kernel<<<persistent, kScoreThreads, items_smem, stream>>>(
-        q_pos, cu_blocks, N, (int)total_blocks, scores, ws);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    qsa_finish_kernel<<<N, kFinishThreads, 0, stream>>>(q_pos, cu_blocks, (int)total_blocks,
-                                                        budget, scores, ws, block_idx,
-                                                        block_score, token_idx);
-    return cudaGetLastError();
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(persistent);
+    cfg.blockDim = dim3(kScoreThreads);
+    cfg.dynamicSmemBytes = items_smem;
+    cfg.stream = stream;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, qsa_collect_kernel, q_pos, cu_blocks, N, (int)total_blocks,
+                           (const float *)scores, ws);
+    if (e != cudaSuccess) return e;
+    static unsigned long long attr_set = 0;        // > 48 KB of dynamic shared memory, per device
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (dev >= 64 || !(attr_set & bit)) {
+        e = cudaFuncSetAttribute(qsa_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kFinishSmem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set |= bit;
+    }
+    cfg.gridDim = dim3(N);
+    cfg.blockDim = dim3(kFinishThreads);
+    cfg.dynamicSmemBytes = kFinishSmem;
+    return cudaLaunchKernelEx(&cfg, qsa_finish_kernel, q_pos, cu_blocks, (int)total_blocks,
+                              budget, (const float *)scores, ws, block_idx, block_score,
+                              token_idx);
 }
 
 }  // namespace gdn

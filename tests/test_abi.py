@@ -256,10 +256,10 @@ def test_qsa_index_with_no_sequences_is_a_no_op(L):
 
 
 def test_qsa_workspace_size(L):
-    # per sequence: 4096-bin histogram, two counters, threshold and rank, 4096 kept and
-    # 8192 candidate (key, block) pairs; then one fp32 score per cached block (256-byte
-    # rounded)
-    rec = 4096 * 4 + 4 * 4 + 4096 * 8 + 8192 * 8
+    # per sequence: 4096-bin histogram, two counters, threshold and rank, the finished-item
+    # counter (padded to 16 bytes), 4096 kept and 8192 candidate (key, block) pairs; then
+    # one fp32 score per cached block (256-byte rounded)
+    rec = 4096 * 4 + 4 * 4 + 4 * 4 + 4096 * 8 + 8192 * 8
     assert L.gdn_qsa_index_workspace_size(3, 1000) == 3 * rec + 4096
     assert L.gdn_qsa_index_workspace_size(-1, 10) == 0
 

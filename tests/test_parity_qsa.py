@@ -209,3 +209,16 @@ def test_qsa_index_full_size():
     cub = inputs.qsa_offsets([nb] * len(sub), DEV)
     _check_index(x["q"][sub], x["q_pos"][sub], rows, cub, w.budget_blocks,
                  tuple(t[sub] for t in out))
+
+
+@pytest.mark.parametrize("budget", [512, 4096])
+def test_qsa_index_cache_past_the_bitmap(budget):
+    """300,000 eligible blocks (past the 262,144-block bitmap of the finish kernel, so the
+    kept list is sorted instead: by rank for <= 1024 kept blocks, bitonic above)."""
+    blocks = [300_000, 1000]
+    cub = inputs.qsa_offsets(blocks, DEV)
+    k_hat = inputs.qsa_cache(sum(blocks), 51, DEV)
+    q = inputs.qsa_queries(2, 52, DEV)
+    q_pos = torch.tensor([4 * b - 1 for b in blocks], dtype=torch.int32, device=DEV)
+    out = _run_index(q, q_pos, k_hat, cub, budget)
+    _check_index(q, q_pos, k_hat, cub, budget, out)
