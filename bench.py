@@ -480,7 +480,83 @@ def job_tokens_per_s(world: int, tokens_per_rank: int, ms_max: float) -> float:
     return world * tokens_per_rank / (ms_max * 1e-3)
 
 
+def qsa_workload(args):
+    w = inputs.qsa_workloads()[0]
+    if args.qsa_seqs != w.num_seqs:
+        w = inputs.QsaWorkload(f"qsa_decode_n{args.qsa_seqs}_ctx1m_budget2048",
+                               (w.ctx_lens[0],) * args.qsa_seqs, w.budget_blocks, w.index)
+    return w
+
+
+def qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world):
+    ms_qsa = max_over_ranks(sum(qtimes) / len(qtimes), world)
+    ms_cmp = max_over_ranks(sum(ctimes) / len(ctimes), world)
+    qsa_bytes = qsa_index_bytes(wq, q_blocks)
+    qsa_gbs = qsa_bytes / (ms_qsa * 1e-3) / 1e9
+    cmp_bytes = q_tokens * 256 + q_blocks * 256
+    cmp_gbs = cmp_bytes / (ms_cmp * 1e-3) / 1e9
+    qsa_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "qsa.cu")
+    scale = wq.num_seqs / 8          # the traffic entries are per launch of the 8-sequence case
+
+    def tr(key):
+        t = profiled_traffic(key, qsa_src)
+        return None if t is None else int(t * scale)
+
+    return {
+        "workload": wq.name, "value": world * wq.num_seqs / (ms_qsa * 1e-3),
+        "unit": "queries/s", "ms_per_call": ms_qsa, "calls": len(qtimes),
+        "budget_blocks": wq.budget_blocks, "cached_blocks": q_blocks,
+        "roofline": {"bound": "hbm", "achieved": qsa_gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": qsa_gbs / peaks["hbm_gbs"],
+                     "traffic": tr("qsa_score"),
+                     "peak_source": f"{peaks['source']} copy bandwidth",
+                     "algorithmic_bytes_per_launch": qsa_bytes,
+                     "timed": "the whole gdn_qsa_index_decode call (score, collect and finish "
+                              "kernels, calls back to back); the score kernel is the dominant one"},
+        "compress": {
+            "workload": f"{wq.num_seqs} x {wq.ctx_lens[0]} raw keys -> {q_blocks} blocks",
+            "value": world * q_tokens / (ms_cmp * 1e-3), "unit": "tokens/s",
+            "ms_per_call": ms_cmp, "calls": len(ctimes),
+            "roofline": {"bound": "hbm", "achieved": cmp_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": cmp_gbs / peaks["hbm_gbs"],
+                         "traffic": tr("qsa_compress"),
+                         "algorithmic_bytes_per_launch": cmp_bytes}},
+    }
+
+
+def run_qsa_only(args):
+    """--section qsa: the QSA indexer and compression alone (one JSON line)."""
+    rank, world, local = dist_init()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import linear_attention_token_b200 as gdn
+    gdn.lib()
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(device)
+    wq = qsa_workload(args)
+    barrier(world)
+    with ClockSampler(local) as clk:
+        qtimes, ctimes, q_blocks, q_tokens = time_qsa(gdn, wq, max(1, args.steps),
+                                                      max(args.warmup, 1), stream, device)
+        barrier(world)
+    sec = qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world)
+    line = {"metric": "QSA indexer queries/s on 1 B200; % of HBM roofline",
+            "value": sec["value"], "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 1), "ms_per_step": sec["ms_per_call"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; block cache ~ N(0, 1/4), query heads ~ N(0, 1))",
+            "config": {"workload": wq.name}, "qsa_indexer": sec,
+            "gpu_launches": 3 * len(qtimes) + len(ctimes), "clocks": clk.summary()}
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args):
+    if args.section == "qsa":
+        return run_qsa_only(args)
     rank, world, local = dist_init()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -505,7 +581,7 @@ def run_ours(args):
         bw_steps = max(1, min(args.steps, 3))
         btimes = time_backward(gdn, x, wp, bw_steps, 1, stream)
         barrier(world)
-        wq = inputs.qsa_workloads()[0]
+        wq = qsa_workload(args)
         q_steps = max(3, min(args.steps, 20))
         qtimes, ctimes, q_blocks, q_tokens = time_qsa(gdn, wq, q_steps, 3, stream, device)
         barrier(world)
@@ -532,13 +608,7 @@ def run_ours(args):
     ver_gbs = ver_bytes / (ms_verify_pass / v_calls * 1e-3) / 1e9
     ver_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode_multi.cu")
     dec_gbs = dec_bytes / (ms_dec_step * 1e-3) / 1e9
-    ms_qsa = max_over_ranks(sum(qtimes) / len(qtimes), world)
-    ms_cmp = max_over_ranks(sum(ctimes) / len(ctimes), world)
-    qsa_bytes = qsa_index_bytes(wq, q_blocks)
-    qsa_gbs = qsa_bytes / (ms_qsa * 1e-3) / 1e9
-    cmp_bytes = q_tokens * 256 + q_blocks * 256
-    cmp_gbs = cmp_bytes / (ms_cmp * 1e-3) / 1e9
-    qsa_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "qsa.cu")
+    qsa = qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world)
 
     line = {
         "metric": METRIC,
@@ -587,33 +657,14 @@ def run_ours(args):
             "kernel": "backward_kernel: exact sequential reverse pass, checkpoint every 64 "
                       "tokens, CUDA cores; bound by the per-head token chain",
         },
-        "qsa_indexer": {
-            "workload": wq.name, "value": world * wq.num_seqs / (ms_qsa * 1e-3),
-            "unit": "queries/s", "ms_per_call": ms_qsa, "calls": len(qtimes),
-            "budget_blocks": wq.budget_blocks, "cached_blocks": q_blocks,
-            "roofline": {"bound": "hbm", "achieved": qsa_gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": qsa_gbs / peaks["hbm_gbs"],
-                         "traffic": profiled_traffic("qsa_score", qsa_src),
-                         "peak_source": f"{peaks['source']} copy bandwidth",
-                         "algorithmic_bytes_per_launch": qsa_bytes,
-                         "timed": "the whole gdn_qsa_index_decode call (4 kernels); the score "
-                                  "kernel is the dominant one"},
-            "compress": {
-                "workload": f"{wq.num_seqs} x {wq.ctx_lens[0]} raw keys -> {q_blocks} blocks",
-                "value": world * q_tokens / (ms_cmp * 1e-3), "unit": "tokens/s",
-                "ms_per_call": ms_cmp, "calls": len(ctimes),
-                "roofline": {"bound": "hbm", "achieved": cmp_gbs, "peak": peaks["hbm_gbs"],
-                             "unit": "GB/s", "frac": cmp_gbs / peaks["hbm_gbs"],
-                             "traffic": profiled_traffic("qsa_compress", qsa_src),
-                             "algorithmic_bytes_per_launch": cmp_bytes}},
-        },
+        "qsa_indexer": qsa,
         "e2e": {"value": world * tok / (ms_e2e * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "path": "gdn_prefill via the C ABI; every step's pinned host inputs copied in and "
                         "outputs + final state copied out inside the timed region; consecutive "
                         "steps alternate two streams so copies overlap"},
         "gpu_launches": (args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls + bw_steps
-                         + 4 * len(qtimes) + len(ctimes)),
+                         + 3 * len(qtimes) + len(ctimes)),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -666,6 +717,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--section", choices=["all", "qsa"], default="all",
+                    help="qsa: time only the QSA indexer and compression (profiling aid)")
+    ap.add_argument("--qsa-seqs", type=int, default=8,
+                    help="sequences of the QSA workload (1,048,576 cached tokens each)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
