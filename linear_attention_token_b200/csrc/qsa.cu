@@ -395,21 +395,6 @@ __global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
 // CTA derives the threshold of every sequence it touches from that sequence's histogram.
 constexpr int kCollectPer = COLLECT_TILE / kScoreThreads;      // scores per thread per item
 
-__device__ __forceinline__ void warp_append(bool pred, uint32_t key, uint32_t idx,
-                                            uint32_t *count, uint2 *list, uint32_t cap) {
-    const unsigned m = __ballot_sync(0xffffffffu, pred);
-    if (!m) return;
-    const int lane = threadIdx.x & 31;
-    const int leader = __ffs(m) - 1;
-    uint32_t base = 0;
-    if (lane == leader) base = atomicAdd(count, (uint32_t)__popc(m));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (pred) {
-        const uint32_t slot = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
-        if (slot < cap) list[slot] = make_uint2(key, idx);
-    }
-}
-
 __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int N,
     int total_blocks, const float *__restrict__ scores, SeqWork *__restrict__ ws)
@@ -417,6 +402,7 @@ __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
     extern __shared__ __align__(16) unsigned char smem[];
     int *scratch = reinterpret_cast<int *>(smem);
     int *item0 = scratch + 36;
+    __shared__ uint32_t s_base[2];
     build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, COLLECT_TILE);
     const int n_items = item0[N];
     const int per = (n_items + gridDim.x - 1) / gridDim.x;
@@ -441,15 +427,40 @@ __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
                 const int row = b + threadIdx.x + kScoreThreads * j;
                 v[j] = row < r1 ? __ldcg(sc + row) : 0.f;
             }
+            // one reservation per list for the whole CTA: per-thread counts packed in one
+            // int (kept blocks in the low 16 bits, candidates in the high 16), one scan
+            uint32_t keys[kCollectPer];
+            unsigned sure_m = 0, cand_m = 0;
 #pragma unroll
             for (int j = 0; j < kCollectPer; ++j) {
                 const int row = b + threadIdx.x + kScoreThreads * j;
-                const uint32_t key = order_key(v[j]);
-                const int bin = (int)(key >> (32 - HBITS));
-                const bool in = row < r1;
-                warp_append(in && (thr < 0 || bin > thr), key, (uint32_t)row, &w.n_sure, w.sure,
-                            SURE_CAP);
-                warp_append(in && bin == thr, key, (uint32_t)row, &w.n_cand, w.cand, CAND_CAP);
+                keys[j] = order_key(v[j]);
+                const int bin = (int)(keys[j] >> (32 - HBITS));
+                if (row < r1) {
+                    if (thr < 0 || bin > thr) sure_m |= 1u << j;
+                    else if (bin == thr) cand_m |= 1u << j;
+                }
+            }
+            int total;
+            const int before = block_exclusive_scan(__popc(sure_m) | (__popc(cand_m) << 16), scratch,
+                                                    total);
+            if (threadIdx.x == 0) {
+                s_base[0] = (total & 0xffff) ? atomicAdd(&w.n_sure, (uint32_t)(total & 0xffff)) : 0u;
+                s_base[1] = (total >> 16) ? atomicAdd(&w.n_cand, (uint32_t)(total >> 16)) : 0u;
+            }
+            __syncthreads();
+            uint32_t slot_s = s_base[0] + (uint32_t)(before & 0xffff);
+            uint32_t slot_c = s_base[1] + (uint32_t)(before >> 16);
+#pragma unroll
+            for (int j = 0; j < kCollectPer; ++j) {
+                const uint32_t row = (uint32_t)(b + threadIdx.x + kScoreThreads * j);
+                if (sure_m & (1u << j)) {
+                    if (slot_s < SURE_CAP) w.sure[slot_s] = make_uint2(keys[j], row);
+                    ++slot_s;
+                } else if (cand_m & (1u << j)) {
+                    if (slot_c < CAND_CAP) w.cand[slot_c] = make_uint2(keys[j], row);
+                    ++slot_c;
+                }
             }
         }
         it = seg_end;
@@ -603,15 +614,21 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
         int total;
         int pos = block_exclusive_scan(local, scratch, total);
         count = min(total, min(budget, SURE_CAP));   // the bitmap holds the kept set
+        uint32_t *ord = reinterpret_cast<uint32_t *>(sel);   // kept blocks in block order
         for (int i = w0; i < w1; ++i) {
             uint32_t m = bm[i];
             while (m) {
                 const int b = __ffs(m) - 1;
                 m &= m - 1;
-                const uint32_t idx = 32u * (uint32_t)i + (uint32_t)b;
-                if (pos < count) put(pos, make_uint2(order_key(__ldcg(sc + idx)), idx));
+                if (pos < count) ord[pos] = 32u * (uint32_t)i + (uint32_t)b;
                 ++pos;
             }
+        }
+        __syncthreads();
+        // one output entry per thread: all score loads in flight at once
+        for (int i = tid; i < count; i += blockDim.x) {
+            const uint32_t idx = ord[i];
+            put(i, make_uint2(order_key(__ldcg(sc + idx)), idx));
         }
     } else {
         int P = 1;
