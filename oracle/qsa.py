@@ -150,3 +150,16 @@ def index_decode(q, q_pos, k_hat, cu_blocks, budget_blocks: int = BLOCK_BUDGET,
         tok = expand_tokens(kept, r)
         ti[n, :len(tok)] = tok
     return bi, bs, ti
+
+
+def index_multi(q, q_pos, k_hat, cu_blocks, budget_blocks: int = BLOCK_BUDGET, r: int = R,
+                rope_dims: int = ROPE_DIMS, base: float = ROPE_BASE):
+    """T consecutive query tokens per sequence against one cache (drafted tokens checked
+    together): q [N, T, H, D]; query j of sequence n sits at position q_pos[n] + j and is
+    indexed exactly as a single query there (index_decode), with its own causal cut.
+    Returns block_idx [N, T, budget], block_score [N, T, budget], token_idx [N, T, r budget]."""
+    q = np.asarray(q, np.float64)
+    N, T = q.shape[0], q.shape[1]
+    outs = [index_decode(q[:, j], np.asarray(q_pos, np.int64) + j, k_hat, cu_blocks,
+                         budget_blocks, r, rope_dims, base) for j in range(T)]
+    return tuple(np.stack([o[i] for o in outs], axis=1) for i in range(3))

@@ -239,3 +239,21 @@ def test_qsa_constants_from_the_pages():
     2048 tokens = 512 blocks."""
     assert (Q0.R, Q0.HEADS, Q0.ROPE_DIMS, Q0.D) == (4, 4, 64, 128)
     assert Q0.TOKEN_BUDGET == 2048 and Q0.BLOCK_BUDGET == 512
+
+
+def test_qsa_multi_query_is_per_query_indexing():
+    """T queries per sequence: query j equals a single query at q_pos + j (with its own
+    causal cut), checked exactly with the rotation off against the fraction brute force."""
+    rng = np.random.default_rng(12)
+    lens = (0, 17, 41, 64)
+    k, _, cu = _rand_int_case(rng, lens, 6, 4)
+    q = rng.integers(-3, 4, size=(len(lens), 3, 4, 6)).astype(np.float64)
+    q_pos = np.array([0, 12, 30, 61])
+    k_hat, cu_b = Q0.compress_keys(k, cu, rope_dims=0)
+    bi, bs, ti = Q0.index_multi(q, q_pos, k_hat, cu_b, budget_blocks=5, rope_dims=0)
+    assert bi.shape == (4, 3, 5) and ti.shape == (4, 3, 20)
+    for j in range(3):
+        want = _brute_index(k, q[:, j], cu, q_pos + j, 5)
+        for n, (_, kept, sc) in enumerate(want):
+            assert list(bi[n, j, :len(kept)]) == kept and np.all(bi[n, j, len(kept):] == -1)
+            assert np.array_equal(bs[n, j, :len(kept)], np.array([float(x) for x in sc]))
