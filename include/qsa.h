@@ -35,7 +35,8 @@ extern "C" {
 #define GDN_QSA_ROPE_DIMS 64     /* dims with rotary encoding (the first 64)           */
 #define GDN_QSA_HEADS 4          /* indexer query heads per token                      */
 #define GDN_QSA_MAX_BUDGET 4096  /* largest budget_blocks accepted                     */
-#define GDN_QSA_MAX_SEQS 4096    /* largest num_seqs accepted by the indexer           */
+#define GDN_QSA_MAX_SEQS 4096    /* largest num_seqs x n_queries accepted by the indexer */
+#define GDN_QSA_MAX_QUERIES 4    /* largest n_queries of gdn_qsa_index_multi            */
 
 /* Steps 1-2: compress keys into the block cache.
  *   k          : [T_total, 128] bf16, the indexer key of every token (before rotation).
@@ -79,6 +80,29 @@ gdn_status gdn_qsa_index_decode(const void *q, const int32_t *q_pos, const void 
                                 int64_t total_blocks, int32_t budget_blocks, float rope_base,
                                 int32_t *block_idx, float *block_score, int32_t *token_idx,
                                 void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of device workspace gdn_qsa_index_multi needs for n_queries queries per sequence
+ * (same zero-fill rule as gdn_qsa_index_workspace_size); 0 for n_queries outside
+ * 1..GDN_QSA_MAX_QUERIES. */
+size_t gdn_qsa_index_multi_workspace_size(int32_t num_seqs, int64_t total_blocks,
+                                          int32_t n_queries);
+
+/* Steps 3-5 for n_queries consecutive tokens per sequence (for instance drafted tokens
+ * checked together): query j of sequence n sits at position q_pos[n] + j and is indexed
+ * exactly as gdn_qsa_index_decode indexes a single query there, with its own causal cut.
+ * Each cache row is read once for all of a sequence's queries.
+ *   q          : [num_seqs, n_queries, 4, 128] bf16.
+ *   block_idx  : [num_seqs, n_queries, budget_blocks] int32, written.
+ *   block_score: [num_seqs, n_queries, budget_blocks] fp32 or NULL.
+ *   token_idx  : [num_seqs, n_queries, 4 * budget_blocks] int32 or NULL.
+ *   workspace  : gdn_qsa_index_multi_workspace_size bytes.
+ * The other arguments are those of gdn_qsa_index_decode.  GDN_ERR_UNSUPPORTED for
+ * n_queries outside 1..GDN_QSA_MAX_QUERIES or num_seqs x n_queries > GDN_QSA_MAX_SEQS. */
+gdn_status gdn_qsa_index_multi(const void *q, const int32_t *q_pos, const void *k_hat,
+                               const int32_t *cu_blocks, int32_t num_seqs, int64_t total_blocks,
+                               int32_t n_queries, int32_t budget_blocks, float rope_base,
+                               int32_t *block_idx, float *block_score, int32_t *token_idx,
+                               void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

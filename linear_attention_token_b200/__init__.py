@@ -12,7 +12,9 @@ from ._binding import (GDN_BF16, GDN_ERR_CUDA, GDN_ERR_INVALID_ARG, GDN_ERR_TIME
                        gdn_get_device_error, gdn_prefill, gdn_prefill_static_scratch,
                        gdn_prefill_workspace_size,
                        gdn_status_string, lib, prefill_workspace, gdn_qsa_compress,
-                       gdn_qsa_index_decode, gdn_qsa_index_workspace_size, qsa_index_workspace)
+                       gdn_qsa_index_decode, gdn_qsa_index_workspace_size, qsa_index_workspace,
+                       gdn_qsa_index_multi, gdn_qsa_index_multi_workspace_size,
+                       qsa_index_multi_workspace)
 
 __all__ = [
     "gdn_prefill", "gdn_prefill_static_scratch", "gdn_decode_step", "gdn_decode_multi", "gdn_backward", "gdn_get_device_error", "gdn_prefill_workspace_size",
@@ -20,5 +22,6 @@ __all__ = [
     "GDN_ERR_INVALID_ARG", "GDN_ERR_UNSUPPORTED", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_F32",
     "GDN_BF16", "GDN_FLAG_QK_L2NORM", "GDN_FLAG_FORCE_CUDA_CORE", "GDN_FLAG_GATE_LOGITS",
     "gdn_qsa_compress", "gdn_qsa_index_decode", "gdn_qsa_index_workspace_size",
-    "qsa_index_workspace",
+    "qsa_index_workspace", "gdn_qsa_index_multi", "gdn_qsa_index_multi_workspace_size",
+    "qsa_index_multi_workspace",
 ]

@@ -24,13 +24,14 @@ GDN_FLAG_GATE_LOGITS = 4
 
 # QSA indexer constants (include/qsa.h)
 GDN_QSA_R, GDN_QSA_DIM, GDN_QSA_ROPE_DIMS, GDN_QSA_HEADS = 4, 128, 64, 4
-GDN_QSA_MAX_BUDGET, GDN_QSA_MAX_SEQS = 4096, 4096
+GDN_QSA_MAX_BUDGET, GDN_QSA_MAX_SEQS, GDN_QSA_MAX_QUERIES = 4096, 4096, 4
 
 # every symbol include/gdn.h and include/qsa.h declare
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
             "gdn_get_device_error", "gdn_status_string", "gdn_prefill_static_scratch",
             "gdn_decode_multi", "gdn_backward", "gdn_backward_workspace_size",
-            "gdn_qsa_compress", "gdn_qsa_index_workspace_size", "gdn_qsa_index_decode")
+            "gdn_qsa_compress", "gdn_qsa_index_workspace_size", "gdn_qsa_index_decode",
+            "gdn_qsa_index_multi_workspace_size", "gdn_qsa_index_multi")
 
 _lib = None
 
@@ -76,6 +77,10 @@ def lib():
         L.gdn_qsa_index_workspace_size.restype = SZ
         L.gdn_qsa_index_decode.argtypes = [P, P, P, P, I32, I64, I32, F, P, P, P, P, SZ, P]
         L.gdn_qsa_index_decode.restype = ctypes.c_int
+        L.gdn_qsa_index_multi_workspace_size.argtypes = [I32, I64, I32]
+        L.gdn_qsa_index_multi_workspace_size.restype = SZ
+        L.gdn_qsa_index_multi.argtypes = [P, P, P, P, I32, I64, I32, I32, F, P, P, P, P, SZ, P]
+        L.gdn_qsa_index_multi.restype = ctypes.c_int
         L.gdn_get_device_error.argtypes = [P, P]
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -318,4 +323,42 @@ def gdn_qsa_index_decode(q, q_pos, k_hat, cu_blocks, budget_blocks: int = 512, *
         _dev(block_score, "block_score"), _dev(token_idx, "token_idx"),
         _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
     _check(st, "gdn_qsa_index_decode")
+    return block_idx, block_score, token_idx
+
+
+def gdn_qsa_index_multi_workspace_size(num_seqs: int, total_blocks: int, n_queries: int) -> int:
+    return int(lib().gdn_qsa_index_multi_workspace_size(num_seqs, total_blocks, n_queries))
+
+
+def qsa_index_multi_workspace(num_seqs: int, total_blocks: int, n_queries: int,
+                              device="cuda") -> torch.Tensor:
+    """A zero-filled workspace of the size gdn_qsa_index_multi needs."""
+    n = gdn_qsa_index_multi_workspace_size(num_seqs, total_blocks, n_queries)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def gdn_qsa_index_multi(q, q_pos, k_hat, cu_blocks, budget_blocks: int = 512, *,
+                        rope_base: float = 10000.0, workspace=None, block_idx=None,
+                        block_score=None, token_idx=None, want_scores: bool = True,
+                        want_tokens: bool = True, stream=None):
+    """Indexer for T consecutive tokens per sequence: q [N, T, 4, 128] bf16 (query j of
+    sequence n at position q_pos[n] + j), q_pos int32 [N], k_hat [total_blocks, 128] bf16,
+    cu_blocks int32 [N + 1].  Returns (block_idx [N, T, budget], block_score or None,
+    token_idx [N, T, 4 budget] or None)."""
+    N, T = q.shape[0], q.shape[1]
+    dev = q.device
+    if workspace is None:
+        workspace = qsa_index_multi_workspace(N, k_hat.shape[0], T, dev)
+    if block_idx is None:
+        block_idx = torch.empty(N, T, budget_blocks, dtype=torch.int32, device=dev)
+    if block_score is None and want_scores:
+        block_score = torch.empty(N, T, budget_blocks, dtype=torch.float32, device=dev)
+    if token_idx is None and want_tokens:
+        token_idx = torch.empty(N, T, GDN_QSA_R * budget_blocks, dtype=torch.int32, device=dev)
+    st = lib().gdn_qsa_index_multi(
+        _dev(q, "q"), _dev(q_pos, "q_pos"), _dev(k_hat, "k_hat"), _dev(cu_blocks, "cu_blocks"),
+        N, k_hat.shape[0], T, int(budget_blocks), float(rope_base), _dev(block_idx, "block_idx"),
+        _dev(block_score, "block_score"), _dev(token_idx, "token_idx"),
+        _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "gdn_qsa_index_multi")
     return block_idx, block_score, token_idx

@@ -35,15 +35,15 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const f
                             float *dbeta, float *dS0, const int32_t *cu, int N, long long T_dense,
                             long long T_total, int H_qk, int H_v, int dkk, int dvv,
                             gdn_dtype dtype, float scale, int opts, void *ws, cudaStream_t stream);
-size_t qsa_index_workspace_bytes(int N, long long total_blocks);
+size_t qsa_index_workspace_bytes(int N, long long total_blocks, int T);
 cudaError_t launch_qsa_compress(const void *k, const int32_t *cu_seqlens, const int32_t *cu_blocks,
                                 const int32_t *pos0, void *k_hat, int N, long long total_blocks,
                                 float rope_base, cudaStream_t stream);
-cudaError_t launch_qsa_index_decode(const void *q, const int32_t *q_pos, const void *k_hat,
-                                    const int32_t *cu_blocks, int N, long long total_blocks,
-                                    int budget, float rope_base, int32_t *block_idx,
-                                    float *block_score, int32_t *token_idx, void *workspace,
-                                    cudaStream_t stream);
+cudaError_t launch_qsa_index(const void *q, const int32_t *q_pos, const void *k_hat,
+                             const int32_t *cu_blocks, int N, long long total_blocks, int T,
+                             int budget, float rope_base, int32_t *block_idx,
+                             float *block_score, int32_t *token_idx, void *workspace,
+                             cudaStream_t stream);
 size_t static_scratch_capacity();
 cudaError_t static_scratch_ptr(void **out);
 }  // namespace gdn
@@ -342,19 +342,29 @@ GDN_API gdn_status gdn_qsa_compress(const void *k, const int32_t *cu_seqlens,
 GDN_API size_t gdn_qsa_index_workspace_size(int32_t num_seqs, int64_t total_blocks)
 {
     if (num_seqs < 0 || total_blocks < 0) return 0;
-    return gdn::qsa_index_workspace_bytes(num_seqs, total_blocks);
+    return gdn::qsa_index_workspace_bytes(num_seqs, total_blocks, 1);
 }
 
-GDN_API gdn_status gdn_qsa_index_decode(const void *q, const int32_t *q_pos, const void *k_hat,
-                                        const int32_t *cu_blocks, int32_t num_seqs,
-                                        int64_t total_blocks, int32_t budget_blocks,
-                                        float rope_base, int32_t *block_idx, float *block_score,
-                                        int32_t *token_idx, void *workspace,
-                                        size_t workspace_bytes, cudaStream_t stream)
+GDN_API size_t gdn_qsa_index_multi_workspace_size(int32_t num_seqs, int64_t total_blocks,
+                                                  int32_t n_queries)
 {
-    if (num_seqs < 0 || num_seqs > GDN_QSA_MAX_SEQS) return num_seqs < 0 ? GDN_ERR_INVALID_ARG
-                                                                          : GDN_ERR_UNSUPPORTED;
-    if (total_blocks < 0 || total_blocks > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    if (num_seqs < 0 || total_blocks < 0 || n_queries < 1 || n_queries > GDN_QSA_MAX_QUERIES)
+        return 0;
+    return gdn::qsa_index_workspace_bytes(num_seqs, total_blocks, n_queries);
+}
+
+namespace {
+gdn_status qsa_index(const void *q, const int32_t *q_pos, const void *k_hat,
+                     const int32_t *cu_blocks, int32_t num_seqs, int64_t total_blocks,
+                     int32_t n_queries, int32_t budget_blocks, float rope_base,
+                     int32_t *block_idx, float *block_score, int32_t *token_idx,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    if (n_queries < 1 || n_queries > GDN_QSA_MAX_QUERIES) return GDN_ERR_UNSUPPORTED;
+    if (num_seqs < 0) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)num_seqs * n_queries > GDN_QSA_MAX_SEQS) return GDN_ERR_UNSUPPORTED;
+    if (total_blocks < 0 || total_blocks > INT32_MAX / GDN_QSA_MAX_QUERIES)
+        return GDN_ERR_INVALID_ARG;
     if (budget_blocks < 1 || budget_blocks > GDN_QSA_MAX_BUDGET) return GDN_ERR_INVALID_ARG;
     if (!rope_base_ok(rope_base)) return GDN_ERR_INVALID_ARG;
     if (num_seqs == 0) return GDN_OK;
@@ -364,13 +374,39 @@ GDN_API gdn_status gdn_qsa_index_decode(const void *q, const int32_t *q_pos, con
         !aligned(cu_blocks, 4) || !aligned(block_idx, 4) || !aligned(block_score, 4) ||
         !aligned(token_idx, 4))
         return GDN_ERR_INVALID_ARG;
-    if (workspace_bytes < gdn::qsa_index_workspace_bytes(num_seqs, total_blocks))
+    if (workspace_bytes < gdn::qsa_index_workspace_bytes(num_seqs, total_blocks, n_queries))
         return GDN_ERR_INVALID_ARG;
-    const cudaError_t e = gdn::launch_qsa_index_decode(q, q_pos, k_hat, cu_blocks, num_seqs,
-                                                       total_blocks, budget_blocks, rope_base,
-                                                       block_idx, block_score, token_idx,
-                                                       workspace, stream);
+    const cudaError_t e = gdn::launch_qsa_index(q, q_pos, k_hat, cu_blocks, num_seqs,
+                                                total_blocks, n_queries, budget_blocks,
+                                                rope_base, block_idx, block_score, token_idx,
+                                                workspace, stream);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+}  // namespace
+
+GDN_API gdn_status gdn_qsa_index_decode(const void *q, const int32_t *q_pos, const void *k_hat,
+                                        const int32_t *cu_blocks, int32_t num_seqs,
+                                        int64_t total_blocks, int32_t budget_blocks,
+                                        float rope_base, int32_t *block_idx, float *block_score,
+                                        int32_t *token_idx, void *workspace,
+                                        size_t workspace_bytes, cudaStream_t stream)
+{
+    return qsa_index(q, q_pos, k_hat, cu_blocks, num_seqs, total_blocks, 1, budget_blocks,
+                     rope_base, block_idx, block_score, token_idx, workspace, workspace_bytes,
+                     stream);
+}
+
+GDN_API gdn_status gdn_qsa_index_multi(const void *q, const int32_t *q_pos, const void *k_hat,
+                                       const int32_t *cu_blocks, int32_t num_seqs,
+                                       int64_t total_blocks, int32_t n_queries,
+                                       int32_t budget_blocks, float rope_base,
+                                       int32_t *block_idx, float *block_score,
+                                       int32_t *token_idx, void *workspace,
+                                       size_t workspace_bytes, cudaStream_t stream)
+{
+    return qsa_index(q, q_pos, k_hat, cu_blocks, num_seqs, total_blocks, n_queries,
+                     budget_blocks, rope_base, block_idx, block_score, token_idx, workspace,
+                     workspace_bytes, stream);
 }
 
 GDN_API const char *gdn_status_string(gdn_status status)

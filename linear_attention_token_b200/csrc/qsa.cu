@@ -102,13 +102,18 @@ __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Blocks of sequence n the query may score: whole blocks at or before its position (and
-// inside the cache's total_blocks rows, whatever the offsets say).
+// Rows of sequence n in the cache (inside its total_blocks rows, whatever the offsets say).
+__device__ __forceinline__ int cached_rows(const int32_t *cu_blocks, int n, int total_blocks) {
+    const int end = cu_blocks[n + 1] < total_blocks ? cu_blocks[n + 1] : total_blocks;
+    return end > cu_blocks[n] ? end - cu_blocks[n] : 0;
+}
+
+// Blocks of sequence n that its query j (at position q_pos[n] + j) may score: whole blocks
+// at or before that position, inside the cache.
 __device__ __forceinline__ int eligible(const int32_t *cu_blocks, const int32_t *q_pos, int n,
-                                        int total_blocks) {
-    const long long end = cu_blocks[n + 1] < total_blocks ? cu_blocks[n + 1] : total_blocks;
-    const long long cached = end - cu_blocks[n];
-    const long long seen = ((long long)q_pos[n] + 1) / QR;
+                                        int total_blocks, int j = 0) {
+    const long long cached = cached_rows(cu_blocks, n, total_blocks);
+    const long long seen = ((long long)q_pos[n] + j + 1) / QR;
     const long long e = cached < seen ? cached : seen;
     return e > 0 ? (int)e : 0;
 }
@@ -142,24 +147,53 @@ __device__ int block_exclusive_scan(int v, int *scratch, int &total) {
     return before;
 }
 
-// item0[n] = first work item of sequence n, item0[N] = item count; a sequence gets
-// ceil(eligible / tile) items.  N <= GDN_QSA_MAX_SEQS.
-__device__ void build_items(int *item0, int *scratch, int N, const int32_t *cu_blocks,
-                            const int32_t *q_pos, int total_blocks, int tile) {
-    const int per = (N + blockDim.x - 1) / blockDim.x;
+// item0[m] = first work item of unit m, item0[M] = item count; a unit gets
+// ceil(eligible / tile) items.  Units are sequences (M = N, eligibility of their last query
+// T - 1, which sees the most blocks) or queries (M = N T, unit m = query m mod T of
+// sequence m / T).  M <= GDN_QSA_MAX_SEQS.
+__device__ __forceinline__ int unit_eligible(const int32_t *cu_blocks, const int32_t *q_pos,
+                                             int total_blocks, int m, int T, bool per_query) {
+    return per_query ? eligible(cu_blocks, q_pos, m / T, total_blocks, m % T)
+                     : eligible(cu_blocks, q_pos, m, total_blocks, T - 1);
+}
+
+__device__ void build_items(int *item0, int *scratch, int M, const int32_t *cu_blocks,
+                            const int32_t *q_pos, int total_blocks, int tile, int T,
+                            bool per_query) {
+    const int per = (M + blockDim.x - 1) / blockDim.x;
     const int m0 = threadIdx.x * per;
     int local = 0;
-    for (int m = m0; m < m0 + per && m < N; ++m)
-        local += (eligible(cu_blocks, q_pos, m, total_blocks) + tile - 1) / tile;
+    for (int m = m0; m < m0 + per && m < M; ++m)
+        local += (unit_eligible(cu_blocks, q_pos, total_blocks, m, T, per_query) + tile - 1) / tile;
     int total;
     int acc = block_exclusive_scan(local, scratch, total);
-    for (int m = m0; m < m0 + per && m < N; ++m) {
+    for (int m = m0; m < m0 + per && m < M; ++m) {
         item0[m] = acc;
-        acc += (eligible(cu_blocks, q_pos, m, total_blocks) + tile - 1) / tile;
+        acc += (unit_eligible(cu_blocks, q_pos, total_blocks, m, T, per_query) + tile - 1) / tile;
     }
-    if (threadIdx.x == 0) item0[N] = total;
+    if (threadIdx.x == 0) item0[M] = total;
     __syncthreads();
 }
+
+// TP values per lane -> lane l holds the sum over its aligned group of W lanes of value
+// (l mod TP): halving exchanges, then the remaining lane halves inside the group.
+template <int TP, int W>
+__device__ __forceinline__ float transpose_sum(float (&x)[TP], int lane) {
+#pragma unroll
+    for (int m = TP / 2; m >= 1; m >>= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < m; ++i) {
+            const float send = upper ? x[i] : x[i + m];
+            const float keep = upper ? x[i + m] : x[i];
+            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+#pragma unroll
+    for (int m = TP; m < W; m <<= 1) x[0] += __shfl_xor_sync(0xffffffffu, x[0], m);
+    return x[0];
+}
+
 
 // Largest n < N with item0[n] <= it (sequences without items are skipped).
 __device__ __forceinline__ int seq_of_item(const int *item0, int N, int it) {
@@ -268,27 +302,31 @@ __device__ void threshold_of(const uint32_t *h, int elig, int budget, int *scrat
 }
 
 // --------------------------------------------------------------------- score
-// Persistent CTAs; CTA c takes the contiguous run of work items [c per, (c + 1) per), so
-// it stays on one sequence for long stretches (one summed query and one histogram hand-off
-// per sequence it touches).  A group of 8 lanes owns a row (lane g owns dims
-// 16 g .. 16 g + 15, 32 bytes), a warp 4 rows per step, unrolled U steps deep so that
-// 4 KB per warp are in flight.
+// Persistent CTAs; CTA c takes the contiguous run of work items [c per, (c + 1) per) over
+// the sequences, so it stays on one sequence for long stretches (one set of summed queries
+// and one histogram hand-off per sequence it touches).  Each cache row is read once for all
+// T queries of its sequence (query j at position q_pos + j scores only the rows it may see).
+// A group of 8 lanes owns a row (lane g owns dims 16 g .. 16 g + 15, 32 bytes), a warp 4
+// rows per step, 4 steps deep (4 KB per warp in flight).  With T > 1 queries each lane
+// holds its 16 dims of all T summed queries; the T partial dots are summed over the group
+// transposed, so lane j of the group ends with query j's score.
 constexpr int kScoreUnroll = 4;
 
-__global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
+template <int T>
+__global__ void __launch_bounds__(kScoreThreads, T == 1 ? 4 : 2) qsa_score_kernel(
     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ q_pos,
     const __nv_bfloat16 *__restrict__ k_hat, const int32_t *__restrict__ cu_blocks, int N,
     int total_blocks, int budget, double base, SeqWork *__restrict__ ws,
     float *__restrict__ scores)
 {
     extern __shared__ __align__(16) unsigned char smem[];
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);
-    float *qbar = reinterpret_cast<float *>(hist + HBINS);
-    int *scratch = reinterpret_cast<int *>(qbar + QD);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem);               // [T][HBINS]
+    float *qbar = reinterpret_cast<float *>(hist + T * HBINS);          // [T][QD]
+    int *scratch = reinterpret_cast<int *>(qbar + T * QD);
     int *item0 = scratch + 36;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 3, gl = lane & 7;
-    for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = 0;
-    build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, SCORE_TILE);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < T * HBINS; i += blockDim.x) hist[i] = 0;
+    build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, SCORE_TILE, T, false);
     const int n_items = item0[N];
     const int per = (n_items + gridDim.x - 1) / gridDim.x;
     int it = blockIdx.x * per;
@@ -296,17 +334,22 @@ __global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
     while (it < it_end) {
         const int n = seq_of_item(item0, N, it);
         const int seg_end = min(it_end, item0[n + 1]);
-        const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
         const int r0 = (it - item0[n]) * SCORE_TILE;
-        const int r1 = min(elig, (seg_end - item0[n]) * SCORE_TILE);
+        const int r1 = min(eligible(cu_blocks, q_pos, n, total_blocks, T - 1),
+                           (seg_end - item0[n]) * SCORE_TILE);
         const long long row0 = cu_blocks[n];
-        if (tid < QD) {                             // sum over heads of RoPE(q_h, q_pos)
-            const __nv_bfloat16 *qn = q + (size_t)n * QHEADS * QD;
-            const int d = tid;
+        const int cached = cached_rows(cu_blocks, n, total_blocks);
+        int elig[T];
+#pragma unroll
+        for (int j = 0; j < T; ++j) elig[j] = eligible(cu_blocks, q_pos, n, total_blocks, j);
+        for (int e = tid; e < T * QD; e += blockDim.x) {   // sum over heads of RoPE(q_h, pos)
+            const int j = e / QD, d = e - j * QD;
+            const __nv_bfloat16 *qn = q + ((size_t)n * T + j) * QHEADS * QD;
             float acc = 0.f;
             if (d < QROPE) {
                 float sn, cs;
-                sincosf(reduced_angle((double)q_pos[n], rotary_freq(base, d & (QHALF - 1))), &sn, &cs);
+                sincosf(reduced_angle((double)q_pos[n] + j, rotary_freq(base, d & (QHALF - 1))),
+                        &sn, &cs);
                 const int pd = d ^ QHALF;           // rotation partner
                 const float sg = d < QHALF ? -sn : sn;
 #pragma unroll
@@ -317,71 +360,101 @@ __global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
 #pragma unroll
                 for (int h = 0; h < QHEADS; ++h) acc += __bfloat162float(qn[h * QD + d]);
             }
-            qbar[d] = acc;
+            qbar[e] = acc;
         }
         __syncthreads();
-        float qv[16];
+        float *sc = scores + (size_t)T * row0;     // query j's scores at sc + j * cached
+        {
+            constexpr int TP = T == 1 ? 1 : (T == 2 ? 2 : 4);
+            const int g = lane >> 3, gl = lane & 7;
+            float qv[T][16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) qv[e] = qbar[16 * gl + e];
-        const __nv_bfloat16 *kb = k_hat + (size_t)row0 * QD + 16 * gl;
-        float *sc = scores + row0;
-        for (int base_row = r0 + 4 * warp; base_row < r1; base_row += 32 * kScoreUnroll) {
-            uint4 a[kScoreUnroll][2];
+            for (int j = 0; j < T; ++j)
 #pragma unroll
-            for (int u = 0; u < kScoreUnroll; ++u) {
-                const int row = base_row + g + 32 * u;
-                if (row < r1) {
-                    a[u][0] = ld_stream(kb + (size_t)row * QD);
-                    a[u][1] = ld_stream(kb + (size_t)row * QD + 8);
-                } else {
-                    a[u][0] = make_uint4(0, 0, 0, 0);
-                    a[u][1] = make_uint4(0, 0, 0, 0);
+                for (int e = 0; e < 16; ++e) qv[j][e] = qbar[j * QD + 16 * gl + e];
+            const int jq = gl < T ? gl : 0;         // the query this lane reports
+            float *scq = sc + (size_t)jq * cached;
+            uint32_t *hq = hist + jq * HBINS;
+            const int eq = gl < T ? eligible(cu_blocks, q_pos, n, total_blocks, jq) : 0;
+            const __nv_bfloat16 *kb = k_hat + (size_t)row0 * QD + 16 * gl;
+            for (int base_row = r0 + 4 * warp; base_row < r1; base_row += 32 * kScoreUnroll) {
+                uint4 a[kScoreUnroll][2];
+#pragma unroll
+                for (int u = 0; u < kScoreUnroll; ++u) {
+                    const int row = base_row + g + 32 * u;
+                    if (row < r1) {
+                        a[u][0] = ld_stream(kb + (size_t)row * QD);
+                        a[u][1] = ld_stream(kb + (size_t)row * QD + 8);
+                    } else {
+                        a[u][0] = make_uint4(0, 0, 0, 0);
+                        a[u][1] = make_uint4(0, 0, 0, 0);
+                    }
                 }
-            }
 #pragma unroll
-            for (int u = 0; u < kScoreUnroll; ++u) {
-                const uint32_t wv[8] = {a[u][0].x, a[u][0].y, a[u][0].z, a[u][0].w,
-                                        a[u][1].x, a[u][1].y, a[u][1].z, a[u][1].w};
-                float s0 = 0.f, s1 = 0.f;
+                for (int u = 0; u < kScoreUnroll; ++u) {
+                    const uint32_t wv[8] = {a[u][0].x, a[u][0].y, a[u][0].z, a[u][0].w,
+                                            a[u][1].x, a[u][1].y, a[u][1].z, a[u][1].w};
+                    float kf[16];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    s0 = fmaf(qv[2 * e], bf_lo(wv[e]), s0);
-                    s1 = fmaf(qv[2 * e + 1], bf_hi(wv[e]), s1);
-                }
-                float sum = s0 + s1;
-                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-                const int row = base_row + g + 32 * u;
-                if (gl == 0 && row < r1) {
-                    sc[row] = sum;
-                    atomicAdd(&hist[order_key(sum) >> (32 - HBITS)], 1u);
+                    for (int e = 0; e < 8; ++e) { kf[2 * e] = bf_lo(wv[e]); kf[2 * e + 1] = bf_hi(wv[e]); }
+                    float p[TP > 1 ? TP : 1];
+#pragma unroll
+                    for (int j = 0; j < (TP > 1 ? TP : 1); ++j) p[j] = 0.f;
+#pragma unroll
+                    for (int j = 0; j < T; ++j) {
+                        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            s0 = fmaf(qv[j][2 * e], kf[2 * e], s0);
+                            s1 = fmaf(qv[j][2 * e + 1], kf[2 * e + 1], s1);
+                        }
+                        p[j] = s0 + s1;
+                    }
+                    float sum;
+                    if constexpr (T == 1) {
+                        sum = p[0];
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                    } else {
+                        sum = transpose_sum<TP, 8>(p, lane);
+                    }
+                    const int row = base_row + g + 32 * u;
+                    if (gl < T && row < eq) {
+                        scq[row] = sum;
+                        atomicAdd(&hq[order_key(sum) >> (32 - HBITS)], 1u);
+                    }
                 }
             }
         }
         __syncthreads();                            // hand this sequence's counts on
-        for (int i = tid; i < HBINS; i += blockDim.x) {
+        for (int i = tid; i < T * HBINS; i += blockDim.x) {
             const uint32_t v = hist[i];
-            if (v) { atomicAdd(&ws[n].hist[i], v); hist[i] = 0; }
+            if (v) { atomicAdd(&ws[(size_t)n * T + i / HBINS].hist[i % HBINS], v); hist[i] = 0; }
         }
-        // the CTA that completes the sequence's last work item derives its threshold
-        // (every thread fences its own counts before the one arrival on the item counter)
+        // the CTA that completes the sequence's last work item derives the thresholds of
+        // its T queries (every thread fences its own counts before the one arrival on the
+        // item counter)
         __threadfence();
         __syncthreads();
         if (tid == 0) {
             const uint32_t mine = (uint32_t)(seg_end - it);
             const uint32_t all = (uint32_t)(item0[n + 1] - item0[n]);
-            scratch[35] = (atomicAdd(&ws[n].items_done, mine) + mine == all) ? 1 : 0;
+            scratch[35] = (atomicAdd(&ws[(size_t)n * T].items_done, mine) + mine == all) ? 1 : 0;
             __threadfence();
         }
         __syncthreads();
         if (scratch[35]) {
-            for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = __ldcg(&ws[n].hist[i]);
-            __syncthreads();
-            int thr, rank;
-            threshold_of(hist, elig, budget, scratch, scratch + 32, thr, rank);
-            if (tid == 0) { ws[n].thr_bin = thr; ws[n].rank = rank; }
-            __syncthreads();
+#pragma unroll 1
+            for (int j = 0; j < T; ++j) {
+                SeqWork &wj = ws[(size_t)n * T + j];
+                for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = __ldcg(&wj.hist[i]);
+                __syncthreads();
+                int thr, rank;
+                threshold_of(hist, elig[j], budget, scratch, scratch + 32, thr, rank);
+                if (tid == 0) { wj.thr_bin = thr; wj.rank = rank; }
+                __syncthreads();
+            }
             for (int i = tid; i < HBINS; i += blockDim.x) hist[i] = 0;
             __syncthreads();
         }
@@ -396,49 +469,52 @@ __global__ void __launch_bounds__(kScoreThreads, 4) qsa_score_kernel(
 constexpr int kCollectPer = COLLECT_TILE / kScoreThreads;      // scores per thread per item
 
 __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
-    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int N,
+    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int N, int T,
     int total_blocks, const float *__restrict__ scores, SeqWork *__restrict__ ws)
 {
     extern __shared__ __align__(16) unsigned char smem[];
     int *scratch = reinterpret_cast<int *>(smem);
     int *item0 = scratch + 36;
     __shared__ uint32_t s_base[2];
-    build_items(item0, scratch, N, cu_blocks, q_pos, total_blocks, COLLECT_TILE);
-    const int n_items = item0[N];
+    const int U = N * T;                            // query units: query u % T of sequence u / T
+    build_items(item0, scratch, U, cu_blocks, q_pos, total_blocks, COLLECT_TILE, T, true);
+    const int n_items = item0[U];
     const int per = (n_items + gridDim.x - 1) / gridDim.x;
     int it = blockIdx.x * per;
     const int it_end = min(n_items, it + per);
     pdl_wait_primary();                             // scores and thresholds are complete
     while (it < it_end) {
-        const int n = seq_of_item(item0, N, it);
-        const int seg_end = min(it_end, item0[n + 1]);
-        const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
-        const int r0 = (it - item0[n]) * COLLECT_TILE;
-        const int r1 = min(elig, (seg_end - item0[n]) * COLLECT_TILE);
-        SeqWork &w = ws[n];
+        const int u = seq_of_item(item0, U, it);
+        const int n = u / T, j = u - n * T;
+        const int seg_end = min(it_end, item0[u + 1]);
+        const int elig = eligible(cu_blocks, q_pos, n, total_blocks, j);
+        const int r0 = (it - item0[u]) * COLLECT_TILE;
+        const int r1 = min(elig, (seg_end - item0[u]) * COLLECT_TILE);
+        SeqWork &w = ws[u];
         const int thr = w.thr_bin;
-        const float *sc = scores + cu_blocks[n];
-        // rows r0 + threadIdx.x + 256 j, all loads of a step issued before any is used;
+        const float *sc = scores + (size_t)T * cu_blocks[n] +
+                          (size_t)j * cached_rows(cu_blocks, n, total_blocks);
+        // rows r0 + threadIdx.x + 256 e, all loads of a step issued before any is used;
         // the loop bound is uniform over the CTA so the warp ballots see every lane
         for (int b = r0; b < r1; b += COLLECT_TILE) {
             float v[kCollectPer];
 #pragma unroll
-            for (int j = 0; j < kCollectPer; ++j) {
-                const int row = b + threadIdx.x + kScoreThreads * j;
-                v[j] = row < r1 ? __ldcg(sc + row) : 0.f;
+            for (int e = 0; e < kCollectPer; ++e) {
+                const int row = b + threadIdx.x + kScoreThreads * e;
+                v[e] = row < r1 ? __ldcg(sc + row) : 0.f;
             }
             // one reservation per list for the whole CTA: per-thread counts packed in one
             // int (kept blocks in the low 16 bits, candidates in the high 16), one scan
             uint32_t keys[kCollectPer];
             unsigned sure_m = 0, cand_m = 0;
 #pragma unroll
-            for (int j = 0; j < kCollectPer; ++j) {
-                const int row = b + threadIdx.x + kScoreThreads * j;
-                keys[j] = order_key(v[j]);
-                const int bin = (int)(keys[j] >> (32 - HBITS));
+            for (int e = 0; e < kCollectPer; ++e) {
+                const int row = b + threadIdx.x + kScoreThreads * e;
+                keys[e] = order_key(v[e]);
+                const int bin = (int)(keys[e] >> (32 - HBITS));
                 if (row < r1) {
-                    if (thr < 0 || bin > thr) sure_m |= 1u << j;
-                    else if (bin == thr) cand_m |= 1u << j;
+                    if (thr < 0 || bin > thr) sure_m |= 1u << e;
+                    else if (bin == thr) cand_m |= 1u << e;
                 }
             }
             int total;
@@ -452,13 +528,13 @@ __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
             uint32_t slot_s = s_base[0] + (uint32_t)(before & 0xffff);
             uint32_t slot_c = s_base[1] + (uint32_t)(before >> 16);
 #pragma unroll
-            for (int j = 0; j < kCollectPer; ++j) {
-                const uint32_t row = (uint32_t)(b + threadIdx.x + kScoreThreads * j);
-                if (sure_m & (1u << j)) {
-                    if (slot_s < SURE_CAP) w.sure[slot_s] = make_uint2(keys[j], row);
+            for (int e = 0; e < kCollectPer; ++e) {
+                const uint32_t row = (uint32_t)(b + threadIdx.x + kScoreThreads * e);
+                if (sure_m & (1u << e)) {
+                    if (slot_s < SURE_CAP) w.sure[slot_s] = make_uint2(keys[e], row);
                     ++slot_s;
-                } else if (cand_m & (1u << j)) {
-                    if (slot_c < CAND_CAP) w.cand[slot_c] = make_uint2(keys[j], row);
+                } else if (cand_m & (1u << e)) {
+                    if (slot_c < CAND_CAP) w.cand[slot_c] = make_uint2(keys[e], row);
                     ++slot_c;
                 }
             }
@@ -480,8 +556,8 @@ constexpr int kBitmapWords = kBitmapBlocks / 32;
 constexpr size_t kFinishSmem = kPassBins * 4 + SURE_CAP * 8 + CAND_CAP * 8 + kBitmapWords * 4;
 
 __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
-    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int total_blocks,
-    int budget, const float *__restrict__ scores, SeqWork *__restrict__ ws,
+    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ cu_blocks, int T,
+    int total_blocks, int budget, const float *__restrict__ scores, SeqWork *__restrict__ ws,
     int32_t *__restrict__ block_idx, float *__restrict__ block_score,
     int32_t *__restrict__ token_idx)
 {
@@ -491,9 +567,10 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
     uint2 *cand = sel + SURE_CAP;
     uint32_t *bm = reinterpret_cast<uint32_t *>(cand + CAND_CAP);
     __shared__ int scratch[36], res[3], s_count;
-    const int n = blockIdx.x, tid = threadIdx.x;
-    SeqWork &w = ws[n];
-    const int elig = eligible(cu_blocks, q_pos, n, total_blocks);
+    const int u = blockIdx.x, tid = threadIdx.x;   // query unit: query u % T of sequence u / T
+    const int n = u / T, jq = u - n * T;
+    SeqWork &w = ws[u];
+    const int elig = eligible(cu_blocks, q_pos, n, total_blocks, jq);
     const bool use_bitmap = elig <= kBitmapBlocks;
     const int n_words = (elig + 31) / 32;
     if (use_bitmap)
@@ -521,7 +598,8 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
     __syncthreads();
 
     if (thr >= 0) {
-        const float *sc = scores + cu_blocks[n];
+        const float *sc = scores + (size_t)T * cu_blocks[n] +
+                          (size_t)jq * cached_rows(cu_blocks, n, total_blocks);
         // every candidate (order key, block) of the threshold bin: from shared memory, or,
         // when the bin overflowed the list, from the scores themselves
         auto for_cand = [&](auto &&f) {
@@ -580,7 +658,7 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
         for_cand([&](uint32_t key, uint32_t idx) {
             if (key > tau || (key == tau && idx <= iota)) {
                 if (use_bitmap) {
-                    atomicOr(&bm[idx >> 5], 1u << (idx & 31));
+                    if (idx < (uint32_t)elig) atomicOr(&bm[idx >> 5], 1u << (idx & 31));
                 } else {
                     const int slot = n_sure + atomicAdd(&s_count, 1);
                     if (slot < SURE_CAP) sel[slot] = make_uint2(key, idx);
@@ -588,14 +666,17 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
             }
         });
     }
-    if (use_bitmap)
-        for (int i = tid; i < n_sure; i += blockDim.x) atomicOr(&bm[sel[i].y >> 5], 1u << (sel[i].y & 31));
+    if (use_bitmap)                                 // (entries are < elig; the test keeps the
+        for (int i = tid; i < n_sure; i += blockDim.x) {   //  bitmap in bounds whatever the lists hold)
+            const uint32_t idx = sel[i].y;
+            if (idx < (uint32_t)elig) atomicOr(&bm[idx >> 5], 1u << (idx & 31));
+        }
     __syncthreads();
     int count = min(thr >= 0 ? n_sure + s_count : n_sure, min(budget, SURE_CAP));
 
-    int32_t *bi = block_idx + (size_t)n * budget;
-    float *bs = block_score ? block_score + (size_t)n * budget : nullptr;
-    int32_t *ti = token_idx ? token_idx + (size_t)n * budget * QR : nullptr;
+    int32_t *bi = block_idx + (size_t)u * budget;
+    float *bs = block_score ? block_score + (size_t)u * budget : nullptr;
+    int32_t *ti = token_idx ? token_idx + (size_t)u * budget * QR : nullptr;
     auto put = [&](int pos, uint2 e) {             // kept block e at output position pos
         bi[pos] = (int32_t)e.y;
         if (bs) bs[pos] = key_value(e.x);
@@ -606,7 +687,8 @@ __global__ void __launch_bounds__(kFinishThreads) qsa_finish_kernel(
     };
     if (use_bitmap) {
         // ordered compaction: thread t owns bitmap words [t per, (t + 1) per)
-        const float *sc = scores + cu_blocks[n];
+        const float *sc = scores + (size_t)T * cu_blocks[n] +
+                          (size_t)jq * cached_rows(cu_blocks, n, total_blocks);
         const int per = (n_words + blockDim.x - 1) / blockDim.x;
         const int w0 = tid * per, w1 = min(n_words, w0 + per);
         int local = 0;
@@ -672,9 +754,9 @@ int sm_count() {
 
 }  // namespace
 
-size_t qsa_index_workspace_bytes(int N, long long total_blocks) {
-    const size_t rec = (size_t)N * sizeof(SeqWork);
-    return rec + (((size_t)total_blocks * sizeof(float) + 255) / 256) * 256;
+size_t qsa_index_workspace_bytes(int N, long long total_blocks, int T) {
+    const size_t rec = (size_t)N * T * sizeof(SeqWork);
+    return rec + (((size_t)total_blocks * T * sizeof(float) + 255) / 256) * 256;
 }
 
 cudaError_t launch_qsa_compress(const void *k, const int32_t *cu_seqlens, const int32_t *cu_blocks,
@@ -690,49 +772,76 @@ cudaError_t launch_qsa_compress(const void *k, const int32_t *cu_seqlens, const 
     return cudaGetLastError();
 }
 
-cudaError_t launch_qsa_index_decode(const void *q, const int32_t *q_pos, const void *k_hat,
-                                    const int32_t *cu_blocks, int N, long long total_blocks,
-                                    int budget, float rope_base, int32_t *block_idx,
-                                    float *block_score, int32_t *token_idx, void *workspace,
-                                    cudaStream_t stream) {
-    SeqWork *ws = static_cast<SeqWork *>(workspace);
-    float *scores = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) +
-                                              (size_t)N * sizeof(SeqWork));
-    const int persistent = sm_count() * 4;
-    const size_t items_smem = (size_t)(36 + N + 1) * sizeof(int);
-    const size_t score_smem = HBINS * sizeof(uint32_t) + QD * sizeof(float) + items_smem;
-    qsa_score_kernel<<<persistent, kScoreThreads, score_smem, stream>>>(
+namespace {
+
+// Opt a kernel in to more than 48 KB of dynamic shared memory, once per device.
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes, unsigned long long &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (dev < 64 && (done & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev < 64) done |= bit;
+    return e;
+}
+
+template <int T>
+cudaError_t launch_score(const void *q, const int32_t *q_pos, const void *k_hat,
+                         const int32_t *cu_blocks, int N, long long total_blocks, int budget,
+                         float rope_base, SeqWork *ws, float *scores, cudaStream_t stream) {
+    static unsigned long long done = 0;
+    const size_t fixed = (size_t)T * (HBINS * sizeof(uint32_t) + QD * sizeof(float));
+    const size_t smem = fixed + (size_t)(36 + N + 1) * sizeof(int);
+    // the limit is set once per device, so for the largest call (GDN_QSA_MAX_SEQS sequences)
+    cudaError_t e = allow_smem(qsa_score_kernel<T>,
+                               fixed + (size_t)(36 + GDN_QSA_MAX_SEQS + 1) * sizeof(int), done);
+    if (e != cudaSuccess) return e;
+    qsa_score_kernel<T><<<sm_count() * (T == 1 ? 4 : 2), kScoreThreads, smem, stream>>>(
         static_cast<const __nv_bfloat16 *>(q), q_pos, static_cast<const __nv_bfloat16 *>(k_hat),
         cu_blocks, N, (int)total_blocks, budget, (double)rope_base, ws, scores);
-    cudaError_t e = cudaGetLastError();
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_qsa_index(const void *q, const int32_t *q_pos, const void *k_hat,
+                             const int32_t *cu_blocks, int N, long long total_blocks, int T,
+                             int budget, float rope_base, int32_t *block_idx,
+                             float *block_score, int32_t *token_idx, void *workspace,
+                             cudaStream_t stream) {
+    SeqWork *ws = static_cast<SeqWork *>(workspace);
+    float *scores = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) +
+                                              (size_t)N * T * sizeof(SeqWork));
+    cudaError_t e;
+    switch (T) {
+    case 1: e = launch_score<1>(q, q_pos, k_hat, cu_blocks, N, total_blocks, budget, rope_base, ws, scores, stream); break;
+    case 2: e = launch_score<2>(q, q_pos, k_hat, cu_blocks, N, total_blocks, budget, rope_base, ws, scores, stream); break;
+    case 3: e = launch_score<3>(q, q_pos, k_hat, cu_blocks, N, total_blocks, budget, rope_base, ws, scores, stream); break;
+    case 4: e = launch_score<4>(q, q_pos, k_hat, cu_blocks, N, total_blocks, budget, rope_base, ws, scores, stream); break;
+    default: return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(persistent);
+    cfg.gridDim = dim3(sm_count() * 4);
     cfg.blockDim = dim3(kScoreThreads);
-    cfg.dynamicSmemBytes = items_smem;
+    cfg.dynamicSmemBytes = (size_t)(36 + N * T + 1) * sizeof(int);
     cfg.stream = stream;
     cfg.attrs = pdl;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, qsa_collect_kernel, q_pos, cu_blocks, N, (int)total_blocks,
+    e = cudaLaunchKernelEx(&cfg, qsa_collect_kernel, q_pos, cu_blocks, N, T, (int)total_blocks,
                            (const float *)scores, ws);
     if (e != cudaSuccess) return e;
-    static unsigned long long attr_set = 0;        // > 48 KB of dynamic shared memory, per device
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (dev >= 64 || !(attr_set & bit)) {
-        e = cudaFuncSetAttribute(qsa_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kFinishSmem);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set |= bit;
-    }
-    cfg.gridDim = dim3(N);
+    static unsigned long long finish_done = 0;
+    if ((e = allow_smem(qsa_finish_kernel, kFinishSmem, finish_done)) != cudaSuccess) return e;
+    cfg.gridDim = dim3(N * T);
     cfg.blockDim = dim3(kFinishThreads);
     cfg.dynamicSmemBytes = kFinishSmem;
-    return cudaLaunchKernelEx(&cfg, qsa_finish_kernel, q_pos, cu_blocks, (int)total_blocks,
+    return cudaLaunchKernelEx(&cfg, qsa_finish_kernel, q_pos, cu_blocks, T, (int)total_blocks,
                               budget, (const float *)scores, ws, block_idx, block_score,
                               token_idx);
 }

@@ -203,6 +203,13 @@ def qsa_queries(N: int, seed: int, device="cpu") -> torch.Tensor:
             .to(torch.bfloat16).contiguous())
 
 
+def qsa_multi_queries(N: int, T: int, seed: int, device="cpu") -> torch.Tensor:
+    """T consecutive query tokens per sequence: [N, T, 4, 128] bf16 ~ N(0, 1)."""
+    gen = torch.Generator(device=torch.device(device)).manual_seed(seed)
+    return (torch.randn(N, T, QSA_HEADS, QSA_DIM, generator=gen, device=device)
+            .to(torch.bfloat16).contiguous())
+
+
 def qsa_cache(total_blocks: int, seed: int, device="cpu") -> torch.Tensor:
     gen = torch.Generator(device=torch.device(device)).manual_seed(seed)
     return ((torch.randn(total_blocks, QSA_DIM, generator=gen, device=device) * 0.5)

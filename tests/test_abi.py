@@ -274,3 +274,39 @@ def test_qsa_constants_match_the_header():
     assert int(vals["GDN_QSA_HEADS"]) == b.GDN_QSA_HEADS == 4
     assert int(vals["GDN_QSA_MAX_BUDGET"]) == b.GDN_QSA_MAX_BUDGET
     assert int(vals["GDN_QSA_MAX_SEQS"]) == b.GDN_QSA_MAX_SEQS
+    assert int(vals["GDN_QSA_MAX_QUERIES"]) == b.GDN_QSA_MAX_QUERIES == 4
+
+
+def _qsa_multi(L, **over):
+    a = dict(q=A, qpos=A + 0x1000, k_hat=A + 0x2000, cub=A + 0x3000, N=2, nb=64, T=4,
+             budget=512, base=10000.0, bi=A + 0x4000, bs=None, ti=None, ws=A + 0x5000,
+             ws_bytes=1 << 40)
+    a.update(over)
+    return L.gdn_qsa_index_multi(P(a["q"]), P(a["qpos"]), P(a["k_hat"]), P(a["cub"]), a["N"],
+                                 a["nb"], a["T"], a["budget"], a["base"], P(a["bi"]), P(a["bs"]),
+                                 P(a["ti"]), P(a["ws"]), a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,expect", [
+    (dict(T=0), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(T=5), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(N=1025), gdn.GDN_ERR_UNSUPPORTED),                 # 1025 x 4 query units > 4096
+    (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(budget=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(ws_bytes=4096), gdn.GDN_ERR_INVALID_ARG),
+    (dict(bs=A + 0x6002), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_qsa_multi_rejects_on_host(L, over, expect):
+    assert _qsa_multi(L, **over) == expect
+
+
+def test_qsa_multi_with_no_sequences_is_a_no_op(L):
+    assert _qsa_multi(L, N=0, q=None, qpos=None, bi=None, ws=None) == gdn.GDN_OK
+
+
+def test_qsa_multi_workspace_size(L):
+    rec = 4096 * 4 + 4 * 4 + 4 * 4 + 4096 * 8 + 8192 * 8
+    # one record per (sequence, query), one fp32 score per (cached block, query)
+    assert L.gdn_qsa_index_multi_workspace_size(3, 1000, 4) == 12 * rec + 16128
+    assert L.gdn_qsa_index_multi_workspace_size(3, 1000, 1) == L.gdn_qsa_index_workspace_size(3, 1000)
+    assert L.gdn_qsa_index_multi_workspace_size(3, 1000, 5) == 0

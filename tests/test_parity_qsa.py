@@ -222,3 +222,76 @@ def test_qsa_index_cache_past_the_bitmap(budget):
     q_pos = torch.tensor([4 * b - 1 for b in blocks], dtype=torch.int32, device=DEV)
     out = _run_index(q, q_pos, k_hat, cub, budget)
     _check_index(q, q_pos, k_hat, cub, budget, out)
+
+
+# ------------------------------------------------------- T queries per sequence
+def _check_multi(q, q_pos, k_hat, cub, budget, out, exact_ties=False):
+    """Query j of every sequence against the oracle's single query at q_pos + j."""
+    bi, bs, ti = out
+    for j in range(q.shape[1]):
+        _check_index(q[:, j], q_pos + j, k_hat, cub, budget, (bi[:, j], bs[:, j], ti[:, j]),
+                     exact_ties)
+
+
+def _run_multi(q, q_pos, k_hat, cub, budget, ws=None):
+    out = gdn.gdn_qsa_index_multi(q, q_pos, k_hat, cub, budget, workspace=ws)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+def test_qsa_multi_ragged(T):
+    w = inputs.qsa_workloads()[1]
+    x = inputs.qsa_decode_inputs(w, DEV)
+    q = inputs.qsa_multi_queries(w.num_seqs, T, 61, DEV)
+    q_pos = torch.tensor([max(0, L - T) for L in w.ctx_lens], dtype=torch.int32, device=DEV)
+    out = _run_multi(q, q_pos, x["k_hat"], x["cu_blocks"], 512)
+    _check_multi(q, q_pos, x["k_hat"], x["cu_blocks"], 512, out)
+
+
+def test_qsa_multi_one_query_equals_decode():
+    w = inputs.qsa_workloads()[1]
+    x = inputs.qsa_decode_inputs(w, DEV)
+    a = _run_multi(x["q"][:, None].contiguous(), x["q_pos"], x["k_hat"], x["cu_blocks"], 300)
+    b = _run_index(x["q"], x["q_pos"], x["k_hat"], x["cu_blocks"], 300)
+    for u, v in zip(a, b):
+        assert torch.equal(u[:, 0], v)
+
+
+def test_qsa_multi_queries_cross_block_boundaries():
+    """Queries at 4b + 1 .. 4b + 4: block b becomes eligible at the third query, block b + 1
+    at none; and a sequence whose first queries see no whole block yet."""
+    blocks = [3000, 700, 5]
+    cub = inputs.qsa_offsets(blocks, DEV)
+    k_hat = inputs.qsa_cache(sum(blocks), 62, DEV)
+    q = inputs.qsa_multi_queries(3, 4, 63, DEV)
+    q_pos = torch.tensor([4 * 1999 + 1, 4 * 699 + 1, 0], dtype=torch.int32, device=DEV)
+    for budget in (512, 2000):
+        out = _run_multi(q, q_pos, k_hat, cub, budget)
+        _check_multi(q, q_pos, k_hat, cub, budget, out)
+
+
+def test_qsa_multi_exact_ties():
+    blocks = [9000, 30000]
+    cub = inputs.qsa_offsets(blocks, DEV)
+    k_hat = torch.cat([inputs.qsa_palette_cache(9000, 3, 64, DEV),
+                       inputs.qsa_palette_cache(30000, 1, 65, DEV)])
+    q = inputs.qsa_multi_queries(2, 3, 66, DEV)
+    q_pos = torch.tensor([4 * 9000 - 3, 4 * 30000 - 3], dtype=torch.int32, device=DEV)
+    out = _run_multi(q, q_pos, k_hat, cub, 512)
+    _check_multi(q, q_pos, k_hat, cub, 512, out, exact_ties=True)
+
+
+def test_qsa_multi_full_size():
+    """8 sequences x 262,144 blocks, 4 queries each (the multi-query bench workload);
+    sequences 0 and 5 checked block by block for all 4 queries."""
+    w = inputs.qsa_workloads()[0]
+    x = inputs.qsa_decode_inputs(w, DEV)
+    q = inputs.qsa_multi_queries(w.num_seqs, 4, 67, DEV)
+    q_pos = torch.tensor([L - 4 for L in w.ctx_lens], dtype=torch.int32, device=DEV)
+    out = _run_multi(q, q_pos, x["k_hat"], x["cu_blocks"], w.budget_blocks)
+    nb = w.blocks[0]
+    sub = [0, 5]
+    rows = torch.cat([x["k_hat"][i * nb:(i + 1) * nb] for i in sub])
+    cub = inputs.qsa_offsets([nb] * len(sub), DEV)
+    _check_multi(q[sub], q_pos[sub], rows, cub, w.budget_blocks, tuple(t[sub] for t in out))
