@@ -360,6 +360,20 @@ def time_qsa(gdn, wq, steps, warmup, stream, device):
         return [a.elapsed_time(b) for a, b in evs]
 
     itimes = timed(call, steps, warmup)
+    # the same caches with 4 query tokens per sequence (drafted tokens checked together)
+    Tq = 4
+    qm = inputs.qsa_multi_queries(N, Tq, inputs.QSA_SEED + 60, device)
+    qm_pos = torch.tensor([L - Tq for L in wq.ctx_lens], dtype=torch.int32, device=device)
+    wsm = gdn.qsa_index_multi_workspace(N, nb, Tq, device)
+    bim = torch.empty(N, Tq, wq.budget_blocks, dtype=torch.int32, device=device)
+    bsm = torch.empty(N, Tq, wq.budget_blocks, dtype=torch.float32, device=device)
+    tim = torch.empty(N, Tq, 4 * wq.budget_blocks, dtype=torch.int32, device=device)
+    mtimes = timed(lambda: gdn.gdn_qsa_index_multi(qm, qm_pos, x["k_hat"], x["cu_blocks"],
+                                                   wq.budget_blocks, workspace=wsm,
+                                                   block_idx=bim, block_score=bsm,
+                                                   token_idx=tim, stream=stream),
+                   steps, warmup)
+    del wsm
     T = sum(wq.ctx_lens)
     k = inputs.qsa_keys(T, inputs.QSA_SEED + 50, device)
     cu = inputs.qsa_offsets(wq.ctx_lens, device)
@@ -367,7 +381,7 @@ def time_qsa(gdn, wq, steps, warmup, stream, device):
     ctimes = timed(lambda: gdn.gdn_qsa_compress(k, cu, x["cu_blocks"], k_hat=k_hat,
                                                 stream=stream), max(1, min(steps, 5)), 1)
     del k, k_hat
-    return itimes, ctimes, nb, T
+    return itimes, ctimes, nb, T, mtimes
 
 
 def cpu_baseline_qsa(wq, seqs=2):
@@ -488,8 +502,12 @@ def qsa_workload(args):
     return w
 
 
-def qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world):
+def qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world, mtimes):
     ms_qsa = max_over_ranks(sum(qtimes) / len(qtimes), world)
+    ms_multi = max_over_ranks(sum(mtimes) / len(mtimes), world)
+    multi_bytes = q_blocks * 256 + wq.num_seqs * 4 * (4 * 128 * 2 + 4) + \
+        wq.num_seqs * 4 * wq.budget_blocks * (4 + 4 + 4 * 4)
+    multi_gbs = multi_bytes / (ms_multi * 1e-3) / 1e9
     ms_cmp = max_over_ranks(sum(ctimes) / len(ctimes), world)
     qsa_bytes = qsa_index_bytes(wq, q_blocks)
     qsa_gbs = qsa_bytes / (ms_qsa * 1e-3) / 1e9
@@ -513,6 +531,15 @@ def qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world):
                      "algorithmic_bytes_per_launch": qsa_bytes,
                      "timed": "the whole gdn_qsa_index_decode call (score, collect and finish "
                               "kernels, calls back to back); the score kernel is the dominant one"},
+        "multi_query": {
+            "workload": f"{wq.name} with 4 query tokens per sequence (drafted tokens, each at "
+                        f"its own position; one gdn_qsa_index_multi call)",
+            "value": world * wq.num_seqs * 4 / (ms_multi * 1e-3), "unit": "queries/s",
+            "ms_per_call": ms_multi, "calls": len(mtimes),
+            "roofline": {"bound": "hbm", "achieved": multi_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": multi_gbs / peaks["hbm_gbs"],
+                         "traffic": None, "algorithmic_bytes_per_launch": multi_bytes,
+                         "timed": "the whole call; the cache is read once for all 4 queries"}},
         "compress": {
             "workload": f"{wq.num_seqs} x {wq.ctx_lens[0]} raw keys -> {q_blocks} blocks",
             "value": world * q_tokens / (ms_cmp * 1e-3), "unit": "tokens/s",
@@ -536,17 +563,18 @@ def run_qsa_only(args):
     wq = qsa_workload(args)
     barrier(world)
     with ClockSampler(local) as clk:
-        qtimes, ctimes, q_blocks, q_tokens = time_qsa(gdn, wq, max(1, args.steps),
-                                                      max(args.warmup, 1), stream, device)
+        qtimes, ctimes, q_blocks, q_tokens, mtimes = time_qsa(gdn, wq, max(1, args.steps),
+                                                              max(args.warmup, 1), stream, device)
         barrier(world)
-    sec = qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world)
+    sec = qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world, mtimes)
     line = {"metric": "QSA indexer queries/s on 1 B200; % of HBM roofline",
             "value": sec["value"], "unit": "queries/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 1), "ms_per_step": sec["ms_per_call"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; block cache ~ N(0, 1/4), query heads ~ N(0, 1))",
             "config": {"workload": wq.name}, "qsa_indexer": sec,
-            "gpu_launches": 3 * len(qtimes) + len(ctimes), "clocks": clk.summary()}
+            "gpu_launches": 3 * len(qtimes) + 3 * len(mtimes) + len(ctimes),
+            "clocks": clk.summary()}
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -583,7 +611,7 @@ def run_ours(args):
         barrier(world)
         wq = qsa_workload(args)
         q_steps = max(3, min(args.steps, 20))
-        qtimes, ctimes, q_blocks, q_tokens = time_qsa(gdn, wq, q_steps, 3, stream, device)
+        qtimes, ctimes, q_blocks, q_tokens, mtimes = time_qsa(gdn, wq, q_steps, 3, stream, device)
         barrier(world)
     clocks = clk.summary()
     if status != 0:
@@ -608,7 +636,7 @@ def run_ours(args):
     ver_gbs = ver_bytes / (ms_verify_pass / v_calls * 1e-3) / 1e9
     ver_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode_multi.cu")
     dec_gbs = dec_bytes / (ms_dec_step * 1e-3) / 1e9
-    qsa = qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world)
+    qsa = qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world, mtimes)
 
     line = {
         "metric": METRIC,
@@ -664,7 +692,7 @@ def run_ours(args):
                         "outputs + final state copied out inside the timed region; consecutive "
                         "steps alternate two streams so copies overlap"},
         "gpu_launches": (args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls + bw_steps
-                         + 3 * len(qtimes) + len(ctimes)),
+                         + 3 * len(qtimes) + 3 * len(mtimes) + len(ctimes)),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
