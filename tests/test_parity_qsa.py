@@ -90,22 +90,25 @@ def test_qsa_compress_full_size_sampled():
 
 
 # -------------------------------------------------------------------- indexer
-def _tol(q, q_pos, k_hat_rows):
+def _tol(q, q_pos, k_hat_rows, scale=8e-6):
     qh = O.rope_partial(q, np.full(q.shape[0], q_pos))
-    return 8e-6 * (np.abs(k_hat_rows) @ np.abs(qh).sum(axis=0))
+    return scale * (np.abs(k_hat_rows) @ np.abs(qh).sum(axis=0))
 
 
-def _check_index(q, q_pos, k_hat, cu_blocks, budget, out, exact_ties=False):
+def _check_index(q, q_pos, k_hat, cu_blocks, budget, out, exact_ties=False, ref_rows=None,
+                 tol_scale=8e-6):
+    """ref_rows: the oracle's own cache (float64, from raw keys) when k_hat was written by
+    the kernel under test; tol_scale then also covers the cache's bf16 rounding."""
     bi, bs, ti = (t.cpu().numpy() for t in out)
     qn = q.float().cpu().numpy()
     qp = q_pos.cpu().numpy()
-    kh = k_hat.float().cpu().numpy()
+    kh = k_hat.float().cpu().numpy() if ref_rows is None else np.asarray(ref_rows, np.float64)
     cb = cu_blocks.cpu().numpy()
     for n in range(qn.shape[0]):
         e = O.eligible_blocks(cb[n + 1] - cb[n], int(qp[n]))
         rows = kh[cb[n]:cb[n] + e]
         s = O.block_scores(qn[n], int(qp[n]), rows)
-        t = _tol(qn[n], int(qp[n]), rows)
+        t = _tol(qn[n], int(qp[n]), rows, tol_scale)
         keep = min(e, budget)
         G = bi[n, :keep]
         assert np.all(bi[n, keep:] == -1) and np.all(np.isneginf(bs[n, keep:]))
@@ -295,3 +298,61 @@ def test_qsa_multi_full_size():
     rows = torch.cat([x["k_hat"][i * nb:(i + 1) * nb] for i in sub])
     cub = inputs.qsa_offsets([nb] * len(sub), DEV)
     _check_multi(q[sub], q_pos[sub], rows, cub, w.budget_blocks, tuple(t[sub] for t in out))
+
+
+# ------------------------------------------------------------- as a decode loop uses it
+def test_qsa_compress_incremental_equals_full():
+    """Compressing only the newest blocks (pos0 = their first token's position, rows at
+    their place in the cache) gives the rows of one full compression, bit for bit."""
+    L = 4 * 1000 + 3
+    k = inputs.qsa_keys(L, 81, DEV)
+    full = torch.empty(L // 4, 128, dtype=torch.bfloat16, device=DEV)
+    gdn.gdn_qsa_compress(k, inputs.qsa_offsets([L], DEV), inputs.qsa_offsets([L // 4], DEV),
+                         k_hat=full)
+    inc = torch.full_like(full, 3.0)
+    done = 0
+    for upto in (400, 1, 0, 599):                  # blocks compressed by each call
+        t0 = 4 * done
+        part = k[t0:t0 + 4 * upto]
+        view = inc[done:done + upto]
+        gdn.gdn_qsa_compress(part, inputs.qsa_offsets([4 * upto], DEV),
+                             inputs.qsa_offsets([upto], DEV), k_hat=view,
+                             pos0=torch.tensor([t0], dtype=torch.int32, device=DEV))
+        done += upto
+    torch.cuda.synchronize()
+    assert done == L // 4 and torch.equal(inc, full)
+
+
+def test_qsa_decode_loop_against_oracle():
+    """Eight decode steps of one sequence: append a key each step, compress a block when its
+    4th token arrives, index the new token's query; every step matches the oracle run on
+    the keys so far."""
+    T0 = 4 * 3000 + 1
+    steps = 8
+    keys = inputs.qsa_keys(T0 + steps, 82, DEV)
+    qs = inputs.qsa_queries(steps, 83, DEV)
+    cap = (T0 + steps) // 4
+    k_hat = torch.zeros(cap, 128, dtype=torch.bfloat16, device=DEV)
+    nb = T0 // 4
+    gdn.gdn_qsa_compress(keys[:4 * nb], inputs.qsa_offsets([4 * nb], DEV),
+                         inputs.qsa_offsets([nb], DEV), k_hat=k_hat[:nb])
+    ws = gdn.qsa_index_workspace(1, cap)
+    for s in range(steps):
+        t = T0 + s                                 # position of this step's token
+        if (t + 1) % 4 == 0:                       # its block is complete: compress it
+            b = t // 4
+            gdn.gdn_qsa_compress(keys[4 * b:4 * b + 4], inputs.qsa_offsets([4], DEV),
+                                 inputs.qsa_offsets([1], DEV), k_hat=k_hat[b:b + 1],
+                                 pos0=torch.tensor([4 * b], dtype=torch.int32, device=DEV))
+            nb = b + 1
+        cub = inputs.qsa_offsets([nb], DEV)
+        q_pos = torch.tensor([t], dtype=torch.int32, device=DEV)
+        out = _run_index(qs[s:s + 1], q_pos, k_hat[:nb], cub, 512, ws)
+        # the oracle builds its own cache from the raw keys of tokens 0..t (float64); the
+        # kernel's cache rounds each element to bf16 (at most 2^-8 of it), which the score
+        # tolerance covers on top of the fp32 arithmetic
+        ref_rows, _ = O.compress_keys(keys[:4 * nb].float().cpu().numpy(), [0, 4 * nb])
+        assert np.all(np.abs(k_hat[:nb].float().cpu().numpy() - ref_rows)
+                      <= 2.0 ** -8 * np.abs(ref_rows) + 1e-5)
+        _check_index(qs[s:s + 1], q_pos, k_hat[:nb], cub, 512, out, ref_rows=ref_rows,
+                     tol_scale=2.0 ** -8 + 8e-6)
