@@ -26,6 +26,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -103,13 +104,22 @@ def load_peaks():
             "source": "fallback"}
 
 
+def source_code_key(source_file: str) -> str:
+    """sha256 (first 16 hex digits) of a CUDA source with its comments and whitespace
+    removed: a comment-only edit keeps the key, any change to the code changes it."""
+    text = open(source_file).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()[:16]
+
+
 def profiled_traffic(kernel_key: str, source_file: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    kernel source as it is now (sha256 of the .cu file recorded in the summary)."""
+    kernel's code as it is now (source_code_key of the .cu file recorded in the summary)."""
     summary = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(summary):
         return None
-    sha = hashlib.sha256(open(source_file, "rb").read()).hexdigest()[:16]
+    sha = source_code_key(source_file)
     for line in open(summary):
         parts = line.split()
         if len(parts) >= 3 and parts[0] == kernel_key and parts[1] == sha:

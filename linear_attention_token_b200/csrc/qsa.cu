@@ -4,21 +4,24 @@
 // section "部品②: QSA").
 //
 //   qsa_compress_kernel   stream of 4 token keys in, one encoded block key out (HBM-bound).
-//   qsa_score_kernel      stream over the block cache: one fp32 score per eligible block
-//                         and a 4096-bin histogram of the scores' top 12 order bits per
-//                         sequence (HBM-bound; the dominant kernel of the indexer).
-//   qsa_collect_kernel    pass over the scores (L2-resident): from the histogram, the bin
-//                         that holds the budget-th score; blocks above it are kept, blocks
-//                         inside it become candidates.
-//   qsa_finish_kernel     per sequence: exact selection among the candidates (two radix
+//   qsa_score_kernel      stream over the block cache, each row read once for the T <= 4
+//                         queries of its sequence: one fp32 score per (query, eligible
+//                         block) and a 4096-bin histogram of the scores' top 12 order
+//                         bits per query (HBM-bound; the dominant kernel of the indexer).
+//                         The CTA that finishes a sequence's last work item derives each
+//                         query's threshold bin (the bin that holds the budget-th score).
+//   qsa_collect_kernel    pass over the scores (L2-resident): blocks above the threshold
+//                         bin are kept, blocks inside it become candidates.
+//   qsa_finish_kernel     per query: exact selection among the candidates (two radix
 //                         passes over the low score bits, then the block index for ties),
-//                         sort by block, write blocks / scores / tokens, re-zero the
-//                         sequence's workspace record.
+//                         blocks written in block order, with scores and tokens; the
+//                         query's workspace record is zeroed again.
 //
-// Scores are reduced to one query vector per sequence: the four heads share the key and
-// the logits are summed, so sum_h q_h . k = (sum_h q_h) . k.  Ranking compares 32-bit
-// order keys of the fp32 scores (a monotone map of the float's bits), and ties fall to
-// the smaller block index, which makes the kept set unique.
+// "Query units": query j of sequence n is unit n T + j; it sits at position q_pos[n] + j
+// and has its own causal cut.  Scores are reduced to one vector per query: its four heads
+// share the key and the logits are summed, so sum_h q_h . k = (sum_h q_h) . k.  Ranking
+// compares 32-bit order keys of the fp32 scores (a monotone map of the float's bits), and
+// ties fall to the smaller block index, which makes the kept set unique.
 #include <math.h>
 #include <stdint.h>
 
@@ -37,7 +40,8 @@ constexpr int SCORE_TILE = 512;                       // cache rows per scoring 
 constexpr int COLLECT_TILE = 4096;                    // score entries per collect work item
 constexpr int kScoreThreads = 256, kFinishThreads = 1024;
 
-// One sequence's record in the indexer workspace (zero between calls except thr/rank).
+// One query unit's record in the indexer workspace (zero between calls except thr/rank;
+// the score kernel counts a sequence's finished work items in its first unit's record).
 struct SeqWork {
     uint32_t hist[HBINS];     // scores per top-12-bit bin, filled by the score kernel
     uint32_t n_sure, n_cand;  // list lengths (n_cand counts past CAND_CAP too)
@@ -495,7 +499,7 @@ __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
         const float *sc = scores + (size_t)T * cu_blocks[n] +
                           (size_t)j * cached_rows(cu_blocks, n, total_blocks);
         // rows r0 + threadIdx.x + 256 e, all loads of a step issued before any is used;
-        // the loop bound is uniform over the CTA so the warp ballots see every lane
+        // the loop bound is uniform over the CTA, as the block scan below needs
         for (int b = r0; b < r1; b += COLLECT_TILE) {
             float v[kCollectPer];
 #pragma unroll
@@ -545,7 +549,7 @@ __global__ void __launch_bounds__(kScoreThreads) qsa_collect_kernel(
 }
 
 // -------------------------------------------------------------------- finish
-// One CTA per sequence.  Dynamic shared memory: the radix-pass histogram (2048 words), the
+// One CTA per query unit.  Dynamic shared memory: the radix-pass histogram (2048 words), the
 // kept list (SURE_CAP pairs), the candidates (CAND_CAP pairs) and a bitmap of kept blocks
 // (kBitmapBlocks bits).  With at most kBitmapBlocks eligible blocks the kept set is marked
 // in the bitmap and written out in block order by one ordered compaction; longer caches
