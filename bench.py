@@ -629,7 +629,8 @@ def run_ours(args):
 
     ms_prefill = max_over_ranks(sum(times) / len(times), world)
     ms_decode_pass = max_over_ranks(sum(dtimes) / len(dtimes), world)
-    e2e_times, h2d, d2h = time_prefill_e2e(gdn, wp, max(4, args.steps), 2, stream, device)
+    e2e_steps = max(4, args.steps)
+    e2e_times, h2d, d2h = time_prefill_e2e(gdn, wp, e2e_steps, 2, stream, device)
     ms_e2e = max_over_ranks(sum(e2e_times) / len(e2e_times), world)
 
     tok = wp.tokens
@@ -701,8 +702,10 @@ def run_ours(args):
                 "path": "gdn_prefill via the C ABI; every step's pinned host inputs copied in and "
                         "outputs + final state copied out inside the timed region; consecutive "
                         "steps alternate two streams so copies overlap"},
+        # our kernels inside timed regions: prefill steps, decode passes, multi-token calls,
+        # backward steps, the end-to-end prefill steps, and the QSA calls (3 kernels each)
         "gpu_launches": (args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls + bw_steps
-                         + 3 * len(qtimes) + 3 * len(mtimes) + len(ctimes)),
+                         + e2e_steps + 3 * len(qtimes) + 3 * len(mtimes) + len(ctimes)),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
