@@ -15,7 +15,9 @@ and the one-token concept code beside it):
 The arithmetic lives in ``gdn_oracle.c`` (plain C, compiled with gcc, no fast
 math); this module only marshals numpy arrays.  Every function here is pinned
 by tests/test_oracle.py (exact rational brute force, a hand-worked example,
-closed forms and invariants) and by tests/test_oracle_mutants.py.
+closed forms and invariants) and by tests/test_oracle_mutants.py.  The backward passes live
+in oracle/backward.py (sequential) and oracle/backward_chunked.py (chunked); the QSA
+indexer in oracle/qsa.py.
 """
 from __future__ import annotations
 
