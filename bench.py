@@ -548,7 +548,7 @@ def qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world, mtime
             "ms_per_call": ms_multi, "calls": len(mtimes),
             "roofline": {"bound": "hbm", "achieved": multi_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": multi_gbs / peaks["hbm_gbs"],
-                         "traffic": None, "algorithmic_bytes_per_launch": multi_bytes,
+                         "traffic": tr("qsa_score_t4"), "algorithmic_bytes_per_launch": multi_bytes,
                          "timed": "the whole call; the cache is read once for all 4 queries"}},
         "compress": {
             "workload": f"{wq.num_seqs} x {wq.ctx_lens[0]} raw keys -> {q_blocks} blocks",
