@@ -277,11 +277,28 @@ def gdn_get_device_error(workspace: torch.Tensor, stream=None) -> int:
 
 
 # ------------------------------------------------------------------ QSA indexer
+def _need(t, name, dtype, shape):
+    """Raise before anything reaches the library if a QSA argument has the wrong type or
+    shape (None in `shape` matches any size)."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != len(shape) or any(s is not None and s != d for s, d in zip(shape, t.shape)):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def gdn_qsa_compress(k, cu_seqlens, cu_blocks, *, k_hat, pos0=None, rope_base: float = 10000.0,
                      stream=None):
     """Block cache from indexer keys: k [T_total, 128] bf16 -> k_hat [total_blocks, 128] bf16
     (written in place and returned); cu_seqlens, cu_blocks int32 [N + 1], pos0 int32 [N]."""
     N = cu_seqlens.numel() - 1
+    _need(k, "k", torch.bfloat16, (None, GDN_QSA_DIM))
+    _need(k_hat, "k_hat", torch.bfloat16, (None, GDN_QSA_DIM))
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    _need(cu_blocks, "cu_blocks", torch.int32, (N + 1,))
+    if pos0 is not None:
+        _need(pos0, "pos0", torch.int32, (N,))
     st = lib().gdn_qsa_compress(
         _dev(k, "k"), _dev(cu_seqlens, "cu_seqlens"), _dev(cu_blocks, "cu_blocks"),
         _dev(pos0, "pos0"), _dev(k_hat, "k_hat"), N, k_hat.shape[0], float(rope_base),
@@ -308,6 +325,10 @@ def gdn_qsa_index_decode(q, q_pos, k_hat, cu_blocks, budget_blocks: int = 512, *
     k_hat [total_blocks, 128] bf16, cu_blocks int32 [N + 1].  Returns (block_idx [N, budget],
     block_score [N, budget] or None, token_idx [N, 4 budget] or None)."""
     N = q.shape[0]
+    _need(q, "q", torch.bfloat16, (N, GDN_QSA_HEADS, GDN_QSA_DIM))
+    _need(q_pos, "q_pos", torch.int32, (N,))
+    _need(k_hat, "k_hat", torch.bfloat16, (None, GDN_QSA_DIM))
+    _need(cu_blocks, "cu_blocks", torch.int32, (N + 1,))
     dev = q.device
     if workspace is None:
         workspace = qsa_index_workspace(N, k_hat.shape[0], dev)
@@ -346,6 +367,10 @@ def gdn_qsa_index_multi(q, q_pos, k_hat, cu_blocks, budget_blocks: int = 512, *,
     cu_blocks int32 [N + 1].  Returns (block_idx [N, T, budget], block_score or None,
     token_idx [N, T, 4 budget] or None)."""
     N, T = q.shape[0], q.shape[1]
+    _need(q, "q", torch.bfloat16, (N, T, GDN_QSA_HEADS, GDN_QSA_DIM))
+    _need(q_pos, "q_pos", torch.int32, (N,))
+    _need(k_hat, "k_hat", torch.bfloat16, (None, GDN_QSA_DIM))
+    _need(cu_blocks, "cu_blocks", torch.int32, (N + 1,))
     dev = q.device
     if workspace is None:
         workspace = qsa_index_multi_workspace(N, k_hat.shape[0], T, dev)

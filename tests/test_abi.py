@@ -310,3 +310,32 @@ def test_qsa_multi_workspace_size(L):
     assert L.gdn_qsa_index_multi_workspace_size(3, 1000, 4) == 12 * rec + 16128
     assert L.gdn_qsa_index_multi_workspace_size(3, 1000, 1) == L.gdn_qsa_index_workspace_size(3, 1000)
     assert L.gdn_qsa_index_multi_workspace_size(3, 1000, 5) == 0
+
+
+def test_qsa_binding_checks_types_and_shapes(L):
+    """Wrong dtypes or shapes raise in the binding before anything reaches the library
+    (these run on CPU tensors: the checks come before the device-pointer checks)."""
+    import torch
+    N = 2
+    q = torch.zeros(N, 4, 128, dtype=torch.bfloat16)
+    pos = torch.zeros(N, dtype=torch.int32)
+    kh = torch.zeros(10, 128, dtype=torch.bfloat16)
+    cub = torch.zeros(N + 1, dtype=torch.int32)
+    with pytest.raises(TypeError, match="k_hat"):
+        gdn.gdn_qsa_index_decode(q, pos, kh.float(), cub)
+    with pytest.raises(TypeError, match="q_pos"):
+        gdn.gdn_qsa_index_decode(q, pos.long(), kh, cub)
+    with pytest.raises(ValueError, match="q must have shape"):
+        gdn.gdn_qsa_index_decode(q[:, :3], pos, kh, cub)
+    with pytest.raises(ValueError, match="cu_blocks"):
+        gdn.gdn_qsa_index_decode(q, pos, kh, cub[:2])
+    with pytest.raises(ValueError, match="q must have shape"):
+        gdn.gdn_qsa_index_multi(q, pos, kh, cub)                  # needs [N, T, 4, 128]
+    with pytest.raises(TypeError, match="k must be"):
+        gdn.gdn_qsa_compress(torch.zeros(40, 128), cub, cub, k_hat=kh)
+    with pytest.raises(ValueError, match="pos0"):
+        gdn.gdn_qsa_compress(torch.zeros(40, 128, dtype=torch.bfloat16), cub, cub, k_hat=kh,
+                             pos0=torch.zeros(5, dtype=torch.int32))
+    # well-formed CPU tensors get as far as the device check
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        gdn.gdn_qsa_index_decode(q, pos, kh, cub)
