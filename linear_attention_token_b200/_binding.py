@@ -106,6 +106,18 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}; libgdn takes float32 or bfloat16")
 
 
+def _check_dtypes(q, same=(), f32=()):
+    """Every (name, tensor) in `same` must have q's dtype and every one in `f32` must be
+    float32 (None entries are skipped): a mismatch would otherwise be read as q's type."""
+    _dtype_code(q)
+    for name, t in same:
+        if t is not None and t.dtype != q.dtype:
+            raise TypeError(f"{name} must have q's dtype {q.dtype}, got {t.dtype}")
+    for name, t in f32:
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32, got {t.dtype}")
+
+
 def _dev(t: Optional[torch.Tensor], name: str):
     if t is None:
         return None
@@ -141,6 +153,8 @@ def gdn_prefill(q, k, v, g, beta, S0=None, cu_seqlens=None, *, out=None, S_final
     Varlen: q is [T_total, H_qk, dk] and cu_seqlens an int32 CUDA tensor [num_seqs + 1].
     Returns (out, S_final); S_final is None when want_state is False and none was given.
     """
+    _check_dtypes(q, (("k", k), ("v", v), ("out", out)),
+                  (("g", g), ("beta", beta), ("S0", S0), ("S_final", S_final)))
     if cu_seqlens is not None:
         T_total, H_qk, dk = q.shape[-3:]
         B, T, N = 1, T_total, cu_seqlens.numel() - 1
@@ -177,6 +191,8 @@ def gdn_prefill_static_scratch(q, k, v, g, beta, S0=None, cu_seqlens=None, *, ou
     static scratch.  ``out`` and ``S_final`` must be given (this call allocates nothing);
     S_final may be None to skip the final state.  Shapes as for gdn_prefill.
     """
+    _check_dtypes(q, (("k", k), ("v", v), ("out", out)),
+                  (("g", g), ("beta", beta), ("S0", S0), ("S_final", S_final)))
     if cu_seqlens is not None:
         T_total, H_qk, dk = q.shape[-3:]
         B, T, N = 1, T_total, cu_seqlens.numel() - 1
@@ -199,6 +215,8 @@ def gdn_prefill_static_scratch(q, k, v, g, beta, S0=None, cu_seqlens=None, *, ou
 def gdn_decode_step(q, k, v, g, beta, S_inout, *, out=None, scale: float = 1.0, flags: int = 0,
                     stream=None):
     """One decode step in place on S_inout [N, H_v, dk, dv]; q,k [N, H_qk, dk]; v [N, H_v, dv]."""
+    _check_dtypes(q, (("k", k), ("v", v), ("out", out)),
+                  (("g", g), ("beta", beta), ("S_inout", S_inout)))
     N, H_qk, dk = q.shape
     H_v, dv = v.shape[-2:]
     if out is None:
@@ -216,6 +234,8 @@ def gdn_decode_multi(q, k, v, g, beta, S_inout, *, n_commit=None, out=None, scal
     """T consecutive tokens per (sequence, head) in one call: q,k [N, T, H_qk, dk];
     v [N, T, H_v, dv]; g, beta [N, T, H_v].  S_inout [N, H_v, dk, dv] becomes the state
     after n_commit[n] tokens (int32 [N] on the device; None = all T).  Returns out."""
+    _check_dtypes(q, (("k", k), ("v", v), ("out", out)),
+                  (("g", g), ("beta", beta), ("S_inout", S_inout)))
     N, T, H_qk, dk = q.shape
     H_v, dv = v.shape[-2:]
     if out is None:
@@ -239,6 +259,8 @@ def gdn_backward(q, k, v, g, beta, d_out, S0=None, dS_final=None, cu_seqlens=Non
     Returns a dict of fp32 tensors dq, dk (like q), dv (like v), dg, dbeta (like g) and
     dS0 ([N, H_v, dk, dv], None when want_dS0 is False).
     """
+    _check_dtypes(q, (("k", k), ("v", v), ("d_out", d_out)),
+                  (("g", g), ("beta", beta), ("S0", S0), ("dS_final", dS_final)))
     if cu_seqlens is not None:
         T_total, H_qk, dk = q.shape[-3:]
         B, T, N = 1, T_total, cu_seqlens.numel() - 1

@@ -339,3 +339,28 @@ def test_qsa_binding_checks_types_and_shapes(L):
     # well-formed CPU tensors get as far as the device check
     with pytest.raises(ValueError, match="CUDA tensor"):
         gdn.gdn_qsa_index_decode(q, pos, kh, cub)
+
+
+def test_gdn_bindings_check_dtypes(L):
+    """A tensor whose dtype differs from q's (or a non-float32 gate or state) raises in the
+    binding instead of being read as the wrong type (CPU tensors: the checks come first)."""
+    import torch
+    bf, f32 = torch.bfloat16, torch.float32
+    q = torch.zeros(4, 2, 128, dtype=bf)
+    v = torch.zeros(4, 2, 128, dtype=bf)
+    g = torch.zeros(4, 2)
+    S = torch.zeros(4, 2, 128, 128)
+    with pytest.raises(TypeError, match="k must have"):
+        gdn.gdn_decode_step(q, q.float(), v, g, g, S)
+    with pytest.raises(TypeError, match="g must be float32"):
+        gdn.gdn_decode_step(q, q, v, g.to(bf), g, S)
+    with pytest.raises(TypeError, match="S_inout must be float32"):
+        gdn.gdn_decode_step(q, q, v, g, g, S.to(bf))
+    with pytest.raises(TypeError, match="v must have"):
+        gdn.gdn_prefill(q, q, v.float(), g, g)
+    with pytest.raises(TypeError, match="d_out must have"):
+        gdn.gdn_backward(q, q, v, g, g, v.float())
+    with pytest.raises(TypeError, match="S_inout must be float32"):
+        gdn.gdn_decode_multi(q[:, None], q[:, None], v[:, None], g[:, None], g[:, None], S.double())
+    with pytest.raises(ValueError, match="CUDA tensor"):      # consistent dtypes pass on
+        gdn.gdn_decode_step(q, q, v, g, g, S)
