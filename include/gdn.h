@@ -49,7 +49,8 @@ typedef enum {
 
 typedef enum {
     GDN_F32 = 0,               /* q, k, v, out in fp32 (CUDA-core kernels)             */
-    GDN_BF16 = 1               /* q, k, v, out in bf16 (tensor-core prefill, dk=dv=128) */
+    GDN_BF16 = 1               /* q, k, v, out in bf16 (tensor-core prefill for dk=dv=128;
+                                  other head dims run on the CUDA-core kernels)         */
 } gdn_dtype;
 
 /* L2-normalise q and k per (token, head) inside the kernel: x / sqrt(sum x^2 + 1e-6). */
@@ -61,9 +62,16 @@ typedef enum {
  * beta = sigmoid(b) (in (0, 1)) as they load them, in fp32. */
 #define GDN_FLAG_GATE_LOGITS 4u
 
-/* Bytes of device workspace gdn_prefill needs for these sizes (at least 256).
- * The workspace holds the device error word; it must be zero-filled before its
- * first use and must stay allocated while work that uses it is in flight. */
+/* Bytes of device workspace that let gdn_prefill use its fastest schedule for these
+ * sizes on the current device (at least 256).  The first 16 bytes hold the device
+ * error word; they must be zero-filled before first use.  When few (sequence, value
+ * head) pairs would leave most SMs idle (long sequences, few heads), the bf16 tensor-core
+ * path splits each sequence into segments that run in parallel; the rest of this size
+ * then holds each segment's state transfer (two dk x dk / dk x dv fp32 matrices) and
+ * start state.  gdn_prefill accepts any workspace of at least 256 bytes: a smaller one
+ * than this size makes it run one unit per sequence (same results, less parallelism).
+ * The workspace must stay allocated while work that uses it is in flight, and calls
+ * that share one must not overlap on the GPU. */
 size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t T_total, int32_t H_v, int32_t dk,
                                   int32_t dv);
 
@@ -174,14 +182,18 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, const float
  * that the library keeps in every GPU that loads it, for as long as the library is
  * loaded; it calls no cudaMalloc, cudaFree or other allocating routine.
  *   - The first call on a device looks up that array's device address (with that
- *     device current); make this first call before any stream capture.
+ *     device current); make this first call before any stream capture.  The address
+ *     is cached per device and looked up again when the device's context changes (for
+ *     instance after cudaDeviceReset).
  *   - Every call on a device shares the one array: calls that may overlap on the GPU
  *     (different streams, or different host threads) race on it.
  *   - Each call clears the array's error word before it launches.  A device-side
  *     timeout on this path is recorded there but not reported back (there is no
  *     workspace to hand to gdn_get_device_error).
- *   - Returns GDN_ERR_UNSUPPORTED if these sizes need more scratch than
- *     GDN_STATIC_SCRATCH_BYTES (gdn_prefill_workspace_size(...) > the maximum). */
+ *   - It always runs one unit per sequence (the segmented schedule would need a
+ *     workspace that grows with the sizes), so it needs only the 256-byte error
+ *     area; it returns GDN_ERR_UNSUPPORTED if that ever exceeded
+ *     GDN_STATIC_SCRATCH_BYTES. */
 #define GDN_STATIC_SCRATCH_BYTES 4096u
 gdn_status gdn_prefill_static_scratch(const void *q, const void *k, const void *v,
                                       const float *g, const float *beta, const float *S0,
@@ -189,6 +201,31 @@ gdn_status gdn_prefill_static_scratch(const void *q, const void *k, const void *
                                       int32_t num_seqs, int32_t B, int64_t T, int32_t H_qk,
                                       int32_t H_v, int32_t dk, int32_t dv, gdn_dtype dtype,
                                       float scale, uint32_t flags, cudaStream_t stream);
+
+/* Scheduling override for the bf16 tensor-core prefill (process-wide, for later calls).
+ * There are two kernels: one CTA per (sequence or segment, value head) carrying all 128
+ * value columns, and a cluster of four CTAs per (sequence, value head) that splits the
+ * value columns and shares each chunk's preparation.
+ *    0  automatic (default): a cost model of the device's SM count picks the kernel and,
+ *       for the first, whether to segment long sequences;
+ *   -1  the single-CTA kernel, one unit per sequence;
+ *   -2  the four-CTA cluster kernel;
+ *   >0  the single-CTA kernel with segments of exactly this many tokens (a multiple of
+ *       64) whenever the workspace is large enough (gdn_prefill_workspace_size accounts
+ *       for the override).
+ * Results do not depend on the schedule beyond rounding.  GDN_ERR_INVALID_ARG for other
+ * values. */
+gdn_status gdn_set_prefill_segment_tokens(int32_t tokens);
+
+/* Every device-side wait of the tensor-core prefill polls its barrier at most this many
+ * times (each poll suspends the thread for at most 2 microseconds, less when the awaited
+ * phase completes) before the kernel gives up and records GDN_ERR_TIMEOUT: with the
+ * default, a wait gives up after at most about 2 seconds.  gdn_set_wait_budget sets the process-wide limit for later launches and
+ * returns the previous one; 0 makes every wait give up at once, which exercises the
+ * recovery path (the kernel drains its own copies and MMAs and exits; the context stays
+ * usable).  The drains after a timeout always use the default limit. */
+#define GDN_DEFAULT_WAIT_BUDGET (1u << 20)
+uint32_t gdn_set_wait_budget(uint32_t polls);
 
 /* Synchronises `stream`, returns the first device-side error recorded in
  * `workspace` (GDN_OK if none) and clears it.  GDN_ERR_CUDA if the stream itself

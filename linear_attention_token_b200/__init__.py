@@ -10,7 +10,8 @@ from ._binding import (GDN_BF16, GDN_ERR_CUDA, GDN_ERR_INVALID_ARG, GDN_ERR_TIME
                        GDN_FLAG_GATE_LOGITS, GDN_FLAG_QK_L2NORM, GDN_OK, EXPORTED, GdnError, gdn_backward, gdn_decode_multi,
                        gdn_decode_step,
                        gdn_get_device_error, gdn_prefill, gdn_prefill_static_scratch,
-                       gdn_prefill_workspace_size,
+                       gdn_prefill_workspace_size, gdn_set_prefill_segment_tokens,
+                       gdn_set_wait_budget,
                        gdn_status_string, lib, prefill_workspace, gdn_qsa_compress,
                        gdn_qsa_index_decode, gdn_qsa_index_workspace_size, qsa_index_workspace,
                        gdn_qsa_index_multi, gdn_qsa_index_multi_workspace_size,
@@ -23,5 +24,5 @@ __all__ = [
     "GDN_BF16", "GDN_FLAG_QK_L2NORM", "GDN_FLAG_FORCE_CUDA_CORE", "GDN_FLAG_GATE_LOGITS",
     "gdn_qsa_compress", "gdn_qsa_index_decode", "gdn_qsa_index_workspace_size",
     "qsa_index_workspace", "gdn_qsa_index_multi", "gdn_qsa_index_multi_workspace_size",
-    "qsa_index_multi_workspace",
+    "qsa_index_multi_workspace", "gdn_set_prefill_segment_tokens", "gdn_set_wait_budget",
 ]

@@ -31,7 +31,8 @@ EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
             "gdn_get_device_error", "gdn_status_string", "gdn_prefill_static_scratch",
             "gdn_decode_multi", "gdn_backward", "gdn_backward_workspace_size",
             "gdn_qsa_compress", "gdn_qsa_index_workspace_size", "gdn_qsa_index_decode",
-            "gdn_qsa_index_multi_workspace_size", "gdn_qsa_index_multi")
+            "gdn_qsa_index_multi_workspace_size", "gdn_qsa_index_multi",
+            "gdn_set_wait_budget", "gdn_set_prefill_segment_tokens")
 
 _lib = None
 
@@ -81,6 +82,10 @@ def lib():
         L.gdn_qsa_index_multi_workspace_size.restype = SZ
         L.gdn_qsa_index_multi.argtypes = [P, P, P, P, I32, I64, I32, I32, F, P, P, P, P, SZ, P]
         L.gdn_qsa_index_multi.restype = ctypes.c_int
+        L.gdn_set_wait_budget.argtypes = [U32]
+        L.gdn_set_wait_budget.restype = U32
+        L.gdn_set_prefill_segment_tokens.argtypes = [I32]
+        L.gdn_set_prefill_segment_tokens.restype = ctypes.c_int
         L.gdn_get_device_error.argtypes = [P, P]
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -131,6 +136,18 @@ def _dev(t: Optional[torch.Tensor], name: str):
 def _stream(stream) -> ctypes.c_void_p:
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def gdn_set_wait_budget(polls: int) -> int:
+    """Set the poll limit of every device-side wait of the tensor-core prefill (process-wide);
+    returns the previous limit.  0 makes every wait give up at once."""
+    return int(lib().gdn_set_wait_budget(int(polls)))
+
+
+def gdn_set_prefill_segment_tokens(tokens: int) -> None:
+    """Prefill schedule override: 0 automatic, -1 one unit per sequence, or a segment
+    length in tokens (a multiple of 64)."""
+    _check(lib().gdn_set_prefill_segment_tokens(int(tokens)), "gdn_set_prefill_segment_tokens")
 
 
 def gdn_prefill_workspace_size(num_seqs: int, T_total: int, H_v: int, dk: int, dv: int) -> int:

@@ -3,6 +3,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "../../include/qsa.h"
 
@@ -18,12 +20,15 @@ cudaError_t launch_prefill_cc(const void *q, const void *k, const void *v, const
                               const int32_t *cu, int N, long long T, int H_qk, int H_v, int dk,
                               int dv, gdn_dtype dtype, float scale, int opts,
                               cudaStream_t stream);
-bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype);
-cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *v, const float *g,
-                                      const float *beta, const float *S0, void *out, float *S_final,
-                                      const int32_t *cu, int N, long long T_dense, long long T_total,
-                                      int H_qk, int H_v, float scale, int opts, DeviceError *err,
-                                      cudaStream_t stream);
+bool prefill_chain_supported(int dk, int dv, gdn_dtype dtype);
+size_t chain_workspace_bytes(int N, long long T_total, int H_v, int sms, int override_tokens);
+int device_sm_count();
+cudaError_t launch_prefill_chain(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *S0, void *out, float *S_final,
+                                 const int32_t *cu, int N, long long T_dense, long long T_total,
+                                 int H_qk, int H_v, float scale, int opts, void *workspace,
+                                 size_t workspace_bytes, uint32_t budget, int seg_override,
+                                 cudaStream_t stream);
 cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, float *S, void *out, const int32_t *n_commit,
                                 int N, int T, int H_qk, int H_v, int dk, int dv, gdn_dtype dtype,
@@ -51,6 +56,9 @@ cudaError_t static_scratch_ptr(void **out);
 namespace {
 
 constexpr size_t kWorkspaceBytes = 256;
+constexpr int kDefaultSms = 148;          // B200; used to size a workspace with no device current
+std::atomic<uint32_t> g_wait_budget{GDN_DEFAULT_WAIT_BUDGET};
+std::atomic<int32_t> g_segment_tokens{0};
 
 // per-call options for the kernels (common.cuh)
 int options_of(uint32_t flags)
@@ -86,8 +94,24 @@ gdn_status common_checks(const void *q, const void *k, const void *v, const floa
 GDN_API size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t T_total, int32_t H_v,
                                           int32_t dk, int32_t dv)
 {
-    (void)num_seqs; (void)T_total; (void)H_v; (void)dk; (void)dv;
-    return kWorkspaceBytes;
+    if (num_seqs <= 0 || T_total <= 0 || H_v <= 0 || !gdn::prefill_chain_supported(dk, dv, GDN_BF16))
+        return kWorkspaceBytes;
+    int sms = gdn::device_sm_count();
+    if (sms <= 0) sms = kDefaultSms;
+    const size_t n = gdn::chain_workspace_bytes(num_seqs, T_total, H_v, sms, g_segment_tokens.load());
+    return n > kWorkspaceBytes ? n : kWorkspaceBytes;
+}
+
+GDN_API gdn_status gdn_set_prefill_segment_tokens(int32_t tokens)
+{
+    if (tokens < -2 || (tokens > 0 && tokens % 64 != 0)) return GDN_ERR_INVALID_ARG;
+    g_segment_tokens.store(tokens);
+    return GDN_OK;
+}
+
+GDN_API uint32_t gdn_set_wait_budget(uint32_t polls)
+{
+    return g_wait_budget.exchange(polls);
 }
 
 GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, const float *g,
@@ -128,11 +152,11 @@ GDN_API gdn_status gdn_prefill(const void *q, const void *k, const void *v, cons
     }
     const int l2 = options_of(flags);
     cudaError_t e;
-    if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
-        e = gdn::launch_prefill_tc_cluster(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
-                                           cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v,
-                                           scale, l2,
-                                           reinterpret_cast<gdn::DeviceError *>(workspace), stream);
+    if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_chain_supported(dk, dv, dtype)) {
+        e = gdn::launch_prefill_chain(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                      cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v, scale, l2,
+                                      workspace, workspace_bytes, g_wait_budget.load(),
+                                      g_segment_tokens.load(), stream);
     } else {
         e = gdn::launch_prefill_cc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
                                    cu_seqlens ? 0 : (long long)T, H_qk, H_v, dk, dv, dtype, scale,
@@ -267,9 +291,8 @@ GDN_API gdn_status gdn_prefill_static_scratch(const void *q, const void *k, cons
     if (N > 0 && H_v > 65535) return GDN_ERR_UNSUPPORTED;
     if ((S0 && !aligned(S0, 16)) || (S_final && !aligned(S_final, 16))) return GDN_ERR_INVALID_ARG;
     const long long T_total = cu_seqlens ? (long long)T : (long long)B * T;
-    // the sizes must fit the library-held scratch
-    if (gdn_prefill_workspace_size(N, T_total, H_v, dk, dv) > gdn::static_scratch_capacity())
-        return GDN_ERR_UNSUPPORTED;
+    // this path needs only the workspace's error word, which must fit the library-held scratch
+    if (kWorkspaceBytes > gdn::static_scratch_capacity()) return GDN_ERR_UNSUPPORTED;
     if (N == 0 || T_total == 0) {
         if (S_final && N > 0) {
             const size_t bytes = (size_t)N * H_v * dk * dv * sizeof(float);
@@ -288,11 +311,11 @@ GDN_API gdn_status gdn_prefill_static_scratch(const void *q, const void *k, cons
         return GDN_ERR_CUDA;
     const int l2 = options_of(flags);
     cudaError_t e;
-    if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_tc_supported(dk, dv, dtype)) {
-        e = gdn::launch_prefill_tc_cluster(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
-                                           cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v,
-                                           scale, l2,
-                                           reinterpret_cast<gdn::DeviceError *>(scratch), stream);
+    if (!(flags & GDN_FLAG_FORCE_CUDA_CORE) && gdn::prefill_chain_supported(dk, dv, dtype)) {
+        // the static scratch holds the error word only: the one-pass schedule
+        e = gdn::launch_prefill_chain(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
+                                      cu_seqlens ? 0 : (long long)T, T_total, H_qk, H_v, scale, l2,
+                                      scratch, kWorkspaceBytes, g_wait_budget.load(), -1, stream);
     } else {
         e = gdn::launch_prefill_cc(q, k, v, g, beta, S0, out, S_final, cu_seqlens, N,
                                    cu_seqlens ? 0 : (long long)T, H_qk, H_v, dk, dv, dtype, scale,

@@ -39,7 +39,8 @@
 // copies and MMAs, and leaves through the final cluster barrier.
 #include <cuda.h>
 #include <cudaTypedefs.h>
-#include <stdlib.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -158,30 +159,6 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, int issued, bool cluste
 static __device__ __align__(1024) unsigned char g4_ring[(size_t)K4_POOL * K4_GCLUSTER];
 static __device__ int g4_pool[K4_POOL];
 
-// Profiling aid, compiled in only with -DGDN_PHASE_TIMERS: CTA (0, 0) records clock64()
-// at fixed points of its chain (per chunk) and of its preparations (per production).
-#ifdef GDN_PHASE_TIMERS
-__device__ unsigned long long g4_chain[64][32];
-__device__ unsigned long long g4_prep[16][16];
-__device__ unsigned long long g4_span[1024][2];      // per CTA: globaltimer at start and end
-#define SPAN(k) do { const unsigned idx_ = blockIdx.y * gridDim.x + blockIdx.x; if (threadIdx.x == 0 && idx_ < 1024) { \
-    unsigned long long gt_; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt_)); g4_span[idx_][(k)] = gt_; } } while (0)
-#define CMARK(c, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (c) < 64) g4_chain[(c)][(k)] = clock64(); } while (0)
-#define PMARK(kk, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (kk) < 16) g4_prep[(kk)][(k)] = clock64(); } while (0)
-#define GMARK(c, k) do { if (blockIdx.x == 0 && blockIdx.y == 0 && (c) < 64) { unsigned long long gt_; \
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(gt_)); g4_chain[(c)][(k)] = gt_; } } while (0)
-extern "C" __attribute__((visibility("default"))) int gdn_debug_cluster_timeline(void *chain, void *prep, void *span)
-{
-    if (cudaMemcpyFromSymbol(chain, g4_chain, sizeof(g4_chain)) != cudaSuccess) return 1;
-    if (cudaMemcpyFromSymbol(span, g4_span, sizeof(g4_span)) != cudaSuccess) return 1;
-    return (int)cudaMemcpyFromSymbol(prep, g4_prep, sizeof(g4_prep));
-}
-#else
-#define CMARK(c, k) do { } while (0)
-#define PMARK(kk, k) do { } while (0)
-#define GMARK(c, k) do { } while (0)
-#define SPAN(k) do { } while (0)
-#endif
 
 // Cold path, kept out of line so its code is not repeated at every wait: the first role
 // of a CTA whose wait runs out records the error and raises the CTA's abort flag.
@@ -209,7 +186,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    SPAN(0);
     const uint32_t r = cluster_rank();
     const int n = blockIdx.x >> 2, h = blockIdx.y;
     const int hq = h / (H_v / H_qk);
@@ -344,7 +320,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 fail(12);
                 break;
             }
-            if (t == 0) CMARK(c, 9);
             tc_fence_after();
             {
                 uint32_t ws[32];
@@ -369,7 +344,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<1>();
-            if (t == 0) CMARK(c, 10);
 
             // ---- S_r += K~^T U_r on the chain (thread 0) and P U_r -> D_PU[s] beside it
             // (thread 32).  gamma_end of the next chunk is waited for before S2, so this
@@ -387,7 +361,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                             umma_bf16(tmem + T4_S, d_kt + ks * 128, d_ut + ks * 64, id_s2, 1);
                         umma_commit(bars + B_S2);
                         ++s2_req;
-                        CMARK(c, 22);
                     }
                 } else if (t == 32) {
                     oks = wait_bar(s ? B_OFREE1 : B_OFREE0, (c >> 1) & 1, false);
@@ -409,7 +382,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             // ---- state: S_r (bf16) for the next chunk's products first (that is what the
             // next W S_r waits for), then D_S <- gamma_end(c+1) S_r (needed only by the next S2)
             if (!group_all<1>(t != 0 || wait_bar(B_S2, c & 1, false))) { fail(14); break; }
-            if (t == 0) CMARK(c, 12);
             tc_fence_after();
             uint32_t rs[32];
             tmem_ld32(tmem + loff + T4_S, rs);
@@ -431,14 +403,13 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             group_sync<1>();
             bool okw = true;
-            if (t == 0) { CMARK(c, 13); okw = issue_ws(c + 1); }
+            if (t == 0) okw = issue_ws(c + 1);
 #pragma unroll
             for (int v = 0; v < 32; ++v) rs[v] = __float_as_uint(ge_next * __uint_as_float(rs[v]));
             tmem_st32(tmem + loff + T4_S, rs);
             tmem_wait_st();
             tc_fence_before();
             if (!group_all<1>(okw)) { fail(18); break; }
-            if (t == 0) CMARK(c, 15);
         }
         if (*abort_flag) {
             if (t == 0) {
@@ -524,7 +495,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             // ---- K~(c) = diag(decay to chunk end) K; rows past the end get weight 0
             if (!group_all<3>(t != 0 || wait_bar(B_CK, c & 1, false))) { fail(10); break; }
             if (c >= 1 && !group_all<3>(t != 0 || wait_bar(B_S2, (c - 1) & 1, false))) { fail(17); break; }
-            if (t == 0) CMARK(c, 7);
             if constexpr (L2N) { normalise_rows(sm + S4_CK); group_sync<3>(); }
 #pragma unroll 2
             for (int u = 0; u < 8; ++u) {
@@ -541,7 +511,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             group_sync<3>();
             if (t == 0) {
-                CMARK(c, 8);
                 mbar_arrive_local(bars + B_KT);
                 if (c + 1 < nch) {             // K of the next chunk into the free buffer
                     ++k_issued;
@@ -590,7 +559,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
             tc_fence_before();
             group_sync<3>();
-            if (t == 0) { mbar_arrive_local(bars + (s ? B_OFREE1 : B_OFREE0)); CMARK(c, 14); }
+            if (t == 0) mbar_arrive_local(bars + (s ? B_OFREE1 : B_OFREE0));
         }
         if (*abort_flag && t == 0) drain_bar(bars + B_CK, k_issued, false);
     } else if (warp < 8) {
@@ -618,10 +587,8 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (p >= nch) break;
             const long long t0 = t_begin + (long long)p * K4_C;
             const int L = (int)min((long long)K4_C, t_end - t0);
-            if (t == 0) PMARK(k, 0);
             if (t < K4_C) { pg[t] = nxt_g; pb[t] = nxt_b; }
             group_sync<2>();
-            if (t == 0) PMARK(k, 10);
             if (q == 0) {
                 const float a0 = pg[2 * l], a1 = pg[2 * l + 1];
                 float s = a0 + a1;
@@ -636,9 +603,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 pinv[2 * l] = expf(-G0); pinv[2 * l + 1] = expf(-G1);
             }
             // ---- inputs: rows past the end zeroed, optional q/k normalisation
-            if (t == 0) PMARK(k, 11);
             if (!group_all<2>(t != 0 || (wait_bar(B_PKQ, k & 1, false) && wait_bar(B_PV, k & 1, false)))) { fail(20); break; }
-            if (t == 0) PMARK(k, 1);
             if (L < K4_C) {
                 const int zr = K4_C - L;
                 for (int e = t; e < 6 * zr * 8; e += 128) {
@@ -679,9 +644,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             // ---- the previous production's staging (overlaying A, T and P) has been read by
             // its bulk stores
             if (k >= 1 && !group_all<2>(t != 0 || wait_bar(B_SFREE, (k - 1) & 1, false))) { fail(21); break; }
-            if (t == 0) PMARK(k, 2);
             if (!group_all<2>(t != 0 || wait_bar(B_P1, k & 1, false))) { fail(22); break; }
-            if (t == 0) PMARK(k, 3);
             tc_fence_after();
 
             // ---- A (fp32, rows 0..63) and P (bf16, rows 64..127) from [K;Q] K^T
@@ -751,12 +714,10 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             tc_fence_before();
             group_sync<2>();
 
-            if (t == 0) PMARK(k, 4);
             if (p + 4 < nch && t < K4_C) fetch_gb(p + 4);    // lands during the inverse
             // ---- T = (I + A)^-1
             invert_unit_lower_64_tf32_wg<TP4>(Af, Tf, t, [] { group_sync<2>(); });
             group_sync<2>();
-            if (t == 0) PMARK(k, 5);
 
             // ---- T' = T diag(beta gamma), T'' = T diag(beta) (bf16, K-major rows i)
             {
@@ -781,11 +742,10 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<2>();
-            if (t == 0) { mbar_arrive_local(bars + B_TT); PMARK(k, 6); }
+            if (t == 0) mbar_arrive_local(bars + B_TT);
 
             // ---- W and U~ (M = 64 layout) into the staging
             if (!group_all<2>(t != 0 || wait_bar(B_WU, k & 1, false))) { fail(23); break; }
-            if (t == 0) PMARK(k, 7);
             tc_fence_after();
             const int i = 16 * q + l;                        // valid for l < 16
 #pragma unroll 1
@@ -819,7 +779,7 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async();
             tc_fence_before();
             group_sync<2>();
-            if (t == 0) { mbar_arrive_local(bars + B_STG); PMARK(k, 8); }
+            if (t == 0) mbar_arrive_local(bars + B_STG);
         }
     } else if (warp == 8) {
         // ========================================================== chain issuer
@@ -856,7 +816,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (k < next_load && mbar_try_wait(bars + ((k & 1) ? B_FULL1 : B_FULL0), (uint32_t)((k >> 1) & 1))) {
                     // the loads this covers have completed, so there is nothing to publish
                     mbar_arrive_remote_relaxed(map_to_rank(bars + B_GFREE0 + ((k >> 2) & 1), (uint32_t)(k & 3)));
-                    CMARK(k, 2);
                     acked = k;
                 }
             };
@@ -883,8 +842,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll 1
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1;
-                CMARK(c, 0);
-                GMARK(c, 26);
                 // chunk c's prepared data has landed (and been acknowledged)
                 {
                     bool okf = true;
@@ -894,7 +851,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                     if (!okf) { fail(33); break; }
                 }
-                CMARK(c, 1);
                 // Q S_r -> D_QS[s] right behind W S_r in the pipe (both read the same S_r tile)
                 if (!wait_ring(B_WSI, c & 1)) { fail(35); break; }
                 if (!wait_ring(L2N ? B_CQN : B_CQ, c & 1)) { fail(30); break; }
@@ -905,7 +861,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     umma_bf16(tmem + T4_QS + 32 * s, d_cq + (ks >> 2) * 512 + (ks & 3) * 2, d_st + ks * 64, id_m64, ks > 0);
                 umma_commit(bars + B_QS);
                 ++qs_req;
-                CMARK(c, 19);
                 // Q of the next chunk into the buffer Q S_r has finished reading
                 if (!wait_ring(B_QS, c & 1)) { fail(34); break; }
                 if (c + 1 < nch) {
@@ -915,12 +870,10 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tma_load_3d(sm + S4_CQ, &tm_q, bars + B_CQ, 0, hq, tn);
                     tma_load_3d(sm + S4_CQ + 8192, &tm_q, bars + B_CQ, 64, hq, tn);
                 }
-                CMARK(c, 24);
                 // ring slot s is free for chunk c + 2 once P U_r (the last MMA reading it) is done
                 if (!wait_ring(s ? B_PU1 : B_PU0, (c >> 1) & 1)) { fail(38); break; }
                 load_limit = c + 2;
                 poll_ring();
-                CMARK(c, 5);
             }
             if (*abort_flag) {
                 // let this thread's loads land before shared memory goes away
@@ -1008,7 +961,6 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
                 bulk_store_global(gchunk + 24576, sm + S4_USTG, 16384);
                 bulk_commit();
                 pend = p;
-                PMARK(k, 9);
             }
             if (pend >= 0 && !*abort_flag) finish_stores();
             bulk_wait_all();
@@ -1031,21 +983,21 @@ prefill_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_q,
         __threadfence();
         atomicExch(&g4_pool[ring_slot], 0);
     }
-    SPAN(1);
 }
 
 // ------------------------------------------------------------------------ host side
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encoder4() {
+    static std::once_flag once;
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    std::call_once(once, [] {
         cudaDriverEntryPointQueryResult q;
         void *p = nullptr;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+    });
     return fn;
 }
 
@@ -1061,44 +1013,52 @@ bool make_map4(CUtensorMap *map, const void *base, long long T_total, int H) {
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-uint32_t wait_budget4() {
-    const char *env = getenv("GDN_TEST_WAIT_BUDGET");
-    return env ? (uint32_t)strtoul(env, nullptr, 10) : K4_DEFAULT_BUDGET;
+struct ClusterDeviceState {
+    bool ready = false;
+};
+constexpr int kMaxDev4 = 128;
+std::mutex g_dev4_mutex;
+ClusterDeviceState g_dev4[kMaxDev4];
+
+// the 226 KB shared-memory opt-in of both instantiations, once per device
+cudaError_t cluster_device_setup() {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev4) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_dev4_mutex);
+    if (!g_dev4[dev].ready) {
+        e = cudaFuncSetAttribute(prefill_tc_cluster_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, K4_SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_tc_cluster_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, K4_SMEM);
+        if (e != cudaSuccess) return e;
+        g_dev4[dev].ready = true;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
-
-bool prefill_tc_supported(int dk, int dv, gdn_dtype dtype)
-{
-    return dk == K4_D && dv == K4_D && dtype == GDN_BF16;
-}
 
 cudaError_t launch_prefill_tc_cluster(const void *q, const void *k, const void *v, const float *g,
                                       const float *beta, const float *S0, void *out, float *S_final,
                                       const int32_t *cu, int N, long long T_dense, long long T_total,
                                       int H_qk, int H_v, float scale, int opts, DeviceError *err,
-                                      cudaStream_t stream)
+                                      uint32_t budget, cudaStream_t stream)
 {
     if (T_total >= (1LL << 31) || (long long)N * 4 > 0x7fffffffLL) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
     if (!make_map4(&mq, q, T_total, H_qk) || !make_map4(&mk, k, T_total, H_qk) ||
         !make_map4(&mv, v, T_total, H_v))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_cluster_kernel<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, K4_SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(prefill_tc_cluster_kernel<true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, K4_SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    const cudaError_t se = cluster_device_setup();
+    if (se != cudaSuccess) return se;
     dim3 grid((unsigned)(4 * N), (unsigned)H_v);
     auto kern = (opts & kOptL2Norm) ? prefill_tc_cluster_kernel<true> : prefill_tc_cluster_kernel<false>;
     kern<<<grid, K4_THREADS, K4_SMEM, stream>>>(
         mq, mk, mv, g, beta, S0, (__nv_bfloat16 *)out, S_final, cu, T_dense, H_qk, H_v, scale,
-        opts, err, wait_budget4());
+        opts, err, budget);
     return cudaGetLastError();
 }
 

@@ -196,3 +196,126 @@ __device__ __forceinline__ void invert_unit_lower_64_tf32_wg(float *A, float *T,
 }
 
 }  // namespace gdn
+
+namespace gdn {
+
+// ---------------------------------------------------------------------------------
+// T = (I + A)^-1 for a 64 x 64 strictly lower triangular A, by one warpgroup (t = 0..127)
+// with every warp busy at each level and no cross-warp dependency inside a level:
+//   1. warp w inverts diagonal block w (16 x 16) in registers, one lane per column,
+//      right-looking: once x_m is final, A[r][m] x_m is added to every later row r, so
+//      the dependent path is 16 FMAs long;
+//   2. 16 -> 32: warp w forms columns [8 (w & 1), +8) of T_HL = -D_H (A_HL D_L) for the
+//      block pair p = w >> 1 (H = 2p + 1, L = 2p);
+//   3. 32 -> 64: warp w forms columns [8w, 8w + 8) of T_HL = -T_HH (A_HL T_LL) with the
+//      32 x 32 halves L = [0, 32), H = [32, 64).
+// Levels 2 and 3 run on the warp-level tensor cores (mma.sync m16n8k8, tf32 operands,
+// fp32 accumulate): T is rounded to bf16 afterwards, and tf32 keeps 10 mantissa bits.
+// The products A_HL D_L / A_HL T_LL pass through A's strict upper triangle, which the
+// caller no longer needs.  Layout: row-major, pitch TP floats (TP = 72 keeps the fragment
+// loads free of bank conflicts).  On entry T's two blocks T[0:16, 16:32] and
+// T[32:48, 48:64] must be zero (they are read as part of T_LL and T_HH and never
+// written); everything else of T is written here.  The caller synchronises the group
+// before (A written) and after (T read).
+template <int TP>
+__device__ __forceinline__ void mma_tile_16x8(const float *X, int ldx, const float *Y, int ldy,
+                                              int K, float (&acc)[4], int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll 4
+    for (int kk = 0; kk < K; kk += 8) {
+        uint32_t a[4], b[2];
+        a[0] = to_tf32(X[g * ldx + kk + t]);
+        a[1] = to_tf32(X[(g + 8) * ldx + kk + t]);
+        a[2] = to_tf32(X[g * ldx + kk + t + 4]);
+        a[3] = to_tf32(X[(g + 8) * ldx + kk + t + 4]);
+        b[0] = to_tf32(Y[(kk + t) * ldy + g]);
+        b[1] = to_tf32(Y[(kk + t + 4) * ldy + g]);
+        mma_16x8x8_tf32(acc, a, b);
+    }
+}
+__device__ __forceinline__ void store_tile_16x8(float *C, int ldc, const float (&acc)[4], float sign,
+                                                int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    C[g * ldc + 2 * t] = sign * acc[0];
+    C[g * ldc + 2 * t + 1] = sign * acc[1];
+    C[(g + 8) * ldc + 2 * t] = sign * acc[2];
+    C[(g + 8) * ldc + 2 * t + 1] = sign * acc[3];
+}
+
+// In place: M holds A on entry and T on exit (its lower triangle with the diagonal; the
+// strict upper triangle is scratch except two blocks, see below).  One warpgroup,
+// t = 0..127, synchronised by `sync()` (a named barrier over exactly those threads):
+//   1. warp w replaces diagonal block w (16 x 16) of A by its inverse D_w, computed in
+//      registers, one lane per column, right-looking (once x_m is final, A[r][m] x_m is
+//      added to every later row r, so the dependent path is 16 FMAs long);
+//   2. 16 -> 32: for the block pair p = w >> 1 (H = 2p + 1, L = 2p), warp w forms columns
+//      [8 (w & 1), +8) of X = A_HL D_L into scratch, and after a barrier replaces those
+//      columns of A_HL by T_HL = -D_H X;
+//   3. 32 -> 64: with the 32 x 32 halves L = [0, 32), H = [32, 64), warp w forms columns
+//      [8w, 8w + 8) of X = A_HL T_LL into scratch and, after a barrier, of T_HL = -T_HH X.
+// Levels 2 and 3 run on the warp-level tensor cores (mma.sync m16n8k8, tf32 operands,
+// fp32 accumulate): T is rounded to bf16 afterwards, and tf32 keeps 10 mantissa bits.
+// Scratch is the upper-right 32 x 32 block (rows 0..31, columns 32..63).  The blocks
+// M[0:16, 16:32] and M[32:48, 48:64] are read as the zero upper parts of T_LL and T_HH:
+// the caller must have zeroed them (they are never written here).  Row pitch TP floats
+// (TP = 72 keeps the fragment loads free of bank conflicts).
+template <int TP, typename Sync>
+__device__ __forceinline__ void invert_unit_lower_64_inplace_wg(float *M, int t, Sync sync)
+{
+    const int warp = t >> 5, lane = t & 31;
+    // 1. diagonal blocks
+    {
+        const int c = lane & 15;
+        float *Mb = M + (16 * warp) * TP + 16 * warp;
+        float acc[16], x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            x[m] = (m < c) ? 0.f : ((m == c) ? 1.f : -acc[m]);
+#pragma unroll
+            for (int r = m + 1; r < 16; ++r) acc[r] = fmaf(Mb[r * TP + m], x[m], acc[r]);
+        }
+        __syncwarp();                                  // every lane has read the block
+        if (lane < 16) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Mb[r * TP + c] = x[r];
+        }
+    }
+    sync();
+    // 2. 16 -> 32 merges
+    {
+        const int p = warp >> 1, nt = warp & 1;
+        const int lo = 32 * p, hi = lo + 16;
+        float *X = M + (16 * p) * TP + 32 + 16 * p + 8 * nt;   // scratch rows 16p.., columns 32 + 16p..
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_tile_16x8<TP>(M + hi * TP + lo, TP, M + lo * TP + lo + 8 * nt, TP, 16, acc, lane);
+        store_tile_16x8(X, TP, acc, 1.f, lane);
+        sync();                                        // A_HL read by both warps of the pair
+        float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_tile_16x8<TP>(M + hi * TP + hi, TP, X, TP, 16, acc2, lane);
+        store_tile_16x8(M + hi * TP + lo + 8 * nt, TP, acc2, -1.f, lane);
+    }
+    sync();
+    // 3. 32 -> 64 merge
+    {
+        const int nc = 8 * warp;
+        float *X = M + 32 + nc;                        // scratch rows 0..31, columns 32 + 8w..
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+            mma_tile_16x8<TP>(M + (32 + 16 * mt) * TP, TP, M + nc, TP, 32, acc[mt], lane);
+        sync();                                        // every warp has read A_HL and T_LL
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) store_tile_16x8(X + 16 * mt * TP, TP, acc[mt], 1.f, lane);
+        __syncwarp();
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile_16x8<TP>(M + (32 + 16 * mt) * TP + 32, TP, X, TP, 32, acc2, lane);
+            store_tile_16x8(M + (32 + 16 * mt) * TP + nc, TP, acc2, -1.f, lane);
+        }
+    }
+}
+
+}  // namespace gdn

@@ -26,12 +26,5 @@ def load():
     P = ctypes.c_void_p
     L.selftest_umma.argtypes = [P, P, P, ctypes.c_int, P]
     L.selftest_cluster.argtypes = [P]
-    L.selftest_umma_timing.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, ctypes.c_int]
-    L.selftest_umma_timing2.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
-    L.selftest_tma_timing.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                      ctypes.c_int, P]
-    L.selftest_contention.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
-    L.selftest_dsmem_bw.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
-    L.selftest_movement.argtypes = [P, ctypes.c_int, ctypes.c_int, P]
     L.selftest_tma.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
     return L

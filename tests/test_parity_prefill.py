@@ -109,6 +109,69 @@ def test_empty_input_copies_state():
     assert torch.equal(S, x["S0"])
 
 
+# ------------------------------------------------------ segmented (sequence-parallel)
+@pytest.fixture
+def segments():
+    """Force the sequence-parallel schedule with a given segment length for one test."""
+    def set_(tokens):
+        gdn.gdn_set_prefill_segment_tokens(tokens)
+    yield set_
+    gdn.gdn_set_prefill_segment_tokens(0)
+
+
+@pytest.mark.parametrize("seg", [64, 128, 192])
+def test_segmented_varlen_gva_ragged(segments, seg):
+    """Segments of `seg` tokens: the transfer pass, the scan and the output pass against
+    the oracle; lengths cut segments at, before and after chunk edges, and include
+    sequences shorter than one segment (a single unit) and empty ones."""
+    segments(seg)
+    lens = [1, 0, 64, 65, 129, 300, 2, 191, 640]
+    x = case(lens, 2, 4, 128, 128, torch.bfloat16, s0_std=0.05, seed=21 + seg)
+    o, S = run(x)
+    check(x, o, S, torch.bfloat16)
+
+
+@pytest.mark.parametrize("seg", [64, 256])
+def test_segmented_dense(segments, seg):
+    """Dense batch, segments per sequence from the batch shape (no unit table)."""
+    segments(seg)
+    x = case([1000, 1000, 1000], 1, 2, 128, 128, torch.bfloat16, s0_std=0.1, seed=31 + seg)
+    o, S = run(x, dense_B=3)
+    check(x, o, S, torch.bfloat16)
+
+
+def test_segmented_strong_decay_and_l2norm(segments):
+    segments(128)
+    x = case([700, 333], 2, 2, 128, 128, torch.bfloat16, s0_std=0.05, seed=41, g_mult=3.0,
+             normalize=False)
+    o, S = run(x, flags=gdn.GDN_FLAG_QK_L2NORM, scale=0.5)
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    check(x, o, S, torch.bfloat16, l2norm=True, scale=0.5)
+
+
+@pytest.mark.parametrize("lens", [[1, 0, 64, 65, 129, 300, 2, 191], [1000, 1000]])
+def test_cluster_kernel(segments, lens):
+    """The four-CTA cluster kernel (value columns split four ways, each chunk prepared by
+    one CTA of the cluster) on ragged varlen input with grouped heads and S0."""
+    segments(-2)
+    x = case(lens, 2, 4, 128, 128, torch.bfloat16, s0_std=0.05, seed=61 + len(lens))
+    o, S = run(x)
+    check(x, o, S, torch.bfloat16)
+
+
+def test_schedules_agree(segments):
+    """The one-unit and segmented schedules give the same results up to rounding."""
+    x = case([900, 450], 2, 2, 128, 128, torch.bfloat16, s0_std=0.05, seed=51)
+    segments(-1)
+    o1, S1 = run(x)
+    segments(192)
+    o2, S2 = run(x)
+    segments(-2)
+    o3, S3 = run(x)
+    assert err(o2, o1) < 1e-2 and err(S2, S1) < 1e-2
+    assert err(o3, o1) < 1e-2 and err(S3, S1) < 1e-2
+
+
 # ---------------------------------------------------------- full-size workloads
 def _full(idx):
     w = inputs.get(idx)

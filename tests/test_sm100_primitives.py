@@ -1,6 +1,6 @@
 """The sm_100a building blocks of the tensor-core prefill, each against a plain
 reference: one tcgen05 MMA per operand placement (K-major / MN-major, negated B,
-N and K of 64 or 128) against torch.matmul in fp32, and one TMA tile load against
+N and K of 64 or 128, A read from TMEM) against torch.matmul in fp32, and one TMA tile load against
 the global tensor it copies."""
 from __future__ import annotations
 
@@ -34,6 +34,10 @@ def L():
     32 | 64 | 128,       # M=64, N=32, K=64:  P U with U in 64-byte-swizzled rows i
     64 | 1 | 128,        # M=128, N=32, K=64: K~^T U, A MN-major, U in 64-byte rows
     64 | 16 | 128 | 4,   # M=128, N=32, K=128, negated 64-byte-swizzled B
+    256 | 16 | 8,        # A from TMEM, B K-major, N=128, K=128: S^T [Q~;W]^T
+    256 | 2 | 8,         # A from TMEM, B MN-major, N=128, K=64:  (U dte)^T K
+    256,                 # A from TMEM, B K-major, N=64, K=64:    U^T P^T
+    256 | 16,            # A from TMEM, B K-major, N=64, K=128
 ])
 def test_umma_placements(L, variant):
     torch.manual_seed(variant)
