@@ -3,22 +3,22 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Prints ONE JSON line.  A step is one gdn_prefill call over the mid-size prefill
-workload (B=2, T=4096, H=16, dk=dv=128, bf16 q/k/v, fp32 g/beta/state, S0=0);
-`value` is whole-job prefill tokens/s with inputs resident in HBM.  The same line
-carries the decode workload (256 sequences x 128 single-token steps, H=32,
-dk=dv=128, bf16 q/k/v, fp32 state ~ N(0, 0.02)) under "decode", the roofline of
-each kernel, the end-to-end figure through the C ABI with host buffers ("e2e"),
-and the CPU oracle timed on this host ("cpu_baseline").  "qsa_indexer" carries the QSA
-compressed indexer: one query per sequence against 8 caches of 262,144 blocks (1,048,576
-tokens each, budget 512 blocks), and the compression of those 8,388,608 keys.
+Prints ONE JSON line.  A step is one gdn_prefill call over the long-context prefill
+workload (B=1, T=262,144, H=16, dk=dv=128, bf16 q/k/v, fp32 g/beta/state, slow decay
+g = -0.1 softplus(N(0,1)), S0=0); `value` is whole-job prefill tokens/s with the inputs
+resident in HBM.  The same line carries, with short keys so that it stays compact:
+"roofline" of that call, "e2e" (the same call through the C ABI from pinned host memory,
+copies inside the timed region), "decode" (256 sequences x 128 single-token steps, H=32,
+fp32 state ~ N(0, 0.02)), "cpu_baseline" (the oracle on this host's cores, on a prefix of
+the workload), and "sections": the mid-size and varlen prefill workloads, multi-token
+decode, the backward pass and the QSA compressed indexer.
 
-Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
-the launching stream; a 256 MB buffer is written between prefill steps (outside
-the events) so no step starts with its inputs in the 126 MB L2.  The decode state
-(537 MB) is larger than L2.  With N > 1 (torchrun) every rank runs its own replica
-of the workload (the layer has no cross-GPU exchange), the job time is the max over
-ranks and `value` counts all ranks' tokens.
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the
+launching stream; a 256 MB buffer is written between prefill steps (outside the events)
+so no step starts with inputs in the 126 MB L2 (the long-context inputs are 4.3 GB in any
+case).  The decode state (537 MB) is larger than L2.  With N > 1 (torchrun) every rank
+runs its own replica of the workload (the layer has no cross-GPU exchange), the job time
+is the max over ranks and `value` counts all ranks' tokens.
 """
 from __future__ import annotations
 
@@ -40,7 +40,8 @@ sys.path.insert(0, ROOT)
 from linear_attention_token_b200 import inputs  # noqa: E402
 
 METRIC = "GDN prefill tokens/s and decode tokens/s on 1 B200; % of tensor/HBM roofline"
-PREFILL_W = 1
+PREFILL_W = 3          # headline: the long-context prefill
+MID_W, VARLEN_W = 1, 2
 DECODE_W = 4
 CHUNK = 64
 
@@ -180,15 +181,23 @@ def flush_l2(buf):
     buf.add_(1)
 
 
+def prefill_args(x, w):
+    """The gdn_prefill arguments for workload w: a dense [B, T] view, or varlen."""
+    if len(set(w.seq_lens)) == 1 and not w.s0_std:
+        B, T = len(w.seq_lens), w.seq_lens[0]
+        view = lambda t: t.view(B, T, *t.shape[1:])
+        return [view(x[n]) for n in ("q", "k", "v", "g", "beta")] + [None, None], B
+    return [x[n] for n in ("q", "k", "v", "g", "beta")] + [x["S0"], x["cu_seqlens"]], len(w.seq_lens)
+
+
 def time_prefill(gdn, x, w, steps, warmup, stream, flush):
-    B, T = len(w.seq_lens), w.seq_lens[0]
-    view = lambda t: t.view(B, T, *t.shape[1:])
-    args = [view(x[n]) for n in ("q", "k", "v", "g", "beta")]
+    args, N = prefill_args(x, w)
     out = torch.empty_like(args[2])
-    S_final = torch.empty(B, w.H_v, w.dk, w.dv, dtype=torch.float32, device=out.device)
-    ws = gdn.prefill_workspace(B, w.tokens, w.H_v, w.dk, w.dv, out.device)
-    call = lambda: gdn.gdn_prefill(*args, None, None, out=out, S_final=S_final, workspace=ws,
-                                   stream=stream)
+    S_final = torch.empty(N, w.H_v, w.dk, w.dv, dtype=torch.float32, device=out.device)
+    ws = gdn.prefill_workspace(N, w.tokens, w.H_v, w.dk, w.dv, out.device)
+    sched = gdn.gdn_prefill_schedule(N, w.tokens, w.H_v, w.dk, w.dv, w.dtype,
+                                     varlen=args[6] is not None, workspace_bytes=ws.numel())
+    call = lambda: gdn.gdn_prefill(*args, out=out, S_final=S_final, workspace=ws, stream=stream)
     with torch.cuda.stream(stream):
         for _ in range(warmup):
             flush_l2(flush)
@@ -205,18 +214,20 @@ def time_prefill(gdn, x, w, steps, warmup, stream, flush):
     stream.synchronize()
     times = [a.elapsed_time(b) for a, b in evs]
     status = gdn.gdn_get_device_error(ws, stream)
-    return times, status
+    del ws, out, S_final
+    return times, status, sched
 
 
 def time_prefill_e2e(gdn, w, steps, warmup, stream, device):
     """Through the public API with HOST buffers: every step copies its inputs in from pinned
     host memory, runs the prefill and copies its result (outputs and final state) back.
-    Consecutive steps alternate between two streams and two buffer sets, so one step's
-    copy out overlaps the next step's copy in (separate copy engines) and compute; the
-    events bracket all `steps` steps."""
+    Consecutive steps alternate between two streams and two device buffer sets, so one
+    step's copy out overlaps the next step's copy in (separate copy engines) and compute;
+    the events bracket all `steps` steps."""
     B, T = len(w.seq_lens), w.seq_lens[0]
     xh = inputs.prefill_inputs(w, device="cpu")
     host = {n: xh[n].view(B, T, *xh[n].shape[1:]).pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    del xh
     streams = [stream, torch.cuda.Stream(device)]
     sets = []
     for _ in range(2):
@@ -255,6 +266,8 @@ def time_prefill_e2e(gdn, w, steps, warmup, stream, device):
     end.record(streams[0])
     torch.cuda.synchronize(device)
     per_step = start.elapsed_time(end) / steps
+    del sets, host
+    torch.cuda.empty_cache()
     return [per_step], h2d, d2h
 
 
@@ -313,7 +326,7 @@ def time_decode_multi(gdn, w, T, passes, warmup, stream, device):
 
 
 def time_backward(gdn, x, w, steps, warmup, stream):
-    """gdn_backward on the prefill workload (d_out random, no dS_final), device-timed."""
+    """gdn_backward on the mid-size prefill workload (d_out random, no dS_final), device-timed."""
     B, T = len(w.seq_lens), w.seq_lens[0]
     view = lambda t: t.view(B, T, *t.shape[1:])
     gen = torch.Generator(device="cpu").manual_seed(inputs.BASE_SEED + 99)
@@ -411,7 +424,10 @@ def cpu_baseline_qsa(wq, seqs=2):
 
 
 def cpu_baseline_prefill(w, max_tokens=None):
-    """The oracle (float variant, all host cores) on the prefill workload, timed."""
+    """The oracle (float variant, all host cores) on the prefill workload, timed; with
+    max_tokens, on the first max_tokens // N tokens of every sequence (the sequential
+    recurrence costs the same per token anywhere in a sequence, so tokens/s from a prefix
+    is the whole workload's rate)."""
     import oracle
     x = inputs.prefill_inputs(w, device="cpu")
     cu = x["cu_seqlens"]
@@ -431,8 +447,8 @@ def cpu_baseline_prefill(w, max_tokens=None):
     ntok = int(cu[-1])
     return {"value": ntok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "seconds": dt,
-            "sample": f"{ntok} tokens x {w.H_v} heads of {w.name} (sequential fp32 recurrence, "
-                      f"{threads} threads over (sequence, head))"}
+            "sample": f"first {ntok} of {w.tokens} tokens x {w.H_v} heads of {w.name} "
+                      f"(sequential fp32 recurrence, {threads} threads over (sequence, head))"}
 
 
 def cpu_baseline_decode(w, steps=2):
@@ -592,6 +608,29 @@ def run_qsa_only(args):
         print(json.dumps(line), flush=True)
 
 
+def prefill_roofline(w, ms, peaks, sched, traffic=None):
+    """Roofline of one prefill call: the method's FLOPs (chunked contractions at tile
+    shape) and algorithmic bytes over the call's device time."""
+    flops = prefill_flops_per_token_head(w.dk, w.dv) * w.tokens * w.H_v
+    tf = flops / (ms * 1e-3) / 1e12
+    byt = prefill_bytes(w)
+    return {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tf / peaks["bf16_tflops"], "traffic": traffic,
+            "peak_src": f"{peaks['source']} bf16 burst", "flops": flops, "bytes": byt,
+            "hbm_frac": byt / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "kernel": sched["kernel"], "launches": sched["launches"]}
+
+
+def short_section(name, value, unit, ms, roof=None, **kw):
+    d = {"w": name, "value": value, "unit": unit, "ms": ms}
+    if roof is not None:
+        d["frac"] = roof["frac"]
+        d["achieved"] = roof["achieved"]
+        d["bound"] = roof["bound"]
+    d.update(kw)
+    return d
+
+
 def run_ours(args):
     if args.section == "qsa":
         return run_qsa_only(args)
@@ -601,53 +640,76 @@ def run_ours(args):
     import linear_attention_token_b200 as gdn
     gdn.lib()                                   # loud failure if libgdn.so is missing
     peaks = load_peaks()
-    wp, wd = inputs.get(PREFILL_W), inputs.get(DECODE_W)
+    wp, wm, wv, wd = (inputs.get(i) for i in (PREFILL_W, MID_W, VARLEN_W, DECODE_W))
     stream = torch.cuda.Stream(device)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-    x = inputs.prefill_inputs(wp, device=device)
+    warm = max(args.warmup, 3)
+    launches = 0
 
     barrier(world)
     with ClockSampler(local) as clk:
-        times, status = time_prefill(gdn, x, wp, args.steps, max(args.warmup, 3), stream, flush)
+        x = inputs.prefill_inputs(wp, device=device)
+        times, status, sched = time_prefill(gdn, x, wp, args.steps, warm, stream, flush)
+        launches += args.steps * sched["launches"]
+        del x
+        torch.cuda.empty_cache()
         barrier(world)
         dec_passes = max(1, min(args.steps, 5))
         dtimes = time_decode(gdn, wd, dec_passes, max(1, min(args.warmup, 3)), stream, device)
+        launches += dec_passes * wd.decode_steps
+        barrier(world)
+        sec_steps = max(3, min(args.steps, 10))
+        xm = inputs.prefill_inputs(wm, device=device)
+        mtimes_p, st_m, sched_m = time_prefill(gdn, xm, wm, sec_steps, warm, stream, flush)
+        launches += sec_steps * sched_m["launches"]
+        bw_steps = max(1, min(args.steps, 3))
+        btimes = time_backward(gdn, xm, wm, bw_steps, 1, stream)
+        launches += bw_steps
+        del xm
+        barrier(world)
+        xv = inputs.prefill_inputs(wv, device=device)
+        vtimes_p, st_v, sched_v = time_prefill(gdn, xv, wv, sec_steps, warm, stream, flush)
+        launches += sec_steps * sched_v["launches"]
+        del xv
+        torch.cuda.empty_cache()
         barrier(world)
         vtimes, v_calls = time_decode_multi(gdn, wd, VERIFY_T, dec_passes, max(1, min(args.warmup, 3)),
                                             stream, device)
-        barrier(world)
-        bw_steps = max(1, min(args.steps, 3))
-        btimes = time_backward(gdn, x, wp, bw_steps, 1, stream)
+        launches += dec_passes * v_calls
         barrier(world)
         wq = qsa_workload(args)
         q_steps = max(3, min(args.steps, 20))
         qtimes, ctimes, q_blocks, q_tokens, mtimes = time_qsa(gdn, wq, q_steps, 3, stream, device)
+        launches += 3 * len(qtimes) + 3 * len(mtimes) + len(ctimes)
         barrier(world)
     clocks = clk.summary()
-    if status != 0:
-        raise RuntimeError(f"device error after prefill: {gdn.gdn_status_string(status)}")
+    for st in (status, st_m, st_v):
+        if st != 0:
+            raise RuntimeError(f"device error after prefill: {gdn.gdn_status_string(st)}")
 
     ms_prefill = max_over_ranks(sum(times) / len(times), world)
     ms_decode_pass = max_over_ranks(sum(dtimes) / len(dtimes), world)
-    e2e_steps = max(4, args.steps)
-    e2e_times, h2d, d2h = time_prefill_e2e(gdn, wp, e2e_steps, 2, stream, device)
+    e2e_steps = max(2, min(args.steps, 4))
+    e2e_times, h2d, d2h = time_prefill_e2e(gdn, wp, e2e_steps, 1, stream, device)
+    launches += e2e_steps * sched["launches"]
     ms_e2e = max_over_ranks(sum(e2e_times) / len(e2e_times), world)
 
     tok = wp.tokens
-    flops = prefill_flops_per_token_head(wp.dk, wp.dv) * tok * wp.H_v
-    pf_tflops = flops / (ms_prefill * 1e-3) / 1e12
-    pf_bytes = prefill_bytes(wp)
-    tc_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "prefill_tc_cluster.cu")
-    dec_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode.cu")
+    pf_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "prefill_chain.cu")
+    roof = prefill_roofline(wp, ms_prefill, peaks, sched, profiled_traffic("prefill_long", pf_src))
     ms_dec_step = ms_decode_pass / wd.decode_steps
     dec_bytes = decode_bytes_per_step(wd)
+    dec_gbs = dec_bytes / (ms_dec_step * 1e-3) / 1e9
+    dec_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode.cu")
+    ms_m = max_over_ranks(sum(mtimes_p) / len(mtimes_p), world)
+    ms_v = max_over_ranks(sum(vtimes_p) / len(vtimes_p), world)
     ms_verify_pass = max_over_ranks(sum(vtimes) / len(vtimes), world)
     ms_bw = max_over_ranks(sum(btimes) / len(btimes), world)
     ver_bytes = decode_multi_bytes_per_call(wd, VERIFY_T)
     ver_gbs = ver_bytes / (ms_verify_pass / v_calls * 1e-3) / 1e9
-    ver_src = os.path.join(ROOT, "linear_attention_token_b200", "csrc", "decode_multi.cu")
-    dec_gbs = dec_bytes / (ms_dec_step * 1e-3) / 1e9
     qsa = qsa_section(gdn, peaks, wq, qtimes, ctimes, q_blocks, q_tokens, world, mtimes)
+    rm = prefill_roofline(wm, ms_m, peaks, sched_m)
+    rv = prefill_roofline(wv, ms_v, peaks, sched_v)
 
     line = {
         "metric": METRIC,
@@ -655,63 +717,52 @@ def run_ours(args):
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
-        "warmup": max(args.warmup, 3),
+        "warmup": warm,
         "ms_per_step": ms_prefill,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded; q,k ~ N(0,1) L2-normalised, v ~ N(0,1), g = -softplus(N(0,1)), "
+        "data": "synthetic (seeded; q,k ~ N(0,1) L2-normalised, v ~ N(0,1), g = -0.1 softplus(N(0,1)), "
                 "beta = sigmoid(N(0,1)))",
-        "config": prefill_config(wp, world),
-        "roofline": {"bound": "tensor", "achieved": pf_tflops,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": pf_tflops / peaks["bf16_tflops"],
-                     "traffic": profiled_traffic("prefill", tc_src),
-                     "peak_source": f"{peaks['source']} bf16 burst",
-                     "flops_per_launch": flops, "algorithmic_bytes_per_launch": pf_bytes,
-                     "hbm_frac": pf_bytes / (ms_prefill * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "config": prefill_config(wp, world, sched),
+        "roofline": roof,
+        "e2e": {"value": world * tok / (ms_e2e * 1e-3), "unit": "tokens/s", "ms": ms_e2e,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "decode": {
-            "workload": wd.name, "value": world * wd.decode_seqs / (ms_dec_step * 1e-3),
+            "w": wd.name, "value": world * wd.decode_seqs / (ms_dec_step * 1e-3),
             "unit": "tokens/s", "ms_per_step": ms_dec_step, "passes": dec_passes,
             "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
-                         "traffic": profiled_traffic("decode", dec_src),
-                         "peak_source": f"{peaks['source']} copy bandwidth",
-                         "algorithmic_bytes_per_launch": dec_bytes},
-        },
-        "decode_multi": {
-            "workload": f"{wd.name} as {VERIFY_T}-token calls", "tokens_per_call": VERIFY_T,
-            "value": world * wd.decode_seqs * wd.decode_steps / (ms_verify_pass * 1e-3),
-            "unit": "tokens/s", "ms_per_call": ms_verify_pass / v_calls, "passes": dec_passes,
-            "roofline": {"bound": "hbm", "achieved": ver_gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": ver_gbs / peaks["hbm_gbs"],
-                         "traffic": profiled_traffic("decode_multi", ver_src),
-                         "peak_source": f"{peaks['source']} copy bandwidth",
-                         "algorithmic_bytes_per_launch": ver_bytes},
-        },
-        "backward": {
-            "workload": wp.name, "value": world * tok / (ms_bw * 1e-3), "unit": "tokens/s",
-            "ms_per_step": ms_bw, "steps": bw_steps,
-            "kernel": "backward_kernel: exact sequential reverse pass, checkpoint every 64 "
-                      "tokens, CUDA cores; bound by the per-head token chain",
-        },
-        "qsa_indexer": qsa,
-        "e2e": {"value": world * tok / (ms_e2e * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": "gdn_prefill via the C ABI; every step's pinned host inputs copied in and "
-                        "outputs + final state copied out inside the timed region; consecutive "
-                        "steps alternate two streams so copies overlap"},
-        # our kernels inside timed regions: prefill steps, decode passes, multi-token calls,
-        # backward steps, the end-to-end prefill steps, and the QSA calls (3 kernels each)
-        "gpu_launches": (args.steps + dec_passes * wd.decode_steps + dec_passes * v_calls + bw_steps
-                         + e2e_steps + 3 * len(qtimes) + 3 * len(mtimes) + len(ctimes)),
+                         "traffic": profiled_traffic("decode", dec_src), "bytes": dec_bytes}},
+        "gpu_launches": launches,
         "clocks": clocks,
+        "sections": {
+            "mid": short_section(wm.name, world * wm.tokens / (ms_m * 1e-3), "tokens/s", ms_m, rm,
+                                 kernel=sched_m["kernel"], seg=sched_m["segment_tokens"]),
+            "varlen": short_section(wv.name, world * wv.tokens / (ms_v * 1e-3), "tokens/s", ms_v, rv,
+                                    kernel=sched_v["kernel"], seg=sched_v["segment_tokens"]),
+            "dec_multi": short_section(f"{wd.name} as {VERIFY_T}-token calls",
+                                       world * wd.decode_seqs * wd.decode_steps / (ms_verify_pass * 1e-3),
+                                       "tokens/s", ms_verify_pass / v_calls,
+                                       {"frac": ver_gbs / peaks["hbm_gbs"], "achieved": ver_gbs, "bound": "hbm"}),
+            "backward": short_section(wm.name, world * wm.tokens / (ms_bw * 1e-3), "tokens/s", ms_bw),
+            "qsa": short_section(qsa["workload"], qsa["value"], "queries/s", qsa["ms_per_call"],
+                                 qsa["roofline"],
+                                 multi={"value": qsa["multi_query"]["value"],
+                                        "ms": qsa["multi_query"]["ms_per_call"],
+                                        "frac": qsa["multi_query"]["roofline"]["frac"]},
+                                 compress={"value": qsa["compress"]["value"],
+                                           "ms": qsa["compress"]["ms_per_call"],
+                                           "frac": qsa["compress"]["roofline"]["frac"]}),
+        },
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_prefill(wp)
-        line["decode"]["cpu_baseline"] = cpu_baseline_decode(wd)
-        line["qsa_indexer"]["cpu_baseline"] = cpu_baseline_qsa(wq)
+        cb = cpu_baseline_prefill(wp, max_tokens=CPU_PREFIX)
+        cb.pop("seconds", None)
+        line["cpu_baseline"] = cb
+        db = cpu_baseline_decode(wd)
+        line["decode"]["cpu_baseline"] = {"value": db["value"], "unit": db["unit"], "cores": db["cores"]}
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -719,26 +770,37 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def prefill_config(wp, world):
-    return {"workload": wp.name, "B": len(wp.seq_lens), "T": wp.seq_lens[0],
-            "H_qk": wp.H_qk, "H_v": wp.H_v, "dk": wp.dk, "dv": wp.dv, "chunk": CHUNK,
-            "state": "fp32", "parallelism": f"replicas x{world}" if world > 1 else "single",
-            "l2": "256 MB buffer written between timed prefill steps (outside the events)"}
+CPU_PREFIX = 65536     # tokens of the long-context workload the oracle baseline runs
+
+
+def prefill_config(wp, world, sched=None):
+    d = {"workload": wp.name, "B": len(wp.seq_lens), "T": wp.seq_lens[0], "H_qk": wp.H_qk,
+         "H_v": wp.H_v, "dk": wp.dk, "dv": wp.dv, "chunk": CHUNK, "state": "fp32",
+         "parallelism": f"replicas x{world}" if world > 1 else "single",
+         "l2": "inputs 4.3 GB > L2; a 256 MB buffer is also written between steps"}
+    if sched is not None:
+        d["schedule"] = f"{sched['kernel']}, segments of {sched['segment_tokens']} tokens" \
+            if sched["segment_tokens"] else sched["kernel"]
+    return d
 
 
 def run_reference(args):
-    """The oracle as it stands, on the host cores, on our arm's workload and metric."""
+    """The oracle as it stands, on the host cores, on our arm's workload and metric: every
+    step runs the sequential recurrence over a prefix of the long-context workload."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     wp = inputs.get(PREFILL_W)
+    prefix = 16384
     for _ in range(args.warmup):
-        cpu_baseline_prefill(wp, max_tokens=512)
-    runs = [cpu_baseline_prefill(wp) for _ in range(args.steps)]
+        cpu_baseline_prefill(wp, max_tokens=1024)
+    runs = [cpu_baseline_prefill(wp, max_tokens=prefix) for _ in range(args.steps)]
     secs = [r["seconds"] for r in runs]
+    ntok = min(prefix, wp.tokens)
     ms = 1e3 * sum(secs) / len(secs)
-    v = wp.tokens / (ms * 1e-3)
+    v = ntok / (ms * 1e-3)
     base = dict(runs[0])
+    base.pop("seconds", None)
     base["value"] = v
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,

@@ -217,6 +217,19 @@ gdn_status gdn_prefill_static_scratch(const void *q, const void *k, const void *
  * values. */
 gdn_status gdn_set_prefill_segment_tokens(int32_t tokens);
 
+/* The schedule gdn_prefill would use for these sizes on the current device (with the
+ * override above and a workspace of workspace_bytes): *kernel is one of GDN_PREFILL_*,
+ * *segment_tokens the segment length (0: one unit per sequence), *launches the number of
+ * kernels one call enqueues.  varlen: nonzero when cu_seqlens is given.  Enqueues nothing. */
+#define GDN_PREFILL_NONE 0          /* no tokens: only S_final is written */
+#define GDN_PREFILL_CUDA_CORE 1     /* fp32 or head dims of 64 */
+#define GDN_PREFILL_CHAIN 2         /* single-CTA tensor-core kernel */
+#define GDN_PREFILL_CLUSTER 3       /* four-CTA cluster tensor-core kernel */
+gdn_status gdn_prefill_schedule(int32_t num_seqs, int64_t T_total, int32_t H_v, int32_t dk,
+                                int32_t dv, gdn_dtype dtype, int32_t varlen,
+                                size_t workspace_bytes, uint32_t flags, int32_t *kernel,
+                                int32_t *segment_tokens, int32_t *launches);
+
 /* Every device-side wait of the tensor-core prefill polls its barrier at most this many
  * times (each poll suspends the thread for at most 2 microseconds, less when the awaited
  * phase completes) before the kernel gives up and records GDN_ERR_TIMEOUT: with the

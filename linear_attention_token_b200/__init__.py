@@ -11,7 +11,7 @@ from ._binding import (GDN_BF16, GDN_ERR_CUDA, GDN_ERR_INVALID_ARG, GDN_ERR_TIME
                        gdn_decode_step,
                        gdn_get_device_error, gdn_prefill, gdn_prefill_static_scratch,
                        gdn_prefill_workspace_size, gdn_set_prefill_segment_tokens,
-                       gdn_set_wait_budget,
+                       gdn_set_wait_budget, gdn_prefill_schedule,
                        gdn_status_string, lib, prefill_workspace, gdn_qsa_compress,
                        gdn_qsa_index_decode, gdn_qsa_index_workspace_size, qsa_index_workspace,
                        gdn_qsa_index_multi, gdn_qsa_index_multi_workspace_size,
@@ -25,4 +25,5 @@ __all__ = [
     "gdn_qsa_compress", "gdn_qsa_index_decode", "gdn_qsa_index_workspace_size",
     "qsa_index_workspace", "gdn_qsa_index_multi", "gdn_qsa_index_multi_workspace_size",
     "qsa_index_multi_workspace", "gdn_set_prefill_segment_tokens", "gdn_set_wait_budget",
+    "gdn_prefill_schedule",
 ]

@@ -32,7 +32,7 @@ EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode_step",
             "gdn_decode_multi", "gdn_backward", "gdn_backward_workspace_size",
             "gdn_qsa_compress", "gdn_qsa_index_workspace_size", "gdn_qsa_index_decode",
             "gdn_qsa_index_multi_workspace_size", "gdn_qsa_index_multi",
-            "gdn_set_wait_budget", "gdn_set_prefill_segment_tokens")
+            "gdn_set_wait_budget", "gdn_set_prefill_segment_tokens", "gdn_prefill_schedule")
 
 _lib = None
 
@@ -82,6 +82,9 @@ def lib():
         L.gdn_qsa_index_multi_workspace_size.restype = SZ
         L.gdn_qsa_index_multi.argtypes = [P, P, P, P, I32, I64, I32, I32, F, P, P, P, P, SZ, P]
         L.gdn_qsa_index_multi.restype = ctypes.c_int
+        L.gdn_prefill_schedule.argtypes = [I32, I64, I32, I32, I32, ctypes.c_int, I32, SZ, U32,
+                                           P, P, P]
+        L.gdn_prefill_schedule.restype = ctypes.c_int
         L.gdn_set_wait_budget.argtypes = [U32]
         L.gdn_set_wait_budget.restype = U32
         L.gdn_set_prefill_segment_tokens.argtypes = [I32]
@@ -148,6 +151,23 @@ def gdn_set_prefill_segment_tokens(tokens: int) -> None:
     """Prefill schedule override: 0 automatic, -1 one unit per sequence, or a segment
     length in tokens (a multiple of 64)."""
     _check(lib().gdn_set_prefill_segment_tokens(int(tokens)), "gdn_set_prefill_segment_tokens")
+
+
+PREFILL_KERNELS = {0: "none", 1: "cuda_core", 2: "chain", 3: "cluster"}
+
+
+def gdn_prefill_schedule(num_seqs: int, T_total: int, H_v: int, dk: int, dv: int,
+                         dtype=torch.bfloat16, varlen: bool = False, workspace_bytes=None,
+                         flags: int = 0) -> dict:
+    """The schedule gdn_prefill would use: {"kernel", "segment_tokens", "launches"}."""
+    if workspace_bytes is None:
+        workspace_bytes = gdn_prefill_workspace_size(num_seqs, T_total, H_v, dk, dv)
+    kern, seg, n = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    _check(lib().gdn_prefill_schedule(num_seqs, T_total, H_v, dk, dv, code, int(varlen),
+                                      int(workspace_bytes), int(flags), ctypes.byref(kern),
+                                      ctypes.byref(seg), ctypes.byref(n)), "gdn_prefill_schedule")
+    return {"kernel": PREFILL_KERNELS[kern.value], "segment_tokens": seg.value, "launches": n.value}
 
 
 def gdn_prefill_workspace_size(num_seqs: int, T_total: int, H_v: int, dk: int, dv: int) -> int:

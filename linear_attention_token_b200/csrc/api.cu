@@ -23,6 +23,8 @@ cudaError_t launch_prefill_cc(const void *q, const void *k, const void *v, const
 bool prefill_chain_supported(int dk, int dv, gdn_dtype dtype);
 size_t chain_workspace_bytes(int N, long long T_total, int H_v, int sms, int override_tokens);
 int device_sm_count();
+void describe_prefill(int N, long long T_total, int H_v, int sms, int override_tokens,
+                      size_t workspace_bytes, bool varlen, int *kind, int *seg_tokens, int *launches);
 cudaError_t launch_prefill_chain(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const float *S0, void *out, float *S_final,
                                  const int32_t *cu, int N, long long T_dense, long long T_total,
@@ -100,6 +102,31 @@ GDN_API size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t T_total, int
     if (sms <= 0) sms = kDefaultSms;
     const size_t n = gdn::chain_workspace_bytes(num_seqs, T_total, H_v, sms, g_segment_tokens.load());
     return n > kWorkspaceBytes ? n : kWorkspaceBytes;
+}
+
+GDN_API gdn_status gdn_prefill_schedule(int32_t num_seqs, int64_t T_total, int32_t H_v,
+                                        int32_t dk, int32_t dv, gdn_dtype dtype, int32_t varlen,
+                                        size_t workspace_bytes, uint32_t flags, int32_t *kernel,
+                                        int32_t *segment_tokens, int32_t *launches)
+{
+    if (!kernel || !segment_tokens || !launches || num_seqs < 0 || T_total < 0 || H_v <= 0)
+        return GDN_ERR_INVALID_ARG;
+    *segment_tokens = 0;
+    if (num_seqs == 0 || T_total == 0) { *kernel = GDN_PREFILL_NONE; *launches = 0; return GDN_OK; }
+    if ((flags & GDN_FLAG_FORCE_CUDA_CORE) || !gdn::prefill_chain_supported(dk, dv, dtype)) {
+        *kernel = GDN_PREFILL_CUDA_CORE;
+        *launches = 1;
+        return GDN_OK;
+    }
+    int sms = gdn::device_sm_count();
+    if (sms <= 0) sms = kDefaultSms;
+    int kind = 0, seg = 0, n = 0;
+    gdn::describe_prefill(num_seqs, T_total, H_v, sms, g_segment_tokens.load(), workspace_bytes,
+                          varlen != 0, &kind, &seg, &n);
+    *kernel = kind == 1 ? GDN_PREFILL_CLUSTER : GDN_PREFILL_CHAIN;
+    *segment_tokens = seg;
+    *launches = n;
+    return GDN_OK;
 }
 
 GDN_API gdn_status gdn_set_prefill_segment_tokens(int32_t tokens)

@@ -983,6 +983,11 @@ PrefillPlan plan_prefill(int N, long long T_total, int H_v, int sms, int overrid
     return pl;
 }
 
+// What launch_prefill_chain will launch for these sizes: kind 0 = this kernel, 1 = the
+// cluster kernel; seg_tokens 0 = one unit per sequence; launches = kernels per call.
+void describe_prefill(int N, long long T_total, int H_v, int sms, int override_tokens,
+                      size_t workspace_bytes, bool varlen, int *kind, int *seg_tokens, int *launches);
+
 size_t chain_workspace_bytes(int N, long long T_total, int H_v, int sms, int override_tokens)
 {
     const PrefillPlan pl = plan_prefill(N, T_total, H_v, sms, override_tokens);
@@ -990,6 +995,17 @@ size_t chain_workspace_bytes(int N, long long T_total, int H_v, int sms, int ove
     if (seg == 0) return kHead;
     const long long U = N + T_total / seg;
     return kHead + (size_t)U * 16 + (size_t)N * 8 + 1024 + 3 * (size_t)U * H_v * kStateBytes;
+}
+
+void describe_prefill(int N, long long T_total, int H_v, int sms, int override_tokens,
+                      size_t workspace_bytes, bool varlen, int *kind, int *seg_tokens, int *launches)
+{
+    const PrefillPlan pl = plan_prefill(N, T_total, H_v, sms, override_tokens);
+    int seg = pl.kind == PrefillPlan::kChain ? pl.seg_tokens : 0;
+    if (seg && workspace_bytes < chain_workspace_bytes(N, T_total, H_v, sms, override_tokens)) seg = 0;
+    *kind = pl.kind == PrefillPlan::kCluster ? 1 : 0;
+    *seg_tokens = seg;
+    *launches = seg ? (varlen ? 4 : 3) : 1;       // plan (varlen), transfers, scan, outputs
 }
 
 bool prefill_chain_supported(int dk, int dv, gdn_dtype dtype)

@@ -87,3 +87,26 @@ def test_traffic_file_is_well_formed():
         assert int(nbytes) > 0
         n += 1
     assert n >= len(known) - 1          # every kernel but possibly the newest entry
+
+
+def test_long_context_workload_counts(bench):
+    """The headline workload: 262,144 tokens x 16 heads; 755.9 GFLOP and 4.33 GB."""
+    w = inputs.get(3)
+    flops = bench.prefill_flops_per_token_head(w.dk, w.dv) * w.tokens * w.H_v
+    assert abs(flops - 755.9e9) < 0.1e9
+    assert bench.prefill_bytes(w) == 262_144 * 8192 * 2 + 262_144 * 16 * 8 + 16 * 128 * 128 * 4
+
+
+def test_prefill_args_dense_and_varlen(bench):
+    # dense workloads run as a [B, T] batch; the varlen one passes cu_seqlens and S0
+    for idx, varlen in ((1, False), (3, False), (2, True)):
+        w = inputs.get(idx)
+        x = {n: None for n in ("q", "k", "v", "g", "beta", "S0")}
+        x["cu_seqlens"] = "offsets"
+        if not varlen:
+            B, T = len(w.seq_lens), w.seq_lens[0]
+            import torch
+            x = {n: torch.zeros(B * T, 1) for n in ("q", "k", "v", "g", "beta")}
+        args, N = bench.prefill_args(x, w)
+        assert N == len(w.seq_lens)
+        assert (args[6] is not None) == varlen
