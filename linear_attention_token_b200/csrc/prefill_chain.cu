@@ -23,12 +23,18 @@
 // a chunk's K, Q and V land in one of three regions as soon as the chain has finished
 // with the chunk three back.
 //
-// Segments.  S_end = M S_in + B is affine in the state entering a segment, so a long
-// sequence splits into segments run in three passes (see launch_prefill_chain):
-//   1. transfer pass: per segment, the chain from S_in = I with U~ = 0 gives M (grid
-//      slice z = 0) and from S_in = 0 gives B (slice 1); no outputs;
-//   2. scan: S_in of segment p + 1 = M_p S_in(p) + B_p, sequentially over segments;
-//   3. output pass: every segment from its true S_in, writing o and the final state.
+// Segments.  Within a segment everything is affine in the state S_in entering it: the
+// outputs are O = O_local + Psi S_in and the end state S_end = M S_in + B, where O_local
+// and B come from the chain started at S_in = 0, and Psi and M from the chain started at
+// S_in = I with U~ = 0 (its "outputs" are exactly Psi_c = (diag(gamma) Q_c - P_c W_c)
+// Phi_c, Phi_c the transfer from the segment start to chunk c).  So a long sequence runs
+// as (see launch_prefill_chain):
+//   1. one pass of chains: for every segment the local chain (grid slice z = 1; the first
+//      segment starts from S0 and is then exact) and, past the first segment, the
+//      transfer chain (slice 0), in parallel;
+//   2. scan: S_in(p + 1) = M_p S_in(p) + B_p over the segments, and S_final;
+//   3. correction: out += Psi S_in(p) for the tokens of every segment p >= 1, a streamed
+//      tensor-core product.
 //
 // Roles (448 threads):
 //   warps 0-3    chain group: E3 and E4; thread 0 issues C1 and C2, thread 32 issues C3
@@ -43,6 +49,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -57,7 +64,6 @@ namespace {
 constexpr int CC = 64;                   // chunk
 constexpr int DD = 128;                  // dk = dv
 constexpr int CH_THREADS = 448;
-constexpr int MODE_OUT = 0, MODE_XFER = 1;
 constexpr int NREG = 3;                  // chunks in flight (regions)
 constexpr uint32_t kDrainBudget = GDN_DEFAULT_WAIT_BUDGET;   // waits after an abort
 constexpr uint32_t kPollNs = 2000;      // longest hardware suspension of one poll
@@ -160,7 +166,8 @@ struct ChainParams {
     __nv_bfloat16 *out;
     const int32_t *cu_seqlens;  // null: dense [N, T_dense]
     const int4 *units;          // null: computed (see unit_of)
-    float *ws_M, *ws_B, *ws_S;  // segment transfers and segment start states
+    float *ws_M, *ws_B, *ws_S;  // per unit: transfer M, local end state B, start state S_in
+    __nv_bfloat16 *ws_Psi;      // transfer-chain outputs Psi, [T_total, H_v, dk]
     long long T_dense;
     int N, H_qk, H_v;
     int seg_tokens;             // 0: one unit per sequence; else tokens per segment
@@ -209,7 +216,7 @@ __device__ __noinline__ void chain_abort(volatile int *abort_flag, DeviceError *
     }
 }
 
-template <int MODE, bool L2N>
+template <bool L2N, bool SEG>
 __global__ void __launch_bounds__(CH_THREADS, 1)
 prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ ChainParams prm)
@@ -218,12 +225,15 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    constexpr bool OUT = MODE == MODE_OUT;
-    const bool xa = !OUT && blockIdx.z == 0;       // transfer M: S_in = I, U~ = 0, no V
+    // segmented: slice z = 0 runs the transfer chain (S_in = I, U~ = 0, no V; its outputs
+    // are Psi, its final state M), slice 1 the local chain (S_in = S0 for the first
+    // segment, else 0; final state B)
+    constexpr bool seg = SEG;
+    const bool xa = SEG && blockIdx.z == 0;
     const int h = blockIdx.y;
     Unit un;
     if (!unit_of(prm, blockIdx.x, un)) return;
-    if (!OUT && un.p + 1 >= un.P) return;          // the last segment's transfer is not used
+    if (xa && un.p == 0) return;                   // the first segment starts from S0: no transfer
     const int hq = h / (prm.H_v / prm.H_qk);
     const int nch = (int)((un.te - un.tb + CC - 1) / CC);
     const size_t st_n = ((size_t)un.n * prm.H_v + h) * DD * DD;          // [N, H_v] slot
@@ -265,7 +275,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // =============================================================== chain group
         const int t = tid, v = tid, q = warp;
         const uint32_t loff = (uint32_t)(32 * q) << 16;
-        const uint32_t id_c1 = idesc_bf16(128, OUT ? 128 : 64, false, false);
+        const uint32_t id_c1 = idesc_bf16(128, 128, false, false);
         const uint32_t id_c2 = idesc_bf16(128, 128, false, true);
         const uint32_t id_c3 = idesc_bf16(128, 64, false, false);
         const uint32_t su = smem_u32(sm + S_U);
@@ -273,11 +283,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         int mma_issued = 0;
 
         auto issue_c1 = [&](int c) {           // thread 0
-            const uint32_t base = smem_u32(region(c)) + (OUT ? SR_Q : SR_W);
+            const uint32_t base = smem_u32(region(c)) + SR_Q;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t bd = sdesc_kmajor(base + (ks >> 2) * SR_KB + (ks & 3) * 32);
-                umma_bf16_ta(tmem + TM_QW + (OUT ? 0 : 64), tmem + TM_SB + 8 * ks, bd, id_c1, ks > 0);
+                umma_bf16_ta(tmem + TM_QW, tmem + TM_SB + 8 * ks, bd, id_c1, ks > 0);
             }
             umma_commit(bars + B_C1);
             ++mma_issued;
@@ -285,9 +295,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
         // ---- initial state: S^T (fp32, scaled by gamma_end(0)) and its bf16 copy
         const float *src = nullptr;
-        if (OUT) src = un.p == 0 ? (prm.S0 ? prm.S0 + st_n : nullptr) : prm.ws_S + st_u;
-        float *dst = OUT ? (un.p + 1 == un.P ? (prm.S_final ? prm.S_final + st_n : nullptr) : nullptr)
-                         : (xa ? prm.ws_M : prm.ws_B) + st_u;
+        if (!xa && un.p == 0 && prm.S0) src = prm.S0 + st_n;
+        float *dst = seg ? (xa ? prm.ws_M : prm.ws_B) + st_u : (prm.S_final ? prm.S_final + st_n : nullptr);
         if (nch == 0) {
             // no token: the final state is the initial one
             if (dst)
@@ -368,7 +377,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 umma_commit(bars + B_C2);
                 umma_commit(bars + rbar(B_RF0, c));
                 ++mma_issued;
-            } else if (OUT && t == 32) {
+            } else if (t == 32) {
                 // ---- C3: O^T += U^T P^T, issued beside C2 (off the chain)
                 tc_fence_after();
                 const uint32_t pt = smem_u32(sm + S_P + (c % NREG) * 8192);
@@ -415,7 +424,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             group_sync<1>();
             bool okw = true;
             if (t == 0) {
-                okw = wait_bar(rbar(B_RDY0, c + 1), rpar(c + 1)) && (!OUT || wait_bar(B_OF, par(c)));
+                okw = wait_bar(rbar(B_RDY0, c + 1), rpar(c + 1)) && wait_bar(B_OF, par(c));
                 if (okw) { tc_fence_after(); issue_c1(c + 1); }
             }
             const float ge = vecbuf(c + 1)[V_GAM + 63];
@@ -451,7 +460,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 // q/k normalisation before P1 reads the tiles; thread t: row t & 63 of K
                 // (t < 64) or Q
                 if (!group_all<2>(t != 0 || wait_bar(rbar(B_LD0, c), rpar(c)))) { fail(10); break; }
-                if (OUT || t < 64) {
+                {
                     const int r = t & 63;
                     unsigned char *r0 = rg + (t >= 64 ? SR_Q : 0) + r * 128;
                     float ss = 0.f;
@@ -476,7 +485,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // ---- A (fp32, rows 0..63) and P (bf16, rows 64..127) from [K;Q] K^T.  The P
             // tile of this region was last read by C3(c - NREG).
             if (!group_all<2>(t != 0 || (wait_bar(rbar(B_VEC0, c), rpar(c)) && wait_bar(B_P1, par(c)) &&
-                                         (!OUT || c < NREG || wait_bar(rbar(B_PF0, c), rpar(c - NREG)))))) {
+                                         (c < NREG || wait_bar(rbar(B_PF0, c), rpar(c - NREG)))))) {
                 fail(11);
                 break;
             }
@@ -495,7 +504,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int jend = 32 * ((q & 1) + 1);      // columns from here on are masked for the warp
                 unsigned char *pt = sm + S_P + (c % NREG) * 8192;
                 const float *fsrc = vb + (factored ? V_INV : V_G);
-                if (is_a || OUT) {
+                {
 #pragma unroll 1
                     for (int jh = 0; jh < 64; jh += 32) {
                         if (is_a && jh >= jend) break;    // the inverse never reads A above the diagonal
@@ -612,7 +621,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int L = (int)min((long long)CC, un.te - t0);
             // lanes (v, v ^ 1) pair up: the even lane writes token 2m's two values, the odd
             // lane token 2m + 1's
-            __nv_bfloat16 *obase = prm.out + ((size_t)t0 * prm.H_v + h) * DD + (v & ~1);
+            __nv_bfloat16 *obase = (xa ? prm.ws_Psi : prm.out) + ((size_t)t0 * prm.H_v + h) * DD + (v & ~1);
             const size_t rstride = (size_t)prm.H_v * DD;
 #pragma unroll
             for (int m = 0; m < 32; ++m) {
@@ -657,7 +666,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             {
                 const int r = t & 63, kb = t >> 6;
                 scale_row128(rg + kb * SR_KB + r * 128, r, vb[V_DTE + r]);
-                if (OUT) scale_row128(rg + kb * SR_KB + SR_Q + r * 128, r, vb[V_GAM + r]);
+                scale_row128(rg + kb * SR_KB + SR_Q + r * 128, r, vb[V_GAM + r]);
             }
             fence_proxy_async();
             group_sync<3>();
@@ -665,9 +674,9 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 mbar_arrive_local(bars + B_WTF);
                 mbar_arrive_local(bars + rbar(B_RDY0, c));
             }
-            if (OUT && c >= 1 && !outputs(c - 1)) { fail(21); break; }
+            if (c >= 1 && !outputs(c - 1)) { fail(21); break; }
         }
-        if (OUT && nch > 0 && !*abort_flag && !outputs(nch - 1)) fail(22);
+        if (nch > 0 && !*abort_flag && !outputs(nch - 1)) fail(22);
     } else if (warp == 12) {
         // =============================================================== prep issuer
         if (lane == 0) {
@@ -748,13 +757,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 okc = c < NREG || wait_bar(rbar(B_RF0, c), rpar(c - NREG));
                 if (okc) {
                     uint64_t *bar = bars + rbar(B_LD0, c);
-                    mbar_arrive_expect_tx(bar, 16384 * (1 + (OUT ? 1 : 0) + (xa ? 0 : 1)));
+                    mbar_arrive_expect_tx(bar, 16384 * (xa ? 2 : 3));
                     tma_load_3d(rg, &tm_k, bar, 0, hq, tc);
                     tma_load_3d(rg + SR_KB, &tm_k, bar, 64, hq, tc);
-                    if (OUT) {
-                        tma_load_3d(rg + SR_Q, &tm_q, bar, 0, hq, tc);
-                        tma_load_3d(rg + SR_KB + SR_Q, &tm_q, bar, 64, hq, tc);
-                    }
+                    tma_load_3d(rg + SR_Q, &tm_q, bar, 0, hq, tc);
+                    tma_load_3d(rg + SR_KB + SR_Q, &tm_q, bar, 64, hq, tc);
                     if (!xa) {
                         tma_load_3d(rg + SR_W, &tm_v, bar, 0, h, tc);
                         tma_load_3d(rg + SR_KB + SR_W, &tm_v, bar, 64, h, tc);
@@ -801,11 +808,12 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (warp == 12) tmem_dealloc(tmem, 512);
 }
 
-// Segment start states: S_in(p + 1) = M_p S_in(p) + B_p for p = 0 .. P - 2, with
-// S_in(0) = S0 (or zero).  One CTA per (sequence, value head, 16 value columns); 256
-// threads, thread t owns row t / 2 and 8 columns.  Exact fp32 on the CUDA cores.
+// Segment start states and the final state: S_in(1) = B_0 (the first segment's chain
+// started from S0), S_in(p + 1) = M_p S_in(p) + B_p, and S_final = S_in(P).  One CTA
+// per (sequence, value head, 16 value columns); 256 threads, thread t owns row t / 2 and 8
+// columns.  Exact fp32 on the CUDA cores.
 __global__ void __launch_bounds__(256)
-segment_scan_kernel(const float *S0, const float *ws_M, const float *ws_B, float *ws_S,
+segment_scan_kernel(const float *ws_M, const float *ws_B, float *ws_S, float *S_final,
                     const int2 *seqs, int N, int H_v, int units_per_seq)
 {
     __shared__ float S[DD][16];
@@ -813,16 +821,20 @@ segment_scan_kernel(const float *S0, const float *ws_M, const float *ws_B, float
     int u0, P;
     if (seqs) { const int2 e = seqs[n]; u0 = e.x; P = e.y; }
     else { u0 = n * units_per_seq; P = units_per_seq; }
-    if (P <= 1) return;
+    if (P < 1) return;
     const int d = t >> 1, cs = 8 * (t & 1);
     for (int e = t; e < DD * 16; e += 256) {
         const int dd = e >> 4, cc = e & 15;
-        S[dd][cc] = S0 ? S0[(((size_t)n * H_v + h) * DD + dd) * DD + c0 + cc] : 0.f;
+        S[dd][cc] = ws_B[(((size_t)u0 * H_v + h) * DD + dd) * DD + c0 + cc];
     }
     __syncthreads();
 #pragma unroll 1
-    for (int p = 0; p + 1 < P; ++p) {
+    for (int p = 1; p < P; ++p) {
         const size_t su = ((size_t)(u0 + p) * H_v + h) * DD * DD;
+        // S_in(p) for the correction pass
+        float *dsts = ws_S + su + (size_t)d * DD + c0 + cs;
+        *reinterpret_cast<float4 *>(dsts) = make_float4(S[d][cs], S[d][cs + 1], S[d][cs + 2], S[d][cs + 3]);
+        *reinterpret_cast<float4 *>(dsts + 4) = make_float4(S[d][cs + 4], S[d][cs + 5], S[d][cs + 6], S[d][cs + 7]);
         const float *Mr = ws_M + su + (size_t)d * DD;
         float acc[8];
         const float4 b0 = *reinterpret_cast<const float4 *>(ws_B + su + (size_t)d * DD + c0 + cs);
@@ -839,13 +851,176 @@ segment_scan_kernel(const float *S0, const float *ws_M, const float *ws_B, float
                 for (int j = 0; j < 8; ++j) acc[j] = fmaf(mv[k], S[e + k][cs + j], acc[j]);
         }
         __syncthreads();
-        float *dsts = ws_S + ((size_t)(u0 + p + 1) * H_v + h) * DD * DD + (size_t)d * DD + c0 + cs;
 #pragma unroll
         for (int j = 0; j < 8; ++j) S[d][cs + j] = acc[j];
-        *reinterpret_cast<float4 *>(dsts) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4 *>(dsts + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         __syncthreads();
     }
+    if (S_final) {
+        float *dst = S_final + (((size_t)n * H_v + h) * DD + d) * DD + c0 + cs;
+        *reinterpret_cast<float4 *>(dst) = make_float4(S[d][cs], S[d][cs + 1], S[d][cs + 2], S[d][cs + 3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(S[d][cs + 4], S[d][cs + 5], S[d][cs + 6], S[d][cs + 7]);
+    }
+}
+
+// Output correction of a segmented call: the local chain of segment p >= 1 started from
+// zero, so its outputs miss Psi S_in(p), where Psi (the transfer chain's outputs) maps the
+// segment's start state to every token's output.  out[t] += Psi[t] S_in(p) for the
+// segment's tokens, on the tensor cores: (Psi S_in)^T = S_in^T Psi^T, A = S_in^T (bf16 in
+// TMEM, lane = value column), B = a 64-token tile of Psi (K-major rows, by TMA), D in TMEM.
+// One CTA per (unit, value head); 160 threads: warps 0-3 convert S_in and run the
+// epilogue (thread 0 issues the MMAs), warp 4 streams Psi through NBUF buffers.
+namespace {
+constexpr int CR_THREADS = 160, CR_NBUF = 4;
+constexpr uint32_t CR_TM_A = 0, CR_TM_D = 64;          // TMEM: S_in^T bf16, two 64-column D
+constexpr uint32_t CR_BAR = CR_NBUF * 16384;
+constexpr uint32_t CR_SMEM = CR_BAR + 16 * 8 + 16 + 1024;
+enum CrBar { CR_LD0 = 0, CR_FREE0 = CR_NBUF, CR_DONE0 = 2 * CR_NBUF, CR_DFREE0 = CR_DONE0 + 2,
+             CR_DRAIN = CR_DFREE0 + 2, CR_COUNT };
+static_assert(CR_COUNT <= 16, "correction barriers");
+}  // namespace
+
+__global__ void __launch_bounds__(CR_THREADS)
+segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi, const __grid_constant__ ChainParams prm)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y;
+    Unit un;
+    if (!unit_of(prm, blockIdx.x, un) || un.p == 0) return;
+    const int nch = (int)((un.te - un.tb + CC - 1) / CC);
+    if (nch == 0) return;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CR_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + CR_BAR + 16 * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + CR_BAR + 16 * 8 + 4);
+    if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+    if (tid == 0) {
+        for (int b = 0; b < CR_COUNT; ++b) mbar_init(bars + b, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t budget = prm.budget;
+    auto wait_bar = [&](int b, uint32_t parity) -> bool {
+        for (uint32_t i = 0; i < budget; ++i) {
+            if (mbar_try_wait_sleep(bars + b, parity, kPollNs)) return true;
+            if (*abort_flag) return false;
+        }
+        return false;
+    };
+    auto fail = [&](int where) { chain_abort(abort_flag, prm.err, where); };
+
+    if (warp < 4) {
+        const int t = tid, v = tid;
+        const uint32_t loff = (uint32_t)(32 * warp) << 16;
+        const bool odd = lane & 1;
+        const uint32_t id_c = idesc_bf16(128, 64, false, false);
+        int issued = 0;
+        // S_in^T (bf16 pairs, lane v, column d / 2)
+        const float *src = prm.ws_S + ((size_t)blockIdx.x * prm.H_v + h) * DD * DD;
+#pragma unroll 1
+        for (int db = 0; db < 4; ++db) {
+            uint32_t xb[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int d = 32 * db + 2 * j;
+                xb[j] = pack2(src[(size_t)d * DD + v], src[(size_t)(d + 1) * DD + v]);
+            }
+            tmem_st16(tmem + loff + CR_TM_A + 16 * db, xb);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        auto issue = [&](int c) -> bool {        // thread 0
+            const int b = c % CR_NBUF;
+            if (!wait_bar(CR_LD0 + b, par(c / CR_NBUF))) return false;
+            tc_fence_after();
+            const uint32_t base = smem_u32(sm + b * 16384);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma_bf16_ta(tmem + CR_TM_D + 64 * (c & 1), tmem + CR_TM_A + 8 * ks,
+                             sdesc_kmajor(base + (ks >> 2) * 8192 + (ks & 3) * 32), id_c, ks > 0);
+            umma_commit(bars + CR_DONE0 + (c & 1));
+            umma_commit(bars + CR_FREE0 + b);
+            ++issued;
+            return true;
+        };
+        bool ok = true;
+        if (t == 0) {
+            ok = issue(0) && (nch < 2 || issue(1));
+            if (!ok) fail(50);
+        }
+        const size_t rstride = (size_t)prm.H_v * DD;
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+            uint32_t ok2;
+            {
+                const bool w = t != 0 || (!*abort_flag && wait_bar(CR_DONE0 + (c & 1), par(c >> 1)));
+                asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+                             "selp.u32 %0, 1, 0, q;\n\t}" : "=r"(ok2) : "r"(w ? 1u : 0u) : "memory");
+            }
+            if (!ok2) { fail(51); break; }
+            tc_fence_after();
+            uint32_t x0[32], x1[32];
+            tmem_ld32(tmem + loff + CR_TM_D + 64 * (c & 1), x0);
+            tmem_ld32(tmem + loff + CR_TM_D + 64 * (c & 1) + 32, x1);
+            tmem_wait_ld();
+            tc_fence_before();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (t == 0 && c + 2 < nch && !issue(c + 2)) fail(52);
+            const long long t0 = un.tb + (long long)c * CC;
+            const int L = (int)min((long long)CC, un.te - t0);
+            __nv_bfloat16 *obase = prm.out + ((size_t)t0 * prm.H_v + h) * DD + (v & ~1);
+            // lanes (v, v ^ 1) pair up: the even lane updates token 2m's two values, the odd
+            // lane token 2m + 1's.  Every old value is loaded before any store, so the 32
+            // loads are in flight together.
+            uint32_t old[32];
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const int r = 2 * m + (odd ? 1 : 0);
+                old[m] = r < L ? __ldcs(reinterpret_cast<const unsigned int *>(obase + (size_t)r * rstride)) : 0u;
+            }
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const uint32_t *xx = m < 16 ? x0 : x1;
+                const int mm = 2 * (m & 15);
+                const float a0 = __uint_as_float(xx[mm]), a1 = __uint_as_float(xx[mm + 1]);
+                const float recv = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
+                const int r = 2 * m + (odd ? 1 : 0);
+                const float2 o = unpack2(old[m]);
+                const uint32_t val = odd ? pack2(o.x + recv, o.y + a1) : pack2(o.x + a0, o.y + recv);
+                if (r < L) __stcs(reinterpret_cast<unsigned int *>(obase + (size_t)r * rstride), val);
+            }
+        }
+        if (*abort_flag && t == 0 && issued > 0) {
+            umma_commit(bars + CR_DRAIN);
+            mbar_wait(bars + CR_DRAIN, 0, kDrainBudget);
+        }
+    } else if (lane == 0) {
+        // loader: Psi tiles of the unit's chunks
+        int ld = 0;
+        const int tbi = (int)un.tb;
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+            const int b = c % CR_NBUF;
+            if (c >= CR_NBUF && !wait_bar(CR_FREE0 + b, par((c - CR_NBUF) / CR_NBUF))) { fail(53); break; }
+            mbar_arrive_expect_tx(bars + CR_LD0 + b, 16384);
+            tma_load_3d(sm + b * 16384, &tm_psi, bars + CR_LD0 + b, 0, h, tbi + c * CC);
+            tma_load_3d(sm + b * 16384 + 8192, &tm_psi, bars + CR_LD0 + b, 64, h, tbi + c * CC);
+            ++ld;
+        }
+        if (*abort_flag)
+            for (int c = max(0, ld - CR_NBUF); c < ld; ++c)
+                mbar_wait(bars + CR_LD0 + c % CR_NBUF, par(c / CR_NBUF), kDrainBudget);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // Unit table of a segmented varlen call: sequence n is split into ceil(len / seg) units
@@ -925,10 +1100,11 @@ cudaError_t device_state(int *sms) {
     DeviceState &s = g_dev[dev];
     if (!s.ready) {
         e = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<MODE_OUT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<MODE_OUT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<MODE_XFER, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<MODE_XFER, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_chain_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CH_SMEM);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(segment_correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CR_SMEM);
         if (e != cudaSuccess) return e;
         s.ready = true;
     }
@@ -953,15 +1129,20 @@ struct PrefillPlan {
 // whose chain per value-column quarter is shorter but takes four SMs per head.
 constexpr double kChainStep = 8400.0, kClusterStep = 4700.0;
 constexpr double kFill = 3.0;           // chunk steps to fill a pipeline at a unit's start
+// The output correction streams Psi and updates out in place; measured, each of its CTAs
+// moves about kCorrectCtaBps and the whole pass about kCorrectBps at most.  kStepSeconds
+// converts its time into chunk steps.
+constexpr double kCorrectCtaBps = 12e9, kCorrectBps = 3e12, kStepSeconds = 4.3e-6;
 
 // Schedule for a call: the cluster kernel (one wave of four-CTA clusters per (sequence,
 // value head)), or this kernel with one unit per sequence, or this kernel with segments of
 // L chunks.  The model counts time on the critical path, assuming equal sequence lengths:
-// unsegmented, ceil(units / slots) waves of C chunks; segmented, the transfer pass runs
-// 2 (P - 1) N H_v units and the output pass P N H_v units, each in ceil(units / SMs)
-// waves of L chunks (a transfer unit at 0.9 of an output unit: no outputs, no Q), and the
-// scan between them about 4 steps.  override_tokens: 0 automatic, -1 one unit per
-// sequence, -2 the cluster kernel, > 0 that segment length.
+// unsegmented, ceil(units / slots) waves of C chunks; segmented, one pass of (2 P - 1)
+// N H_v units (a local and, past the first segment, a transfer chain per segment) in
+// ceil(units / SMs) waves of L chunks, the scan (about 4 steps) and the output correction
+// (reads Psi, reads and writes out: HBM-bound, kCorrectBytesPerStep bytes per chunk step).
+// override_tokens: 0 automatic, -1 one unit per sequence, -2 the cluster kernel, > 0 that
+// segment length.
 PrefillPlan plan_prefill(int N, long long T_total, int H_v, int sms, int override_tokens)
 {
     PrefillPlan pl{PrefillPlan::kChain, 0};
@@ -974,10 +1155,14 @@ PrefillPlan plan_prefill(int N, long long T_total, int H_v, int sms, int overrid
     double best = waves(units0, sms) * ((double)C + kFill) * kChainStep;
     const double cluster = waves(units0, sms / 4) * ((double)C + kFill) * kClusterStep;
     if (cluster < best) { best = cluster; pl.kind = PrefillPlan::kCluster; }
+    // bytes of out (read and written) and Psi (read), bf16, of the segments past the first
+    const double corr_bytes = (double)T_total * H_v * DD * 2 * 3;
     for (long long L = 8; L < C; L += (L < 64 ? 4 : (L < 512 ? 16 : 64))) {
         const long long P = (C + L - 1) / L;
-        const double t = (0.9 * waves(2 * (P - 1) * units0, sms) * ((double)L + kFill) +
-                          waves(P * units0, sms) * ((double)L + kFill) + 4.0) * kChainStep;
+        const double ctas = (double)(P - 1) * units0;
+        const double corr = corr_bytes * (double)(P - 1) / (double)P /
+                            std::min(kCorrectBps, ctas * kCorrectCtaBps) / kStepSeconds;
+        const double t = (waves((2 * P - 1) * units0, sms) * ((double)L + kFill) + 4.0 + corr) * kChainStep;
         if (t < 0.97 * best) { best = t; pl.kind = PrefillPlan::kChain; pl.seg_tokens = (int)(L * CC); }
     }
     return pl;
@@ -994,7 +1179,8 @@ size_t chain_workspace_bytes(int N, long long T_total, int H_v, int sms, int ove
     const int seg = pl.kind == PrefillPlan::kChain ? pl.seg_tokens : 0;
     if (seg == 0) return kHead;
     const long long U = N + T_total / seg;
-    return kHead + (size_t)U * 16 + (size_t)N * 8 + 1024 + 3 * (size_t)U * H_v * kStateBytes;
+    return kHead + (size_t)U * 16 + (size_t)N * 8 + 1024 + 3 * (size_t)U * H_v * kStateBytes +
+           (size_t)T_total * H_v * DD * 2;
 }
 
 void describe_prefill(int N, long long T_total, int H_v, int sms, int override_tokens,
@@ -1062,6 +1248,7 @@ cudaError_t launch_prefill_chain(const void *q, const void *k, const void *v, co
         prm.ws_M = reinterpret_cast<float *>(p);
         prm.ws_B = prm.ws_M + (size_t)U * H_v * DD * DD;
         prm.ws_S = prm.ws_B + (size_t)U * H_v * DD * DD;
+        prm.ws_Psi = reinterpret_cast<__nv_bfloat16 *>(prm.ws_S + (size_t)U * H_v * DD * DD);
         prm.seg_tokens = seg;
         if (cu) {
             segment_plan_kernel<<<1, 32, 0, stream>>>(cu, N, seg, U, units, seqs);
@@ -1072,18 +1259,20 @@ cudaError_t launch_prefill_chain(const void *q, const void *k, const void *v, co
             U = N * prm.units_per_seq;
             seqs = nullptr;
         }
-        // pass 1: the transfers (M in grid slice z = 0, B in slice 1)
-        auto kx = l2n ? prefill_chain_kernel<MODE_XFER, true> : prefill_chain_kernel<MODE_XFER, false>;
-        kx<<<dim3((unsigned)U, (unsigned)H_v, 2), CH_THREADS, CH_SMEM, stream>>>(mq, mk, mv, prm);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        // pass 2: segment start states
-        segment_scan_kernel<<<dim3((unsigned)N, (unsigned)H_v, DD / 16), 256, 0, stream>>>(
-            S0, prm.ws_M, prm.ws_B, prm.ws_S, seqs, N, H_v, prm.units_per_seq);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    // pass 3 (or the only pass): outputs and final states
-    auto ko = l2n ? prefill_chain_kernel<MODE_OUT, true> : prefill_chain_kernel<MODE_OUT, false>;
-    ko<<<dim3((unsigned)U, (unsigned)H_v, 1), CH_THREADS, CH_SMEM, stream>>>(mq, mk, mv, prm);
+    // the chains: per unit, the local chain (slice 1, or the only slice) and, for segments
+    // past the first, the transfer chain (slice 0)
+    auto kc = seg ? (l2n ? prefill_chain_kernel<true, true> : prefill_chain_kernel<false, true>)
+                  : (l2n ? prefill_chain_kernel<true, false> : prefill_chain_kernel<false, false>);
+    kc<<<dim3((unsigned)U, (unsigned)H_v, seg ? 2 : 1), CH_THREADS, CH_SMEM, stream>>>(mq, mk, mv, prm);
+    if ((e = cudaGetLastError()) != cudaSuccess || !seg) return e;
+    // segment start states and final states, then the output corrections
+    segment_scan_kernel<<<dim3((unsigned)N, (unsigned)H_v, DD / 16), 256, 0, stream>>>(
+        prm.ws_M, prm.ws_B, prm.ws_S, S_final, seqs, N, H_v, prm.units_per_seq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    CUtensorMap mpsi;
+    if (!make_map(&mpsi, prm.ws_Psi, T_total, H_v)) return cudaErrorInvalidValue;
+    segment_correct_kernel<<<dim3((unsigned)U, (unsigned)H_v), CR_THREADS, CR_SMEM, stream>>>(mpsi, prm);
     return cudaGetLastError();
 }
 
