@@ -144,7 +144,7 @@ __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ uint32_t par(int k) { return (uint32_t)(k & 1); }
 // every element of a 128-byte row of bf16 scaled by f, in place; the 16-byte pieces are
 // taken in swizzled order, so the rows of a warp's threads touch different banks
-__device__ __forceinline__ void scale_row128(unsigned char *row, int r, float f) {
+__device__ __noinline__ void scale_row128(unsigned char *row, int r, float f) {
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
         unsigned char *pp = row + (((cc ^ r) & 7) << 4);
@@ -208,6 +208,21 @@ __device__ __forceinline__ bool unit_of(const ChainParams &prm, int x, Unit &u)
     return true;
 }
 
+// Bounded wait on barrier b of `bars` for the given phase parity: at most `budget` polls
+// of up to kPollNs each; gives up early once another role of this CTA has aborted.  Out
+// of line: it is called from some thirty places, and the kernel's roles run different code
+// at once, so every copy of the loop would compete for the instruction cache.
+__device__ __noinline__ bool bounded_wait(uint64_t *bars, int b, uint32_t parity, uint32_t budget,
+                                          const volatile int *abort_flag)
+{
+    uint64_t *bar = bars + b;
+    for (uint32_t i = 0; i < budget; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, kPollNs)) return true;
+        if (*abort_flag) return false;
+    }
+    return false;
+}
+
 __device__ __noinline__ void chain_abort(volatile int *abort_flag, DeviceError *err, int where)
 {
     if (!*abort_flag) {
@@ -255,15 +270,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const uint32_t budget = prm.budget;
 
-    // bounded wait: at most `budget` polls of up to kPollNs each; gives up early once
-    // another role of this CTA has aborted
     auto wait_bar = [&](int b, uint32_t parity) -> bool {
-        uint64_t *bar = bars + b;
-        for (uint32_t i = 0; i < budget; ++i) {
-            if (mbar_try_wait_sleep(bar, parity, kPollNs)) return true;
-            if (*abort_flag) return false;
-        }
-        return false;
+        return bounded_wait(bars, b, parity, budget, abort_flag);
     };
     auto fail = [&](int where) { chain_abort(abort_flag, prm.err, where); };
     auto region = [&](int c) -> unsigned char * { return sm + S_REG + (c % NREG) * SR_BYTES; };
@@ -342,7 +350,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 break;
             }
             tc_fence_after();
-#pragma unroll
+#pragma unroll 1
             for (int h2 = 0; h2 < 2; ++h2) {
                 uint32_t ws[32], ut[32];
                 tmem_ld32(tmem + loff + TM_QW + 64 + 32 * h2, ws);
@@ -410,7 +418,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 break;
             }
             // bf16 copy first (the next C1 waits for it), then the pre-scaling
-#pragma unroll
+#pragma unroll 1
             for (int db = 0; db < 4; ++db) {
                 uint32_t xs[32], xb[16];
                 tmem_ld32(tmem + loff + TM_S + 32 * db, xs);
@@ -428,7 +436,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (okw) { tc_fence_after(); issue_c1(c + 1); }
             }
             const float ge = vecbuf(c + 1)[V_GAM + 63];
-#pragma unroll
+#pragma unroll 1
             for (int db = 0; db < 4; ++db) {
                 uint32_t xs[32];
                 tmem_ld32(tmem + loff + TM_S + 32 * db, xs);
@@ -645,7 +653,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int d = v, kb = d >> 6, dc = d & 63;
                 const uint32_t wbase = smem_u32(rg + kb * SR_KB + SR_W);
                 const uint32_t bofs = (uint32_t)((dc & 7) * 2) - (odd ? 2u : 0u);
-#pragma unroll
+#pragma unroll 1
                 for (int h2 = 0; h2 < 2; ++h2) {
                     uint32_t x[32];
                     tmem_ld32(tmem + loff + TM_WT + 32 * h2, x);
@@ -906,11 +914,7 @@ segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi, const __grid_
     const uint32_t tmem = *tmem_slot;
     const uint32_t budget = prm.budget;
     auto wait_bar = [&](int b, uint32_t parity) -> bool {
-        for (uint32_t i = 0; i < budget; ++i) {
-            if (mbar_try_wait_sleep(bars + b, parity, kPollNs)) return true;
-            if (*abort_flag) return false;
-        }
-        return false;
+        return bounded_wait(bars, b, parity, budget, abort_flag);
     };
     auto fail = [&](int where) { chain_abort(abort_flag, prm.err, where); };
 
