@@ -181,10 +181,11 @@ gdn_status gdn_backward(const void *q, const void *k, const void *v, const float
  * needs.  This entry point instead uses a scratch array of GDN_STATIC_SCRATCH_BYTES
  * that the library keeps in every GPU that loads it, for as long as the library is
  * loaded; it calls no cudaMalloc, cudaFree or other allocating routine.
- *   - The first call on a device looks up that array's device address (with that
- *     device current); make this first call before any stream capture.  The address
- *     is cached per device and looked up again when the device's context changes (for
- *     instance after cudaDeviceReset).
+ *   - Every call asks the runtime for that array's device address in the current
+ *     context (cudaGetSymbolAddress: a table lookup once the library's module is
+ *     loaded, and right again after cudaDeviceReset makes a new primary context).
+ *     Make the first call on a device before any stream capture, since it may load
+ *     the module.
  *   - Every call on a device shares the one array: calls that may overlap on the GPU
  *     (different streams, or different host threads) race on it.
  *   - Each call clears the array's error word before it launches.  A device-side

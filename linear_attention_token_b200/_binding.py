@@ -181,6 +181,45 @@ def prefill_workspace(num_seqs: int, T_total: int, H_v: int, dk: int, dv: int,
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def _prefill_shapes(q, k, v, g, beta, S0, cu_seqlens, out, S_final):
+    """Sizes (B, T, N, H_qk, H_v, dk, dv) of a prefill call, after checking every operand
+    against them: the library reads and writes exactly these extents, so a wrong shape, an
+    int64 offset table or a tensor on another device would otherwise be an out-of-bounds
+    device access instead of a Python error."""
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+            raise ValueError("cu_seqlens must be 1-D with num_seqs + 1 entries")
+        if q.dim() != 3:
+            raise ValueError("varlen q must be [T_total, H_qk, dk]")
+        T_total, H_qk, dk = q.shape
+        B, T, N = 1, T_total, cu_seqlens.numel() - 1
+    else:
+        if q.dim() == 4:
+            B, T, H_qk, dk = q.shape
+        elif q.dim() == 3:
+            B, (T, H_qk, dk) = 1, q.shape
+        else:
+            raise ValueError("q must be [B, T, H_qk, dk] or [T, H_qk, dk]")
+        N = B
+    lead = tuple(q.shape[:-2])
+    if v.dim() != q.dim() or tuple(v.shape[:-2]) != lead:
+        raise ValueError(f"v {tuple(v.shape)} does not match q {tuple(q.shape)}")
+    H_v, dv = v.shape[-2:]
+    want = {"k": tuple(q.shape), "g": lead + (H_v,), "beta": lead + (H_v,),
+            "out": tuple(v.shape), "S0": (N, H_v, dk, dv), "S_final": (N, H_v, dk, dv)}
+    for name, t in (("k", k), ("g", g), ("beta", beta), ("out", out), ("S0", S0),
+                    ("S_final", S_final)):
+        if t is not None and tuple(t.shape) != want[name]:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want[name]}")
+    for name, t in (("k", k), ("v", v), ("g", g), ("beta", beta), ("out", out), ("S0", S0),
+                    ("S_final", S_final), ("cu_seqlens", cu_seqlens)):
+        if t is not None and t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
+    return B, T, N, H_qk, H_v, dk, dv
+
+
 def gdn_prefill(q, k, v, g, beta, S0=None, cu_seqlens=None, *, out=None, S_final=None,
                 scale: float = 1.0, flags: int = 0, workspace=None, want_state: bool = True,
                 stream=None):
@@ -192,18 +231,8 @@ def gdn_prefill(q, k, v, g, beta, S0=None, cu_seqlens=None, *, out=None, S_final
     """
     _check_dtypes(q, (("k", k), ("v", v), ("out", out)),
                   (("g", g), ("beta", beta), ("S0", S0), ("S_final", S_final)))
-    if cu_seqlens is not None:
-        T_total, H_qk, dk = q.shape[-3:]
-        B, T, N = 1, T_total, cu_seqlens.numel() - 1
-        if cu_seqlens.dtype != torch.int32:
-            raise TypeError("cu_seqlens must be int32")
-    else:
-        if q.dim() == 4:
-            B, T, H_qk, dk = q.shape
-        else:
-            B, (T, H_qk, dk) = 1, q.shape
-        T_total, N = B * T, B
-    H_v, dv = v.shape[-2:]
+    B, T, N, H_qk, H_v, dk, dv = _prefill_shapes(q, k, v, g, beta, S0, cu_seqlens, out, S_final)
+    T_total = B * T
     if out is None:
         out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
     if S_final is None and want_state:
@@ -230,16 +259,9 @@ def gdn_prefill_static_scratch(q, k, v, g, beta, S0=None, cu_seqlens=None, *, ou
     """
     _check_dtypes(q, (("k", k), ("v", v), ("out", out)),
                   (("g", g), ("beta", beta), ("S0", S0), ("S_final", S_final)))
-    if cu_seqlens is not None:
-        T_total, H_qk, dk = q.shape[-3:]
-        B, T, N = 1, T_total, cu_seqlens.numel() - 1
-    else:
-        if q.dim() == 4:
-            B, T, H_qk, dk = q.shape
-        else:
-            B, (T, H_qk, dk) = 1, q.shape
-        N = B
-    H_v, dv = v.shape[-2:]
+    if out is None:
+        raise ValueError("out must be given: this entry point allocates nothing")
+    B, T, N, H_qk, H_v, dk, dv = _prefill_shapes(q, k, v, g, beta, S0, cu_seqlens, out, S_final)
     st = lib().gdn_prefill_static_scratch(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
         _dev(S0, "S0"), _dev(out, "out"), _dev(S_final, "S_final"),

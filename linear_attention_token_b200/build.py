@@ -35,7 +35,8 @@ def _stale(out: str) -> bool:
     if not os.path.exists(out):
         return True
     t = os.path.getmtime(out)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
+    deps = (sources() + glob.glob(os.path.join(CSRC, "*.cuh")) +
+            glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -8,6 +8,7 @@
 // the n_commit-th token (the accepted prefix).
 #include "common.cuh"
 #include "sm100.cuh"
+#include "device_once.h"
 
 namespace gdn {
 
@@ -196,6 +197,10 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const 
     }
 }
 
+// shared-memory opt-in and SM count, per device, per instantiation
+template <int DK, int DV, typename TIn>
+PerDevice g_multi_setup;
+
 template <int DK, int DV, typename TIn>
 static cudaError_t launch_decode_multi_t(const void *q, const void *k, const void *v,
                                          const float *g, const float *beta, float *S, void *out,
@@ -205,18 +210,15 @@ static cudaError_t launch_decode_multi_t(const void *q, const void *k, const voi
     const long long heads = (long long)N * H_v;
     if (heads == 0) return cudaSuccess;
     constexpr int smem = decode_multi_smem<DK, DV, TIn>();
-    static int sms = 0;
-    static bool attr_set = false;
-    if (!attr_set) {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(decode_multi_kernel<DK, DV, TIn>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    int sms = 0;
+    cudaError_t e = g_multi_setup<DK, DV, TIn>.ensure(
+        [] {
+            return cudaFuncSetAttribute(decode_multi_kernel<DK, DV, TIn>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        decode_multi_smem<DK, DV, TIn>());
+        },
+        &sms);
+    if (e != cudaSuccess) return e;
     const long long grid = heads < 2LL * sms ? heads : 2LL * sms;
     decode_multi_kernel<DK, DV, TIn><<<(unsigned)grid, 256, smem, stream>>>(
         (const TIn *)q, (const TIn *)k, (const TIn *)v, g, beta, S, (TIn *)out, n_commit, T,

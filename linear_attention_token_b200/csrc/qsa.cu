@@ -26,6 +26,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "device_once.h"
 #include "../../include/qsa.h"
 
 namespace gdn {
@@ -780,27 +781,27 @@ namespace {
 
 // Opt a kernel in to more than 48 KB of dynamic shared memory, once per device.
 template <typename K>
-cudaError_t allow_smem(K kernel, size_t bytes, unsigned long long &done) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (dev < 64 && (done & bit)) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess && dev < 64) done |= bit;
-    return e;
+cudaError_t allow_smem(K kernel, size_t bytes, PerDevice &once) {
+    return once.ensure([&] {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)bytes);
+    });
 }
+
+template <int T>
+PerDevice g_score_setup;
+PerDevice g_finish_setup;
 
 template <int T>
 cudaError_t launch_score(const void *q, const int32_t *q_pos, const void *k_hat,
                          const int32_t *cu_blocks, int N, long long total_blocks, int budget,
                          float rope_base, SeqWork *ws, float *scores, cudaStream_t stream) {
-    static unsigned long long done = 0;
     const size_t fixed = (size_t)T * (HBINS * sizeof(uint32_t) + QD * sizeof(float));
     const size_t smem = fixed + (size_t)(36 + N + 1) * sizeof(int);
     // the limit is set once per device, so for the largest call (GDN_QSA_MAX_SEQS sequences)
     cudaError_t e = allow_smem(qsa_score_kernel<T>,
-                               fixed + (size_t)(36 + GDN_QSA_MAX_SEQS + 1) * sizeof(int), done);
+                               fixed + (size_t)(36 + GDN_QSA_MAX_SEQS + 1) * sizeof(int),
+                               g_score_setup<T>);
     if (e != cudaSuccess) return e;
     qsa_score_kernel<T><<<sm_count() * (T == 1 ? 4 : 2), kScoreThreads, smem, stream>>>(
         static_cast<const __nv_bfloat16 *>(q), q_pos, static_cast<const __nv_bfloat16 *>(k_hat),
@@ -840,8 +841,7 @@ cudaError_t launch_qsa_index(const void *q, const int32_t *q_pos, const void *k_
     e = cudaLaunchKernelEx(&cfg, qsa_collect_kernel, q_pos, cu_blocks, N, T, (int)total_blocks,
                            (const float *)scores, ws);
     if (e != cudaSuccess) return e;
-    static unsigned long long finish_done = 0;
-    if ((e = allow_smem(qsa_finish_kernel, kFinishSmem, finish_done)) != cudaSuccess) return e;
+    if ((e = allow_smem(qsa_finish_kernel, kFinishSmem, g_finish_setup)) != cudaSuccess) return e;
     cfg.gridDim = dim3(N * T);
     cfg.blockDim = dim3(kFinishThreads);
     cfg.dynamicSmemBytes = kFinishSmem;

@@ -10,7 +10,7 @@
  *   text under Eq. (1): alpha_t in (0,1) is the decay gate, beta_t in (0,1) the
  *             write strength;
  *   concept code: the output is read after the update, y = S^T q.
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent:
  *   alpha_t = exp(g_t); S is dk x dv with dv contiguous; value head h reads
  *   q/k head h / (H_v / H_qk); the output is multiplied by `scale`; the optional
  *   q/k L2 normalisation divides by sqrt(sum x^2 + 1e-6).
