@@ -608,6 +608,37 @@ def run_qsa_only(args):
         print(json.dumps(line), flush=True)
 
 
+def run_prefill_only(args):
+    """--section prefill: one prefill workload alone (one JSON line), optionally cut to its
+    first --prefill-tokens tokens per sequence, so a profiler can capture a few launches on
+    a small case of the same kernels."""
+    import dataclasses
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    import linear_attention_token_b200 as gdn
+    gdn.lib()
+    peaks = load_peaks()
+    w = inputs.get(args.prefill_workload)
+    if args.prefill_tokens:
+        n = int(args.prefill_tokens)
+        w = dataclasses.replace(w, name=f"{w.name}_first{n}",
+                                seq_lens=tuple(min(n, L) for L in w.seq_lens))
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    x = inputs.prefill_inputs(w, device=device)
+    with ClockSampler(0) as clk:
+        times, status, sched = time_prefill(gdn, x, w, max(1, args.steps), max(args.warmup, 1),
+                                            stream, flush)
+    if status != 0:
+        raise RuntimeError(f"device error after prefill: {gdn.gdn_status_string(status)}")
+    ms = sum(times) / len(times)
+    print(json.dumps({"metric": "GDN prefill tokens/s on 1 B200", "value": w.tokens / (ms * 1e-3),
+                      "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps,
+                      "config": {"workload": w.name, "schedule": sched},
+                      "roofline": prefill_roofline(w, ms, peaks, sched),
+                      "clocks": clk.summary()}), flush=True)
+
+
 def prefill_roofline(w, ms, peaks, sched, traffic=None):
     """Roofline of one prefill call: the method's FLOPs (chunked contractions at tile
     shape) and algorithmic bytes over the call's device time."""
@@ -634,6 +665,8 @@ def short_section(name, value, unit, ms, roof=None, **kw):
 def run_ours(args):
     if args.section == "qsa":
         return run_qsa_only(args)
+    if args.section == "prefill":
+        return run_prefill_only(args)
     rank, world, local = dist_init()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -820,8 +853,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--section", choices=["all", "qsa"], default="all",
-                    help="qsa: time only the QSA indexer and compression (profiling aid)")
+    ap.add_argument("--section", choices=["all", "qsa", "prefill"], default="all",
+                    help="qsa: time only the QSA indexer and compression; prefill: one prefill "
+                         "workload alone (profiling aids)")
+    ap.add_argument("--prefill-workload", type=int, choices=[1, 2, 3], default=PREFILL_W,
+                    help="--section prefill: the workload (1 mid-size, 2 varlen, 3 long context)")
+    ap.add_argument("--prefill-tokens", type=int, default=0,
+                    help="--section prefill: keep only the first N tokens of each sequence")
     ap.add_argument("--qsa-seqs", type=int, default=8,
                     help="sequences of the QSA workload (1,048,576 cached tokens each)")
     args = ap.parse_args()

@@ -13,8 +13,9 @@
 // The state chain runs transposed: S^T (value column v in TMEM lane v, key index d in
 // column d) stays in TMEM for the whole unit, and every chain product has the 128 value
 // columns as its M dimension, so one CTA carries a whole head at full MMA width:
-//   C1  [ (Q~ S)^T | (W S)^T ] = S^T [Q~; W]^T     (A = S^T bf16 in TMEM, N = 128)
-//   E3  U^T = U~^T - (W S)^T  -> shared memory (bf16)
+//   C1  (Q~ S)^T = S^T Q~^T, and (W S)^T - U~^T = S^T W^T + (-U~^T), accumulated onto
+//       the -U~^T that P3 left in one of two buffers (A = S^T bf16 in TMEM, N = 64 each)
+//   E3  U^T = -((W S)^T - U~^T)  -> shared memory (bf16)
 //   C2  S^T += U^T K~                               (S^T pre-scaled by gamma_end)
 //   C3  O^T = (Q~ S)^T + U^T P^T                     (off the chain, second issuer)
 //   E4  S^T -> bf16 copy for the next C1, then S^T *= gamma_end(next)
@@ -70,8 +71,9 @@ constexpr uint32_t kPollNs = 2000;      // longest hardware suspension of one po
 
 // TMEM columns (512 allocated)
 constexpr uint32_t TM_S = 0;        // 128: S^T fp32 (lane v, column d), pre-scaled by gamma_end
-constexpr uint32_t TM_QW = 128;     // 128: [ O^T (Q~ S + P U)^T | (W S)^T ], lane v, column token
-constexpr uint32_t TM_UT = 256;     // 64:  U~^T fp32 (lane v, column token)
+constexpr uint32_t TM_QW = 128;     // 64:  O^T = (Q~ S + P U)^T, lane v, column token
+constexpr uint32_t TM_WU0 = 192;    // 2 x 64: -U^T = (W S)^T - U~^T of chunks of parity 0, 1
+constexpr uint32_t TM_WU1 = 256;    //   (P3 writes -U~^T, C1 adds (W S)^T; lane v, column token)
 constexpr uint32_t TM_SB = 320;     // 64:  S^T bf16 pairs (A operand of C1)
 constexpr uint32_t TM_KQ = 384;     // 64:  [K;Q] K^T (lanes 0-63 K K^T, 64-127 Q K^T)
 constexpr uint32_t TM_WT = 448;     // 64:  W^T fp32 (lane d, column token)
@@ -104,7 +106,9 @@ enum Bar {
     B_LD0 = 0, B_LD1, B_LD2,           // loader: K (Q, V) of the region's chunk landed
     B_VEC0, B_VEC1, B_VEC2,            // loader: vectors of the buffer's chunk
     B_IN,                              // prep: inputs normalised (q/k L2 norm only)
-    B_P1, B_KQF, B_TT, B_P2, B_WTF, B_P3, B_UF,
+    B_P1, B_KQF, B_TT, B_P2, B_WTF,
+    B_P30, B_P31,                      // P3 of chunks of parity 0, 1
+    B_UF0, B_UF1,                      // chain: -U^T buffer of parity 0, 1 read
     B_RDY0, B_RDY1, B_RDY2,            // output group: chunk ready for the chain
     B_C1, B_C2, B_C3, B_OF,
     B_RF0, B_RF1, B_RF2,               // commit: region free (after C2)
@@ -145,7 +149,7 @@ __device__ __forceinline__ uint32_t par(int k) { return (uint32_t)(k & 1); }
 // every element of a 128-byte row of bf16 scaled by f, in place; the 16-byte pieces are
 // taken in swizzled order, so the rows of a warp's threads touch different banks
 __device__ __noinline__ void scale_row128(unsigned char *row, int r, float f) {
-#pragma unroll
+#pragma unroll 2
     for (int cc = 0; cc < 8; ++cc) {
         unsigned char *pp = row + (((cc ^ r) & 7) << 4);
         uint4 w = *reinterpret_cast<const uint4 *>(pp);
@@ -154,6 +158,14 @@ __device__ __noinline__ void scale_row128(unsigned char *row, int r, float f) {
         for (int e = 0; e < 4; ++e) { const float2 x = unpack2(wv[e]); wv[e] = pack2(x.x * f, x.y * f); }
         *reinterpret_cast<uint4 *>(pp) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
+}
+
+// The gate prologue of one loader lane's two tokens: (log-decay g0, g1, strength b0, b1);
+// a token past the unit contributes nothing.  Out of line: one copy of the gate code.
+__device__ __noinline__ float4 gate_pair(float g0, float g1, float b0, float b1, bool in0, bool in1,
+                                         int opts) {
+    return make_float4(in0 ? gate_log_decay(g0, opts) : 0.f, in1 ? gate_log_decay(g1, opts) : 0.f,
+                       in0 ? gate_strength(b0, opts) : 0.f, in1 ? gate_strength(b1, opts) : 0.f);
 }
 
 }  // namespace
@@ -283,7 +295,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // =============================================================== chain group
         const int t = tid, v = tid, q = warp;
         const uint32_t loff = (uint32_t)(32 * q) << 16;
-        const uint32_t id_c1 = idesc_bf16(128, 128, false, false);
+        const uint32_t id_c1 = idesc_bf16(128, 64, false, false);
         const uint32_t id_c2 = idesc_bf16(128, 128, false, true);
         const uint32_t id_c3 = idesc_bf16(128, 64, false, false);
         const uint32_t su = smem_u32(sm + S_U);
@@ -291,11 +303,14 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         int mma_issued = 0;
 
         auto issue_c1 = [&](int c) {           // thread 0
-            const uint32_t base = smem_u32(region(c)) + SR_Q;
-#pragma unroll
+            const uint32_t rq = smem_u32(region(c)) + SR_Q, rw = smem_u32(region(c)) + SR_W;
+            const uint32_t wu = tmem + ((c & 1) ? TM_WU1 : TM_WU0);
+#pragma unroll 1
             for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t bd = sdesc_kmajor(base + (ks >> 2) * SR_KB + (ks & 3) * 32);
-                umma_bf16_ta(tmem + TM_QW, tmem + TM_SB + 8 * ks, bd, id_c1, ks > 0);
+                const uint32_t ko = (ks >> 2) * SR_KB + (ks & 3) * 32;
+                // (W S)^T onto P3's -U~^T (the transfer chain has U~ = 0: a fresh sum)
+                umma_bf16_ta(wu, tmem + TM_SB + 8 * ks, sdesc_kmajor(rw + ko), id_c1, !xa || ks > 0);
+                umma_bf16_ta(tmem + TM_QW, tmem + TM_SB + 8 * ks, sdesc_kmajor(rq + ko), id_c1, ks > 0);
             }
             umma_commit(bars + B_C1);
             ++mma_issued;
@@ -344,17 +359,18 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
 #pragma unroll 1
         for (int c = 0; ok && c < nch; ++c) {
-            // ---- E3: U^T = U~^T - (W S)^T  ->  U^T (bf16, K-major rows v)
-            if (!group_all<1>(t != 0 || (wait_bar(B_C1, par(c)) && (xa || wait_bar(B_P3, par(c)))))) {
+            // ---- E3: U^T = -((W S)^T - U~^T)  ->  U^T (bf16, K-major rows v).  C1 was
+            // issued after RDY(c), which the output group raised only once P3(c) was done.
+            if (!group_all<1>(t != 0 || wait_bar(B_C1, par(c)))) {
                 fail(3);
                 break;
             }
             tc_fence_after();
+            const uint32_t wu = (c & 1) ? TM_WU1 : TM_WU0;
 #pragma unroll 1
             for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t ws[32], ut[32];
-                tmem_ld32(tmem + loff + TM_QW + 64 + 32 * h2, ws);
-                if (!xa) tmem_ld32(tmem + loff + TM_UT + 32 * h2, ut);
+                uint32_t nu[32];
+                tmem_ld32(tmem + loff + wu + 32 * h2, nu);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -362,9 +378,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int j = 8 * k + 2 * e;
-                        const float u0 = (xa ? 0.f : __uint_as_float(ut[j])) - __uint_as_float(ws[j]);
-                        const float u1 = (xa ? 0.f : __uint_as_float(ut[j + 1])) - __uint_as_float(ws[j + 1]);
-                        pu[e] = pack2(u0, u1);
+                        pu[e] = pack2(-__uint_as_float(nu[j]), -__uint_as_float(nu[j + 1]));
                     }
                     *reinterpret_cast<uint4 *>(sm + S_U + sw128(v, 4 * h2 + k)) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
                 }
@@ -373,12 +387,12 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             tc_fence_before();
             group_sync<1>();
             if (t == 0) {
-                if (!xa) mbar_arrive_local(bars + B_UF);
+                if (!xa) mbar_arrive_local(bars + B_UF0 + (c & 1));
                 mbar_arrive_local(bars + rbar(B_VF0, c));
                 tc_fence_after();
                 // ---- C2: S^T += U^T K~
                 const uint32_t kreg = smem_u32(region(c));
-#pragma unroll
+#pragma unroll 1
                 for (int ks = 0; ks < 4; ++ks)
                     umma_bf16(tmem + TM_S, sdesc_kmajor(su + ks * 32),
                               sdesc_mnmajor(kreg + ks * 2048, SR_KB), id_c2, 1);
@@ -389,7 +403,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 // ---- C3: O^T += U^T P^T, issued beside C2 (off the chain)
                 tc_fence_after();
                 const uint32_t pt = smem_u32(sm + S_P + (c % NREG) * 8192);
-#pragma unroll
+#pragma unroll 1
                 for (int ks = 0; ks < 4; ++ks)
                     umma_bf16(tmem + TM_QW, sdesc_kmajor(su + ks * 32), sdesc_kmajor(pt + ks * 32), id_c3, 1);
                 umma_commit(bars + B_C3);
@@ -514,18 +528,18 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const float *fsrc = vb + (factored ? V_INV : V_G);
                 {
 #pragma unroll 1
-                    for (int jh = 0; jh < 64; jh += 32) {
+                    for (int jh = 0; jh < 64; jh += 16) {
                         if (is_a && jh >= jend) break;    // the inverse never reads A above the diagonal
-                        float xv[32];
+                        float xv[16];
                         if (jh >= jend) {
 #pragma unroll
-                            for (int u = 0; u < 32; ++u) xv[u] = 0.f;
+                            for (int u = 0; u < 16; ++u) xv[u] = 0.f;
                         } else {
-                            uint32_t kr[32];
-                            tmem_ld32(tmem + loff + TM_KQ + jh, kr);
+                            uint32_t kr[16];
+                            tmem_ld16(tmem + loff + TM_KQ + jh, kr);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int u = 0; u < 32; u += 4) {
+                            for (int u = 0; u < 16; u += 4) {
                                 const float4 f4 = *reinterpret_cast<const float4 *>(fsrc + jh + u);
                                 const float fj[4] = {f4.x, f4.y, f4.z, f4.w};
 #pragma unroll
@@ -539,11 +553,11 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         }
                         if (is_a) {
 #pragma unroll
-                            for (int u = 0; u < 32; u += 4)
+                            for (int u = 0; u < 16; u += 4)
                                 *reinterpret_cast<float4 *>(Mf + i * TP + jh + u) = make_float4(xv[u], xv[u + 1], xv[u + 2], xv[u + 3]);
                         } else {
 #pragma unroll
-                            for (int h2 = 0; h2 < 4; ++h2)
+                            for (int h2 = 0; h2 < 2; ++h2)
                                 *reinterpret_cast<uint4 *>(pt + sw128(i, (jh >> 3) + h2)) = make_uint4(
                                     pack2(xv[8 * h2 + 0], xv[8 * h2 + 1]), pack2(xv[8 * h2 + 2], xv[8 * h2 + 3]),
                                     pack2(xv[8 * h2 + 4], xv[8 * h2 + 5]), pack2(xv[8 * h2 + 6], xv[8 * h2 + 7]));
@@ -557,9 +571,9 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (t == 0) mbar_arrive_local(bars + B_KQF);
             // ---- T = (I + A)^-1, in place
             invert_unit_lower_64_inplace_wg<TP>(Mf, t, [] { group_sync<2>(); });
-            // ---- T' = T diag(beta gamma), T'' = T diag(beta) (bf16, K-major rows i), once
+            // ---- T' = T diag(beta gamma), -T'' = -T diag(beta) (bf16, K-major rows i), once
             // the previous chunk's P2 and P3 have read the last ones
-            if (!group_all<2>(t != 0 || c == 0 || (wait_bar(B_P2, par(c - 1)) && (xa || wait_bar(B_P3, par(c - 1)))))) {
+            if (!group_all<2>(t != 0 || c == 0 || (wait_bar(B_P2, par(c - 1)) && (xa || wait_bar(B_P30 + ((c - 1) & 1), par((c - 1) >> 1)))))) {
                 fail(12);
                 break;
             }
@@ -567,7 +581,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int i = t >> 1, half = t & 1;           // row i, columns [32 half, +32)
                 const float *trow = Mf + i * TP + 32 * half;
                 unsigned char *tp1 = sm + S_TT, *tp2 = sm + S_TT + 8192;
-#pragma unroll
+#pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     const int j0 = 32 * half + 8 * cc;
                     uint4 o1 = make_uint4(0u, 0u, 0u, 0u), o2 = o1;
@@ -586,7 +600,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         for (int e = 0; e < 8; ++e) {
                             const float tt = (j0 + e <= i) ? tv[e] : 0.f;
                             w1[e] = tt * gv[e];
-                            w2[e] = tt * bv[e];
+                            w2[e] = -tt * bv[e];
                         }
                         o1 = make_uint4(pack2(w1[0], w1[1]), pack2(w1[2], w1[3]), pack2(w1[4], w1[5]), pack2(w1[6], w1[7]));
                         o2 = make_uint4(pack2(w2[0], w2[1]), pack2(w2[2], w2[3]), pack2(w2[4], w2[5]), pack2(w2[6], w2[7]));
@@ -608,6 +622,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const uint32_t loff = (uint32_t)(32 * q) << 16;
         const bool odd = l & 1;
         const float scale = prm.scale;
+        // outputs of chunk c: O^T (lane v) is read out of TMEM and the accumulator handed
+        // back to the chain first; the rows are written after that
         auto outputs = [&](int c) -> bool {
             if (!group_all<3>(t != 0 || wait_bar(B_C3, par(c)))) return false;
             tc_fence_after();
@@ -642,49 +658,50 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             return true;
         };
 #pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-            unsigned char *rg = region(c);
-            const float *vb = vecbuf(c);
-            // ---- W^T (lane d) -> W rows (K-major, token i) over V in the region's W slots
-            // (P3 has read V); P2 and P3 follow P1, so Q and K are free to scale
-            if (!group_all<3>(t != 0 || (wait_bar(B_P2, par(c)) && (xa || wait_bar(B_P3, par(c)))))) { fail(20); break; }
-            tc_fence_after();
-            {
-                const int d = v, kb = d >> 6, dc = d & 63;
-                const uint32_t wbase = smem_u32(rg + kb * SR_KB + SR_W);
-                const uint32_t bofs = (uint32_t)((dc & 7) * 2) - (odd ? 2u : 0u);
+        for (int c = 0; c <= nch; ++c) {
+            if (c < nch) {
+                unsigned char *rg = region(c);
+                const float *vb = vecbuf(c);
+                // ---- W^T (lane d) -> W rows (K-major, token i) over V in the region's W slots
+                // (P3 has read V); P2 and P3 follow P1, so Q and K are free to scale
+                if (!group_all<3>(t != 0 || (wait_bar(B_P2, par(c)) && (xa || wait_bar(B_P30 + (c & 1), par(c >> 1)))))) { fail(20); break; }
+                tc_fence_after();
+                {
+                    const int d = v, kb = d >> 6, dc = d & 63;
+                    const uint32_t wbase = smem_u32(rg + kb * SR_KB + SR_W);
+                    const uint32_t bofs = (uint32_t)((dc & 7) * 2) - (odd ? 2u : 0u);
 #pragma unroll 1
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t x[32];
-                    tmem_ld32(tmem + loff + TM_WT + 32 * h2, x);
-                    tmem_wait_ld();
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t x[32];
+                        tmem_ld32(tmem + loff + TM_WT + 32 * h2, x);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int ii = 0; ii < 32; ii += 2) {
-                        const float send = __uint_as_float(odd ? x[ii] : x[ii + 1]);
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                        const int r = 32 * h2 + ii + (odd ? 1 : 0);
-                        const uint32_t val = odd ? pack2(recv, __uint_as_float(x[ii + 1]))
-                                                 : pack2(__uint_as_float(x[ii]), recv);
-                        st_shared_u32(wbase + sw128(r, dc >> 3) + bofs, val);
+                        for (int ii = 0; ii < 32; ii += 2) {
+                            const float send = __uint_as_float(odd ? x[ii] : x[ii + 1]);
+                            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                            const int r = 32 * h2 + ii + (odd ? 1 : 0);
+                            const uint32_t val = odd ? pack2(recv, __uint_as_float(x[ii + 1]))
+                                                     : pack2(__uint_as_float(x[ii]), recv);
+                            st_shared_u32(wbase + sw128(r, dc >> 3) + bofs, val);
+                        }
                     }
                 }
-            }
-            tc_fence_before();
-            // ---- K~ = diag(dte) K and Q~ = diag(gamma) Q, rows in place
-            {
-                const int r = t & 63, kb = t >> 6;
-                scale_row128(rg + kb * SR_KB + r * 128, r, vb[V_DTE + r]);
-                scale_row128(rg + kb * SR_KB + SR_Q + r * 128, r, vb[V_GAM + r]);
-            }
-            fence_proxy_async();
-            group_sync<3>();
-            if (t == 0) {
-                mbar_arrive_local(bars + B_WTF);
-                mbar_arrive_local(bars + rbar(B_RDY0, c));
+                tc_fence_before();
+                // ---- K~ = diag(dte) K and Q~ = diag(gamma) Q, rows in place
+                {
+                    const int r = t & 63, kb = t >> 6;
+                    scale_row128(rg + kb * SR_KB + r * 128, r, vb[V_DTE + r]);
+                    scale_row128(rg + kb * SR_KB + SR_Q + r * 128, r, vb[V_GAM + r]);
+                }
+                fence_proxy_async();
+                group_sync<3>();
+                if (t == 0) {
+                    mbar_arrive_local(bars + B_WTF);
+                    mbar_arrive_local(bars + rbar(B_RDY0, c));
+                }
             }
             if (c >= 1 && !outputs(c - 1)) { fail(21); break; }
         }
-        if (nch > 0 && !*abort_flag && !outputs(nch - 1)) fail(22);
     } else if (warp == 12) {
         // =============================================================== prep issuer
         if (lane == 0) {
@@ -700,7 +717,7 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     return false;
                 tc_fence_after();
                 const uint32_t rg = smem_u32(region(c));
-#pragma unroll
+#pragma unroll 1
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t a = rg + (ks >> 2) * SR_KB + (ks & 3) * 32;
                     umma_bf16(tmem + TM_KQ, sdesc_kmajor(a), sdesc_kmajor(a), id_p1, ks > 0);
@@ -719,20 +736,21 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 // P2: W^T = K^T T'^T
                 if (!wait_bar(B_TT, par(c)) || (c > 0 && !wait_bar(B_WTF, par(c - 1)))) { fail(31); break; }
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int ks = 0; ks < 4; ++ks)
                     umma_bf16(tmem + TM_WT, sdesc_mnmajor(rg + ks * 2048, SR_KB), sdesc_kmajor(tpa + ks * 32),
                               id_p23, ks > 0);
                 umma_commit(bars + B_P2);
-                // P3: U~^T = V^T T''^T, V in the W slots (transfer M: U~ = 0, nothing to do)
+                // P3: -U~^T = V^T (-T'')^T, V in the W slots, into the -U^T buffer of the
+                // chunk's parity once E3(c - 2) has read it (transfer M: U~ = 0, no P3)
                 if (!xa) {
-                    if (c > 0 && !wait_bar(B_UF, par(c - 1))) { fail(32); break; }
+                    if (c > 1 && !wait_bar(B_UF0 + (c & 1), par((c >> 1) - 1))) { fail(32); break; }
                     tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                     for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tmem + TM_UT, sdesc_mnmajor(rg + SR_W + ks * 2048, SR_KB),
+                        umma_bf16(tmem + ((c & 1) ? TM_WU1 : TM_WU0), sdesc_mnmajor(rg + SR_W + ks * 2048, SR_KB),
                                   sdesc_kmajor(tpa + 8192 + ks * 32), id_p23, ks > 0);
-                    umma_commit(bars + B_P3);
+                    umma_commit(bars + B_P30 + (c & 1));
                 }
             }
             if (*abort_flag && issued > 0) {
@@ -745,14 +763,19 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         // ==================================================================== loader
         const int l = lane;
         int ld_issued[NREG] = {};
-        float pg0 = 0.f, pg1 = 0.f, pb0 = 0.f, pb1 = 0.f;    // g, beta of tokens 2l, 2l+1
+        // g, beta of tokens 2l, 2l+1 as stored (loaded a chunk ahead), and whether the
+        // tokens lie inside the unit
+        float rg0 = 0.f, rg1 = 0.f, rb0 = 0.f, rb1 = 0.f;
+        bool in0 = false, in1 = false;
         auto fetch = [&](int c) {
             const long long t0 = un.tb + (long long)c * CC;
             const long long i0 = t0 + 2 * l, i1 = i0 + 1;
-            pg0 = i0 < un.te ? gate_log_decay(prm.g[(size_t)i0 * prm.H_v + h], prm.opts) : 0.f;
-            pg1 = i1 < un.te ? gate_log_decay(prm.g[(size_t)i1 * prm.H_v + h], prm.opts) : 0.f;
-            pb0 = i0 < un.te ? gate_strength(prm.beta[(size_t)i0 * prm.H_v + h], prm.opts) : 0.f;
-            pb1 = i1 < un.te ? gate_strength(prm.beta[(size_t)i1 * prm.H_v + h], prm.opts) : 0.f;
+            in0 = i0 < un.te;
+            in1 = i1 < un.te;
+            rg0 = in0 ? prm.g[(size_t)i0 * prm.H_v + h] : 0.f;
+            rg1 = in1 ? prm.g[(size_t)i1 * prm.H_v + h] : 0.f;
+            rb0 = in0 ? prm.beta[(size_t)i0 * prm.H_v + h] : 0.f;
+            rb1 = in1 ? prm.beta[(size_t)i1 * prm.H_v + h] : 0.f;
         };
         if (nch > 0) fetch(0);
 #pragma unroll 1
@@ -783,6 +806,8 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // ---- vectors of chunk c: G (in-chunk cumsum), gamma, exp(-G), decay to chunk
             // end, beta gamma
             float *vb = vecbuf(c);
+            const float4 gt = gate_pair(rg0, rg1, rb0, rb1, in0, in1, prm.opts);
+            const float pg0 = gt.x, pg1 = gt.y, pb0 = gt.z, pb1 = gt.w;
             float sc = pg0 + pg1;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -875,20 +900,28 @@ segment_scan_kernel(const float *ws_M, const float *ws_B, float *ws_S, float *S_
 // segment's start state to every token's output.  out[t] += Psi[t] S_in(p) for the
 // segment's tokens, on the tensor cores: (Psi S_in)^T = S_in^T Psi^T, A = S_in^T (bf16 in
 // TMEM, lane = value column), B = a 64-token tile of Psi (K-major rows, by TMA), D in TMEM.
-// One CTA per (unit, value head); 160 threads: warps 0-3 convert S_in and run the
-// epilogue (thread 0 issues the MMAs), warp 4 streams Psi through NBUF buffers.
+// The pass is bound by HBM (read Psi, read and write out), so every chunk's Psi and out
+// tiles come in by TMA several chunks ahead, the sum is formed in shared memory and a full
+// chunk goes back by a TMA store; the partial last chunk of a sequence is written row by
+// row, so no store reaches past the unit.
+// One CTA per (unit, value head), two per SM; 160 threads: warps 0-3 convert S_in and run
+// the epilogue (thread 0 issues the MMAs and the stores), warp 4 loads.
 namespace {
-constexpr int CR_THREADS = 160, CR_NBUF = 4;
+constexpr int CR_THREADS = 160, CR_NBUF = 3;
 constexpr uint32_t CR_TM_A = 0, CR_TM_D = 64;          // TMEM: S_in^T bf16, two 64-column D
-constexpr uint32_t CR_BAR = CR_NBUF * 16384;
+constexpr uint32_t CR_BUF = 32768;                     // Psi tile (16 KB) | out tile (16 KB)
+constexpr uint32_t CR_OUT = 16384;
+constexpr uint32_t CR_BAR = CR_NBUF * CR_BUF;
 constexpr uint32_t CR_SMEM = CR_BAR + 16 * 8 + 16 + 1024;
-enum CrBar { CR_LD0 = 0, CR_FREE0 = CR_NBUF, CR_DONE0 = 2 * CR_NBUF, CR_DFREE0 = CR_DONE0 + 2,
-             CR_DRAIN = CR_DFREE0 + 2, CR_COUNT };
+enum CrBar { CR_LD0 = 0, CR_FREE0 = CR_NBUF, CR_DONE0 = 2 * CR_NBUF, CR_DRAIN = CR_DONE0 + 2,
+             CR_COUNT };
 static_assert(CR_COUNT <= 16, "correction barriers");
+static_assert(2 * (CR_SMEM + 1024) <= 233472, "two correction CTAs per SM");
 }  // namespace
 
 __global__ void __launch_bounds__(CR_THREADS)
-segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi, const __grid_constant__ ChainParams prm)
+segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi,
+                       const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ ChainParams prm)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -921,9 +954,8 @@ segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi, const __grid_
     if (warp < 4) {
         const int t = tid, v = tid;
         const uint32_t loff = (uint32_t)(32 * warp) << 16;
-        const bool odd = lane & 1;
         const uint32_t id_c = idesc_bf16(128, 64, false, false);
-        int issued = 0;
+        int issued = 0, stored = 0;
         // S_in^T (bf16 pairs, lane v, column d / 2)
         const float *src = prm.ws_S + ((size_t)blockIdx.x * prm.H_v + h) * DD * DD;
 #pragma unroll 1
@@ -939,82 +971,97 @@ segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi, const __grid_
         tmem_wait_st();
         tc_fence_before();
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        auto issue = [&](int c) -> bool {        // thread 0
+        auto issue = [&](int c) -> bool {        // thread 0; D(c & 1) was read at c - 2
             const int b = c % CR_NBUF;
             if (!wait_bar(CR_LD0 + b, par(c / CR_NBUF))) return false;
             tc_fence_after();
-            const uint32_t base = smem_u32(sm + b * 16384);
+            const uint32_t base = smem_u32(sm + b * CR_BUF);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 umma_bf16_ta(tmem + CR_TM_D + 64 * (c & 1), tmem + CR_TM_A + 8 * ks,
                              sdesc_kmajor(base + (ks >> 2) * 8192 + (ks & 3) * 32), id_c, ks > 0);
             umma_commit(bars + CR_DONE0 + (c & 1));
-            umma_commit(bars + CR_FREE0 + b);
             ++issued;
             return true;
         };
-        bool ok = true;
-        if (t == 0) {
-            ok = issue(0) && (nch < 2 || issue(1));
-            if (!ok) fail(50);
-        }
-        const size_t rstride = (size_t)prm.H_v * DD;
+        if (t == 0 && !issue(0)) fail(50);
+        // element (token r, value v) of a 64-token out tile: two 64-value boxes of 128-byte
+        // rows in the 128-byte swizzle
+        const uint32_t vcol = (uint32_t)(v >> 6) * 8192u, vb2 = (uint32_t)(v & 63) * 2u;
+        const long long rstride = (long long)prm.H_v * DD;
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
+            const int b = c % CR_NBUF;
+            // the store of chunk c - 1 has read its tile: the buffer goes back to the loader
+            // a whole chunk before the tile it will hold is needed.  The next chunk's MMA
+            // (into the D buffer read at c - 1) runs beside this chunk's epilogue.
+            if (t == 0) {
+                if (c >= 1) {
+                    bulk_wait_read_all();
+                    mbar_arrive_local(bars + CR_FREE0 + (c - 1) % CR_NBUF);
+                }
+                if (c + 1 < nch && !*abort_flag && !issue(c + 1)) fail(51);
+            }
             uint32_t ok2;
             {
                 const bool w = t != 0 || (!*abort_flag && wait_bar(CR_DONE0 + (c & 1), par(c >> 1)));
                 asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
                              "selp.u32 %0, 1, 0, q;\n\t}" : "=r"(ok2) : "r"(w ? 1u : 0u) : "memory");
             }
-            if (!ok2) { fail(51); break; }
+            if (!ok2) { fail(52); break; }
             tc_fence_after();
+            const long long t0 = un.tb + (long long)c * CC;
+            const int L = (int)min((long long)CC, un.te - t0);
+            unsigned char *ot = sm + b * CR_BUF + CR_OUT + vcol;
             uint32_t x0[32], x1[32];
             tmem_ld32(tmem + loff + CR_TM_D + 64 * (c & 1), x0);
             tmem_ld32(tmem + loff + CR_TM_D + 64 * (c & 1) + 32, x1);
             tmem_wait_ld();
             tc_fence_before();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (t == 0 && c + 2 < nch && !issue(c + 2)) fail(52);
-            const long long t0 = un.tb + (long long)c * CC;
-            const int L = (int)min((long long)CC, un.te - t0);
-            __nv_bfloat16 *obase = prm.out + ((size_t)t0 * prm.H_v + h) * DD + (v & ~1);
-            // lanes (v, v ^ 1) pair up: the even lane updates token 2m's two values, the odd
-            // lane token 2m + 1's.  Every old value is loaded before any store, so the 32
-            // loads are in flight together.
-            uint32_t old[32];
 #pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const int r = 2 * m + (odd ? 1 : 0);
-                old[m] = r < L ? __ldcs(reinterpret_cast<const unsigned int *>(obase + (size_t)r * rstride)) : 0u;
+            for (int r = 0; r < 64; ++r) {
+                const uint32_t off = (uint32_t)r * 128u + ((((vb2 >> 4) ^ (uint32_t)(r & 7)) << 4) | (vb2 & 15u));
+                __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(ot + off);
+                const float d = __uint_as_float(r < 32 ? x0[r] : x1[r - 32]);
+                const __nv_bfloat16 o = __float2bfloat16_rn(__bfloat162float(*e) + d);
+                if (L == CC) *e = o;
+                else if (r < L) prm.out[(size_t)(t0 + r) * rstride + (size_t)h * DD + v] = o;
             }
-#pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const uint32_t *xx = m < 16 ? x0 : x1;
-                const int mm = 2 * (m & 15);
-                const float a0 = __uint_as_float(xx[mm]), a1 = __uint_as_float(xx[mm + 1]);
-                const float recv = __shfl_xor_sync(0xffffffffu, odd ? a0 : a1, 1);
-                const int r = 2 * m + (odd ? 1 : 0);
-                const float2 o = unpack2(old[m]);
-                const uint32_t val = odd ? pack2(o.x + recv, o.y + a1) : pack2(o.x + a0, o.y + recv);
-                if (r < L) __stcs(reinterpret_cast<unsigned int *>(obase + (size_t)r * rstride), val);
+            if (L == CC) fence_proxy_async();
+            // every thread has read D(c) (the next MMA into it is issued at c + 1) and, for a
+            // full chunk, written the tile
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (t == 0) {
+                if (L == CC) {
+                    unsigned char *o0 = sm + b * CR_BUF + CR_OUT;
+                    tma_store_3d(&tm_out, o0, 0, h, (int)t0);
+                    tma_store_3d(&tm_out, o0 + 8192, 64, h, (int)t0);
+                    bulk_commit();
+                    ++stored;
+                }
             }
         }
-        if (*abort_flag && t == 0 && issued > 0) {
-            umma_commit(bars + CR_DRAIN);
-            mbar_wait(bars + CR_DRAIN, 0, kDrainBudget);
+        if (t == 0) {
+            if (*abort_flag && issued > 0) {
+                umma_commit(bars + CR_DRAIN);
+                mbar_wait(bars + CR_DRAIN, 0, kDrainBudget);
+            }
+            if (stored > 0) bulk_wait_all();
         }
     } else if (lane == 0) {
-        // loader: Psi tiles of the unit's chunks
+        // loader: Psi and out tiles of the unit's chunks
         int ld = 0;
         const int tbi = (int)un.tb;
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
             const int b = c % CR_NBUF;
             if (c >= CR_NBUF && !wait_bar(CR_FREE0 + b, par((c - CR_NBUF) / CR_NBUF))) { fail(53); break; }
-            mbar_arrive_expect_tx(bars + CR_LD0 + b, 16384);
-            tma_load_3d(sm + b * 16384, &tm_psi, bars + CR_LD0 + b, 0, h, tbi + c * CC);
-            tma_load_3d(sm + b * 16384 + 8192, &tm_psi, bars + CR_LD0 + b, 64, h, tbi + c * CC);
+            unsigned char *buf = sm + b * CR_BUF;
+            mbar_arrive_expect_tx(bars + CR_LD0 + b, CR_BUF);
+            tma_load_3d(buf, &tm_psi, bars + CR_LD0 + b, 0, h, tbi + c * CC);
+            tma_load_3d(buf + 8192, &tm_psi, bars + CR_LD0 + b, 64, h, tbi + c * CC);
+            tma_load_3d(buf + CR_OUT, &tm_out, bars + CR_LD0 + b, 0, h, tbi + c * CC);
+            tma_load_3d(buf + CR_OUT + 8192, &tm_out, bars + CR_LD0 + b, 64, h, tbi + c * CC);
             ++ld;
         }
         if (*abort_flag)
@@ -1274,9 +1321,10 @@ cudaError_t launch_prefill_chain(const void *q, const void *k, const void *v, co
     segment_scan_kernel<<<dim3((unsigned)N, (unsigned)H_v, DD / 16), 256, 0, stream>>>(
         prm.ws_M, prm.ws_B, prm.ws_S, S_final, seqs, N, H_v, prm.units_per_seq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    CUtensorMap mpsi;
-    if (!make_map(&mpsi, prm.ws_Psi, T_total, H_v)) return cudaErrorInvalidValue;
-    segment_correct_kernel<<<dim3((unsigned)U, (unsigned)H_v), CR_THREADS, CR_SMEM, stream>>>(mpsi, prm);
+    CUtensorMap mpsi, mout;
+    if (!make_map(&mpsi, prm.ws_Psi, T_total, H_v) || !make_map(&mout, prm.out, T_total, H_v))
+        return cudaErrorInvalidValue;
+    segment_correct_kernel<<<dim3((unsigned)U, (unsigned)H_v), CR_THREADS, CR_SMEM, stream>>>(mpsi, mout, prm);
     return cudaGetLastError();
 }
 
