@@ -626,6 +626,7 @@ def run_prefill_only(args):
     stream = torch.cuda.Stream(device)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     x = inputs.prefill_inputs(w, device=device)
+    gdn.gdn_set_prefill_segment_tokens(args.segment_tokens)
     with ClockSampler(0) as clk:
         times, status, sched = time_prefill(gdn, x, w, max(1, args.steps), max(args.warmup, 1),
                                             stream, flush)
@@ -860,6 +861,9 @@ def main():
                     help="--section prefill: the workload (1 mid-size, 2 varlen, 3 long context)")
     ap.add_argument("--prefill-tokens", type=int, default=0,
                     help="--section prefill: keep only the first N tokens of each sequence")
+    ap.add_argument("--segment-tokens", type=int, default=0,
+                    help="--section prefill: schedule override (0 automatic, -1 one unit per "
+                         "sequence, -2 cluster kernel, else a segment length)")
     ap.add_argument("--qsa-seqs", type=int, default=8,
                     help="sequences of the QSA workload (1,048,576 cached tokens each)")
     args = ap.parse_args()

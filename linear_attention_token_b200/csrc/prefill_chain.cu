@@ -900,14 +900,13 @@ segment_scan_kernel(const float *ws_M, const float *ws_B, float *ws_S, float *S_
 // segment's start state to every token's output.  out[t] += Psi[t] S_in(p) for the
 // segment's tokens, on the tensor cores: (Psi S_in)^T = S_in^T Psi^T, A = S_in^T (bf16 in
 // TMEM, lane = value column), B = a 64-token tile of Psi (K-major rows, by TMA), D in TMEM.
-// The pass is bound by HBM (read Psi, read and write out), so every chunk's Psi and out
-// tiles come in by TMA several chunks ahead, the sum is formed in shared memory and a full
-// chunk goes back by a TMA store; the partial last chunk of a sequence is written row by
-// row, so no store reaches past the unit.
-// One CTA per (unit, value head), two per SM; 160 threads: warps 0-3 convert S_in and run
-// the epilogue (thread 0 issues the MMAs and the stores), warp 4 loads.
+// The pass streams Psi and out (read and written once), so every chunk's Psi and out tiles
+// come in by TMA a few chunks ahead; two warpgroups add D to the out tile, 32 tokens each,
+// and write the sums back as pairs of values.
+// One CTA per (unit, value head), two per SM; 288 threads: warps 0-7 convert S_in and run
+// the epilogue (thread 0 issues the MMAs), warp 8 loads.
 namespace {
-constexpr int CR_THREADS = 160, CR_NBUF = 3;
+constexpr int CR_THREADS = 288, CR_NBUF = 3;
 constexpr uint32_t CR_TM_A = 0, CR_TM_D = 64;          // TMEM: S_in^T bf16, two 64-column D
 constexpr uint32_t CR_BUF = 32768;                     // Psi tile (16 KB) | out tile (16 KB)
 constexpr uint32_t CR_OUT = 16384;
@@ -951,15 +950,17 @@ segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi,
     };
     auto fail = [&](int where) { chain_abort(abort_flag, prm.err, where); };
 
-    if (warp < 4) {
-        const int t = tid, v = tid;
-        const uint32_t loff = (uint32_t)(32 * warp) << 16;
+    if (warp < 8) {
+        const int t = tid, half = warp >> 2, v = 32 * (warp & 3) + lane;
+        const uint32_t loff = (uint32_t)(32 * (warp & 3)) << 16;
+        const bool odd = lane & 1;
         const uint32_t id_c = idesc_bf16(128, 64, false, false);
-        int issued = 0, stored = 0;
-        // S_in^T (bf16 pairs, lane v, column d / 2)
+        int issued = 0;
+        // S_in^T (bf16 pairs, lane v, column d / 2); warpgroup `half` converts d in
+        // [64 half, 64 half + 64)
         const float *src = prm.ws_S + ((size_t)blockIdx.x * prm.H_v + h) * DD * DD;
 #pragma unroll 1
-        for (int db = 0; db < 4; ++db) {
+        for (int db = 2 * half; db < 2 * half + 2; ++db) {
             uint32_t xb[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -970,7 +971,7 @@ segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi,
         }
         tmem_wait_st();
         tc_fence_before();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         auto issue = [&](int c) -> bool {        // thread 0; D(c & 1) was read at c - 2
             const int b = c % CR_NBUF;
             if (!wait_bar(CR_LD0 + b, par(c / CR_NBUF))) return false;
@@ -988,65 +989,52 @@ segment_correct_kernel(const __grid_constant__ CUtensorMap tm_psi,
         // element (token r, value v) of a 64-token out tile: two 64-value boxes of 128-byte
         // rows in the 128-byte swizzle
         const uint32_t vcol = (uint32_t)(v >> 6) * 8192u, vb2 = (uint32_t)(v & 63) * 2u;
-        const long long rstride = (long long)prm.H_v * DD;
+        const size_t rstride = (size_t)prm.H_v * DD;
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
             const int b = c % CR_NBUF;
-            // the store of chunk c - 1 has read its tile: the buffer goes back to the loader
-            // a whole chunk before the tile it will hold is needed.  The next chunk's MMA
-            // (into the D buffer read at c - 1) runs beside this chunk's epilogue.
-            if (t == 0) {
-                if (c >= 1) {
-                    bulk_wait_read_all();
-                    mbar_arrive_local(bars + CR_FREE0 + (c - 1) % CR_NBUF);
-                }
-                if (c + 1 < nch && !*abort_flag && !issue(c + 1)) fail(51);
-            }
+            // the next chunk's MMA (into the D buffer read at c - 1) runs beside this epilogue
+            if (t == 0 && c + 1 < nch && !*abort_flag && !issue(c + 1)) fail(51);
             uint32_t ok2;
             {
                 const bool w = t != 0 || (!*abort_flag && wait_bar(CR_DONE0 + (c & 1), par(c >> 1)));
-                asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+                asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 256, p;\n\t"
                              "selp.u32 %0, 1, 0, q;\n\t}" : "=r"(ok2) : "r"(w ? 1u : 0u) : "memory");
             }
             if (!ok2) { fail(52); break; }
             tc_fence_after();
-            const long long t0 = un.tb + (long long)c * CC;
-            const int L = (int)min((long long)CC, un.te - t0);
-            unsigned char *ot = sm + b * CR_BUF + CR_OUT + vcol;
-            uint32_t x0[32], x1[32];
-            tmem_ld32(tmem + loff + CR_TM_D + 64 * (c & 1), x0);
-            tmem_ld32(tmem + loff + CR_TM_D + 64 * (c & 1) + 32, x1);
+            uint32_t x[32];                          // tokens 32 half + j
+            tmem_ld32(tmem + loff + CR_TM_D + 64 * (c & 1) + 32 * half, x);
             tmem_wait_ld();
             tc_fence_before();
+            const long long t0 = un.tb + (long long)c * CC;
+            const int L = (int)min((long long)CC, un.te - t0);
+            const unsigned char *ot = sm + b * CR_BUF + CR_OUT + vcol;
+            // lanes (v, v ^ 1) pair up: the even lane writes token 2m's two values, the odd
+            // lane token 2m + 1's
+            __nv_bfloat16 *obase = prm.out + ((size_t)t0 * prm.H_v + h) * DD + (v & ~1);
 #pragma unroll
-            for (int r = 0; r < 64; ++r) {
-                const uint32_t off = (uint32_t)r * 128u + ((((vb2 >> 4) ^ (uint32_t)(r & 7)) << 4) | (vb2 & 15u));
-                __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(ot + off);
-                const float d = __uint_as_float(r < 32 ? x0[r] : x1[r - 32]);
-                const __nv_bfloat16 o = __float2bfloat16_rn(__bfloat162float(*e) + d);
-                if (L == CC) *e = o;
-                else if (r < L) prm.out[(size_t)(t0 + r) * rstride + (size_t)h * DD + v] = o;
-            }
-            if (L == CC) fence_proxy_async();
-            // every thread has read D(c) (the next MMA into it is issued at c + 1) and, for a
-            // full chunk, written the tile
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (t == 0) {
-                if (L == CC) {
-                    unsigned char *o0 = sm + b * CR_BUF + CR_OUT;
-                    tma_store_3d(&tm_out, o0, 0, h, (int)t0);
-                    tma_store_3d(&tm_out, o0 + 8192, 64, h, (int)t0);
-                    bulk_commit();
-                    ++stored;
+            for (int m = 0; m < 16; ++m) {
+                float o[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = 32 * half + 2 * m + e;
+                    const uint32_t off = (uint32_t)r * 128u + ((((vb2 >> 4) ^ (uint32_t)(r & 7)) << 4) | (vb2 & 15u));
+                    o[e] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(ot + off)) +
+                           __uint_as_float(x[2 * m + e]);
                 }
+                const float recv = __shfl_xor_sync(0xffffffffu, odd ? o[0] : o[1], 1);
+                const int r = 32 * half + 2 * m + (odd ? 1 : 0);
+                const uint32_t val = odd ? pack2(recv, o[1]) : pack2(o[0], recv);
+                if (r < L) *reinterpret_cast<uint32_t *>(obase + (size_t)r * rstride) = val;
             }
+            // every thread has read D(c) and both tiles: the buffer goes back to the loader
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (t == 0) mbar_arrive_local(bars + CR_FREE0 + b);
         }
-        if (t == 0) {
-            if (*abort_flag && issued > 0) {
-                umma_commit(bars + CR_DRAIN);
-                mbar_wait(bars + CR_DRAIN, 0, kDrainBudget);
-            }
-            if (stored > 0) bulk_wait_all();
+        if (t == 0 && *abort_flag && issued > 0) {
+            umma_commit(bars + CR_DRAIN);
+            mbar_wait(bars + CR_DRAIN, 0, kDrainBudget);
         }
     } else if (lane == 0) {
         // loader: Psi and out tiles of the unit's chunks
@@ -1180,10 +1168,10 @@ struct PrefillPlan {
 // whose chain per value-column quarter is shorter but takes four SMs per head.
 constexpr double kChainStep = 8400.0, kClusterStep = 4700.0;
 constexpr double kFill = 3.0;           // chunk steps to fill a pipeline at a unit's start
-// The output correction streams Psi and updates out in place; measured, each of its CTAs
+// The output correction streams Psi and out in and out once; measured, each of its CTAs
 // moves about kCorrectCtaBps and the whole pass about kCorrectBps at most.  kStepSeconds
-// converts its time into chunk steps.
-constexpr double kCorrectCtaBps = 12e9, kCorrectBps = 3e12, kStepSeconds = 4.3e-6;
+// (kChainStep at the full clock) converts its time into chunk steps.
+constexpr double kCorrectCtaBps = 21e9, kCorrectBps = 6e12, kStepSeconds = 4.3e-6;
 
 // Schedule for a call: the cluster kernel (one wave of four-CTA clusters per (sequence,
 // value head)), or this kernel with one unit per sequence, or this kernel with segments of
@@ -1208,7 +1196,14 @@ PrefillPlan plan_prefill(int N, long long T_total, int H_v, int sms, int overrid
     if (cluster < best) { best = cluster; pl.kind = PrefillPlan::kCluster; }
     // bytes of out (read and written) and Psi (read), bf16, of the segments past the first
     const double corr_bytes = (double)T_total * H_v * DD * 2 * 3;
-    for (long long L = 8; L < C; L += (L < 64 ? 4 : (L < 512 ? 16 : 64))) {
+    // segment lengths (in chunks) from the longest down: a shorter segment (more segments,
+    // more transfer chains and correction) must be 3 % better to be taken
+    long long Ls[128];
+    int nL = 0;
+    for (long long L = 8; L < C && nL < 128; L += (L < 64 ? 4 : (L < 512 ? 16 : (L < 4096 ? 64 : 512))))
+        Ls[nL++] = L;
+    for (int i = nL - 1; i >= 0; --i) {
+        const long long L = Ls[i];
         const long long P = (C + L - 1) / L;
         const double ctas = (double)(P - 1) * units0;
         const double corr = corr_bytes * (double)(P - 1) / (double)P /

@@ -65,15 +65,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
           "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
-// Tiled store of a box from this CTA's shared memory, tracked by this thread's bulk
-// async-groups (bulk_commit / bulk_wait_*).  Coordinates must not be negative.
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1,
-                                             int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
-        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -17,7 +17,7 @@ math); this module only marshals numpy arrays.  Every function here is pinned
 by tests/test_oracle.py (exact rational brute force, a hand-worked example,
 closed forms and invariants) and by tests/test_oracle_mutants.py.  The backward passes live
 in oracle/backward.py (sequential) and oracle/backward_chunked.py (chunked); the QSA
-indexer in oracle/qsa.py.
+indexer in oracle/qsa.py; the segmented (sequence-parallel) form in oracle/segments.py.
 """
 from __future__ import annotations
 
