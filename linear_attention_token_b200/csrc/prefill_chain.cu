@@ -1168,6 +1168,7 @@ struct PrefillPlan {
 // whose chain per value-column quarter is shorter but takes four SMs per head.
 constexpr double kChainStep = 8400.0, kClusterStep = 4700.0;
 constexpr double kFill = 3.0;           // chunk steps to fill a pipeline at a unit's start
+constexpr double kScanStep = 1.5;       // chunk steps per segment of the (sequential) scan
 // The output correction streams Psi and out in and out once; measured, each of its CTAs
 // moves about kCorrectCtaBps and the whole pass about kCorrectBps at most.  kStepSeconds
 // (kChainStep at the full clock) converts its time into chunk steps.
@@ -1208,7 +1209,8 @@ PrefillPlan plan_prefill(int N, long long T_total, int H_v, int sms, int overrid
         const double ctas = (double)(P - 1) * units0;
         const double corr = corr_bytes * (double)(P - 1) / (double)P /
                             std::min(kCorrectBps, ctas * kCorrectCtaBps) / kStepSeconds;
-        const double t = (waves((2 * P - 1) * units0, sms) * ((double)L + kFill) + 4.0 + corr) * kChainStep;
+        const double t = (waves((2 * P - 1) * units0, sms) * ((double)L + kFill) + kScanStep * (double)P + corr) *
+                         kChainStep;
         if (t < 0.97 * best) { best = t; pl.kind = PrefillPlan::kChain; pl.seg_tokens = (int)(L * CC); }
     }
     return pl;
