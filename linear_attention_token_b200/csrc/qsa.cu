@@ -316,6 +316,21 @@ __device__ void threshold_of(const uint32_t *h, int elig, int budget, int *scrat
 // holds its 16 dims of all T summed queries; the T partial dots are summed over the group
 // transposed, so lane j of the group ends with query j's score.
 constexpr int kScoreUnroll = 4;
+constexpr int kMmaTiles = 2;            // 16-row tiles per warp and pass (T > 1 path)
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+// D += A (16 x 16, bf16, row-major fragment) * B (16 x 8, bf16, column fragment), fp32 D
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 template <int T>
 __global__ void __launch_bounds__(kScoreThreads, T == 1 ? 4 : 2) qsa_score_kernel(
@@ -369,7 +384,78 @@ __global__ void __launch_bounds__(kScoreThreads, T == 1 ? 4 : 2) qsa_score_kerne
         }
         __syncthreads();
         float *sc = scores + (size_t)T * row0;     // query j's scores at sc + j * cached
-        {
+        if constexpr (T > 1) {
+            // Several queries: the rows against the T summed queries as a skinny contraction
+            // on the tensor cores, 16 rows per m16n8k16 tile.  Column n of B holds the high
+            // (n < 4) or low (n >= 4) bf16 part of summed query n & 3, so a score keeps about
+            // 16 significant bits of the query (the keys are bf16 already) and is the sum of
+            // columns j and j + 4.  The 128 dims are permuted consistently in A and B so that
+            // lane (g, t) reads dims [32 t, 32 t + 32) of rows g and g + 8 as four 16-byte
+            // loads each: in k step s its fragment pairs are dims 32 t + 4 s + {0, 1} and
+            // + {2, 3}.
+            const int g = lane >> 2, t4 = lane & 3;
+            uint32_t bq[8][2];
+            {
+                const int j = g & 3;
+                const bool lo = g >= 4;
+#pragma unroll
+                for (int st = 0; st < 8; ++st)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int d = 32 * t4 + 4 * st + 2 * hh;
+                        const float x0 = j < T ? qbar[j * QD + d] : 0.f;
+                        const float x1 = j < T ? qbar[j * QD + d + 1] : 0.f;
+                        const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
+                        const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
+                        bq[st][hh] = lo ? pack_bf16x2(x0 - h0, x1 - h1) : pack_bf16x2(x0, x1);
+                    }
+            }
+            // after the exchange lane t4 reports queries jq, jq + 1 of row g (t4 < 2) or
+            // row g + 8 (t4 >= 2)
+            const int jq = 2 * (t4 & 1);
+            const bool upper = t4 >= 2;
+            const int eqa = jq < T ? eligible(cu_blocks, q_pos, n, total_blocks, jq) : 0;
+            const int eqb = jq + 1 < T ? eligible(cu_blocks, q_pos, n, total_blocks, jq + 1) : 0;
+            const __nv_bfloat16 *kb = k_hat + (size_t)row0 * QD + 32 * t4;
+            constexpr int kWarps = kScoreThreads / 32;
+            for (int tb = r0 + 16 * warp; tb < r1; tb += 16 * kWarps * kMmaTiles) {
+                uint4 ra[kMmaTiles][2][4];
+#pragma unroll
+                for (int u = 0; u < kMmaTiles; ++u)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int row = tb + 16 * kWarps * u + g + 8 * hh;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            ra[u][hh][i] = row < r1 ? ld_stream(kb + (size_t)row * QD + 8 * i)
+                                                    : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                for (int u = 0; u < kMmaTiles; ++u) {
+                    const uint32_t *wa = reinterpret_cast<const uint32_t *>(ra[u][0]);
+                    const uint32_t *wb = reinterpret_cast<const uint32_t *>(ra[u][1]);
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int st = 0; st < 8; ++st)
+                        mma_bf16_16816(d, wa[2 * st], wb[2 * st], wa[2 * st + 1], wb[2 * st + 1],
+                                       bq[st][0], bq[st][1]);
+                    // lane t4 holds columns 2 t4, 2 t4 + 1 of rows g (d0, d1) and g + 8 (d2,
+                    // d3); its partner t4 ^ 2 holds the other part of the same two queries
+                    const float x0 = __shfl_xor_sync(0xffffffffu, upper ? d[0] : d[2], 2);
+                    const float x1 = __shfl_xor_sync(0xffffffffu, upper ? d[1] : d[3], 2);
+                    const float sa = (upper ? d[2] : d[0]) + x0, sb = (upper ? d[3] : d[1]) + x1;
+                    const int row = tb + 16 * kWarps * u + g + (upper ? 8 : 0);
+                    if (row < eqa) {
+                        sc[(size_t)jq * cached + row] = sa;
+                        atomicAdd(&hist[jq * HBINS + (order_key(sa) >> (32 - HBITS))], 1u);
+                    }
+                    if (row < eqb) {
+                        sc[(size_t)(jq + 1) * cached + row] = sb;
+                        atomicAdd(&hist[(jq + 1) * HBINS + (order_key(sb) >> (32 - HBITS))], 1u);
+                    }
+                }
+            }
+        } else {
             constexpr int TP = T == 1 ? 1 : (T == 2 ? 2 : 4);
             const int g = lane >> 3, gl = lane & 7;
             float qv[T][16];
