@@ -60,24 +60,32 @@ def test_decode_steps_replay():
     assert w.decode_steps > 0
 
 
-def test_prefill_replay():
+@pytest.mark.parametrize("schedule", [0, -1, 128, -2])
+def test_prefill_replay(schedule):
+    """Every prefill schedule captures: automatic, one unit per sequence, 128-token segments
+    (unit table, local and transfer chains, scan, correction) and the cluster kernel."""
     lens = [300, 517]
     x = inputs.draw(sum(lens), 4, 8, 128, 128, torch.bfloat16, 73, DEV)
     S0 = inputs.draw_state(2, 8, 128, 128, 0.05, 74, DEV)
     cu = inputs.cu_seqlens_of(lens).to(DEV)
     out = torch.empty_like(x["v"])
     Sf = torch.empty(2, 8, 128, 128, device=DEV)
-    ws = gdn.prefill_workspace(2, sum(lens), 8, 128, 128)
-    call = lambda: gdn.gdn_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], S0, cu, out=out,
-                                   S_final=Sf, workspace=ws)
-    call()
-    torch.cuda.synchronize()
-    want_o, want_S = out.clone(), Sf.clone()
-    g = _capture(call)
-    out.zero_(); Sf.zero_()
-    g.replay()
-    torch.cuda.synchronize()
-    assert torch.equal(out, want_o) and torch.equal(Sf, want_S)
+    gdn.gdn_set_prefill_segment_tokens(schedule)
+    try:
+        ws = gdn.prefill_workspace(2, sum(lens), 8, 128, 128)
+        call = lambda: gdn.gdn_prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], S0, cu,
+                                       out=out, S_final=Sf, workspace=ws)
+        call()
+        torch.cuda.synchronize()
+        want_o, want_S = out.clone(), Sf.clone()
+        g = _capture(call)
+        for _ in range(2):
+            out.zero_(); Sf.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(out, want_o) and torch.equal(Sf, want_S)
+    finally:
+        gdn.gdn_set_prefill_segment_tokens(0)
     assert gdn.gdn_get_device_error(ws) == gdn.GDN_OK
 
 
