@@ -75,8 +75,8 @@ def test_traffic_key_ignores_comments_only(bench, tmp_path):
 def test_traffic_file_is_well_formed():
     """Each entry: kernel key, 16 hex digits of the code key, bytes per launch.  (An entry
     whose code key no longer matches the source is allowed: bench.py then reports null.)"""
-    known = {"prefill", "decode", "decode_multi", "backward", "qsa_score", "qsa_compress",
-             "qsa_score_t4"}
+    known = {"prefill_long", "prefill", "decode", "decode_multi", "backward", "qsa_score",
+             "qsa_compress", "qsa_score_t4"}
     n = 0
     for line in open(os.path.join(ROOT, "profiles", "traffic.txt")):
         if not line.strip() or line.startswith("#"):
