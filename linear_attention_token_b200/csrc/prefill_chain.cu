@@ -115,6 +115,7 @@ enum Bar {
     B_RF0, B_RF1, B_RF2,               // commit: region free (after C2)
     B_PF0, B_PF1, B_PF2,               // commit: P tile free (after C3)
     B_VF0, B_VF1, B_VF2,               // chain: vector buffer free
+    B_KS0, B_KS1, B_KS2,               // output group: K~ of the region's chunk scaled (C2 may read)
     B_DRAIN0, B_DRAIN1, B_DRAIN2,
     B_COUNT
 };
@@ -390,16 +391,20 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (t == 0) {
                 if (!xa) mbar_arrive_local(bars + B_UF0 + (c & 1));
                 mbar_arrive_local(bars + rbar(B_VF0, c));
-                tc_fence_after();
-                // ---- C2: S^T += U^T K~
-                const uint32_t kreg = smem_u32(region(c));
+                // ---- C2: S^T += U^T K~, once the output group has scaled K~
+                if (!wait_bar(rbar(B_KS0, c), rpar(c))) {
+                    fail(7);
+                } else {
+                    tc_fence_after();
+                    const uint32_t kreg = smem_u32(region(c));
 #pragma unroll 1
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(tmem + TM_S, sdesc_kmajor(su + ks * 32),
-                              sdesc_mnmajor(kreg + ks * 2048, SR_KB), id_c2, 1);
-                umma_commit(bars + B_C2);
-                umma_commit(bars + rbar(B_RF0, c));
-                ++mma_issued;
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tmem + TM_S, sdesc_kmajor(su + ks * 32),
+                                  sdesc_mnmajor(kreg + ks * 2048, SR_KB), id_c2, 1);
+                    umma_commit(bars + B_C2);
+                    umma_commit(bars + rbar(B_RF0, c));
+                    ++mma_issued;
+                }
             } else if (t == 32) {
                 // ---- C3: O^T += U^T P^T, issued beside C2 (off the chain)
                 tc_fence_after();
@@ -688,12 +693,9 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                 }
                 tc_fence_before();
-                // ---- K~ = diag(dte) K and Q~ = diag(gamma) Q, rows in place
-                {
-                    const int r = t & 63, kb = t >> 6;
-                    scale_row128(rg + kb * SR_KB + r * 128, r, vb[V_DTE + r]);
-                    scale_row128(rg + kb * SR_KB + SR_Q + r * 128, r, vb[V_GAM + r]);
-                }
+                // ---- Q~ = diag(gamma) Q, rows in place: with W, what C1 reads
+                const int r = t & 63, kb = t >> 6;
+                scale_row128(rg + kb * SR_KB + SR_Q + r * 128, r, vb[V_GAM + r]);
                 fence_proxy_async();
                 group_sync<3>();
                 if (t == 0) {
@@ -701,7 +703,16 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     mbar_arrive_local(bars + rbar(B_RDY0, c));
                 }
             }
+            // the outputs of chunk c - 1 (the chain's next C1 waits for their read-out) ...
             if (c >= 1 && !outputs(c - 1)) { fail(21); break; }
+            // ... then K~ = diag(dte) K in place, which only C2(c) reads, after C1 and E3
+            if (c < nch) {
+                const int r = t & 63, kb = t >> 6;
+                scale_row128(region(c) + kb * SR_KB + r * 128, r, vecbuf(c)[V_DTE + r]);
+                fence_proxy_async();
+                group_sync<3>();
+                if (t == 0) mbar_arrive_local(bars + rbar(B_KS0, c));
+            }
         }
     } else if (warp == 12) {
         // =============================================================== prep issuer
@@ -727,31 +738,56 @@ prefill_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 ++issued;
                 return true;
             };
-            if (nch > 0 && !issue_p1(0)) fail(30);
-#pragma unroll 1
-            for (int c = 0; c < nch && !*abort_flag; ++c) {
+            // P2 (W^T = K^T T'^T) and P3 (-U~^T = V^T (-T'')^T, V in the W slots, into the
+            // -U^T buffer of the chunk's parity once C2 and C3 of chunk c - 2 have read the
+            // U^T left there; the transfer chain has U~ = 0 and no P3)
+            auto issue_p23 = [&](int c) -> bool {
                 const uint32_t rg = smem_u32(region(c));
-                // the next chunk's P1 goes out as soon as this chunk's A/P epilogue has read
-                // the accumulator, ahead of this chunk's P2 and P3
-                if (c + 1 < nch && !issue_p1(c + 1)) { fail(30); break; }
-                // P2: W^T = K^T T'^T
-                if (!wait_bar(B_TT, par(c)) || (c > 0 && !wait_bar(B_WTF, par(c - 1)))) { fail(31); break; }
                 tc_fence_after();
 #pragma unroll 1
                 for (int ks = 0; ks < 4; ++ks)
                     umma_bf16(tmem + TM_WT, sdesc_mnmajor(rg + ks * 2048, SR_KB), sdesc_kmajor(tpa + ks * 32),
                               id_p23, ks > 0);
                 umma_commit(bars + B_P2);
-                // P3: -U~^T = V^T (-T'')^T, V in the W slots, into the -U^T buffer of the
-                // chunk's parity once E3(c - 2) has read it (transfer M: U~ = 0, no P3)
                 if (!xa) {
-                    if (c > 1 && !wait_bar(B_UF0 + (c & 1), par((c >> 1) - 1))) { fail(32); break; }
+                    if (c > 1 && !wait_bar(B_UF0 + (c & 1), par((c >> 1) - 1))) return false;
                     tc_fence_after();
 #pragma unroll 1
                     for (int ks = 0; ks < 4; ++ks)
                         umma_bf16(tmem + ((c & 1) ? TM_WU1 : TM_WU0), sdesc_mnmajor(rg + SR_W + ks * 2048, SR_KB),
                                   sdesc_kmajor(tpa + 8192 + ks * 32), id_p23, ks > 0);
                     umma_commit(bars + B_P30 + (c & 1));
+                }
+                return true;
+            };
+            if (nch > 0 && !issue_p1(0)) fail(30);
+            // Chunk c: P1 of chunk c + 1 (its tiles landed, the accumulator read for chunk c)
+            // and P2, P3 of chunk c (T' of chunk c formed, W^T of chunk c - 1 read), in
+            // whichever order their inputs arrive: a region that the chain frees late then
+            // holds back P1 only, not this chunk's W and U~.  Polled with short naps, at most
+            // `budget` polls per chunk.
+#pragma unroll 1
+            for (int c = 0; c < nch && !*abort_flag; ++c) {
+                bool need_p1 = c + 1 < nch, need_p23 = true;
+                uint32_t polls = 0;
+                while (need_p1 || need_p23) {
+                    if (*abort_flag) break;
+                    if (need_p1 &&
+                        (L2N ? mbar_try_wait(bars + B_IN, par(c + 1))
+                             : mbar_try_wait(bars + rbar(B_LD0, c + 1), rpar(c + 1))) &&
+                        mbar_try_wait(bars + B_KQF, par(c))) {
+                        need_p1 = false;
+                        if (!issue_p1(c + 1)) { fail(30); break; }
+                        continue;
+                    }
+                    if (need_p23 && mbar_try_wait(bars + B_TT, par(c)) &&
+                        (c == 0 || mbar_try_wait(bars + B_WTF, par(c - 1)))) {
+                        need_p23 = false;
+                        if (!issue_p23(c)) { fail(32); break; }
+                        continue;
+                    }
+                    if (++polls > budget) { fail(need_p23 ? 31 : 30); break; }
+                    __nanosleep(200);
                 }
             }
             if (*abort_flag && issued > 0) {
