@@ -1234,15 +1234,12 @@ PrefillPlan plan_prefill(int N, long long T_total, int H_v, int sms, int overrid
     if (cluster < best) { best = cluster; pl.kind = PrefillPlan::kCluster; }
     // bytes of out (read and written) and Psi (read), bf16, of the segments past the first
     const double corr_bytes = (double)T_total * H_v * DD * 2 * 3;
-    // segment lengths (in chunks) from the longest down: a shorter segment (more segments,
-    // more transfer chains and correction) must be 3 % better to be taken
-    long long Ls[128];
-    int nL = 0;
-    for (long long L = 8; L < C && nL < 128; L += (L < 64 ? 4 : (L < 512 ? 16 : (L < 4096 ? 64 : 512))))
-        Ls[nL++] = L;
-    for (int i = nL - 1; i >= 0; --i) {
-        const long long L = Ls[i];
-        const long long P = (C + L - 1) / L;
+    // segment counts from the fewest up, each with segments of equal length L = ceil(C / P)
+    // chunks (so the last one is not left short while the others set the time); more
+    // segments (more transfer chains, scan steps and correction) must be 3 % better
+    for (long long P = 2; P <= C / 8; ++P) {
+        const long long L = (C + P - 1) / P;
+        if ((C + L - 1) / L != P) continue;              // that length is P' < P segments
         const double ctas = (double)(P - 1) * units0;
         const double corr = corr_bytes * (double)(P - 1) / (double)P /
                             std::min(kCorrectBps, ctas * kCorrectCtaBps) / kStepSeconds;
