@@ -65,9 +65,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
           "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
 
 // Generic-proxy shared-memory writes made visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async() {
@@ -326,10 +323,6 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
     uint32_t v;
     asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
     return v;
-}
-// 32-bit store to a shared::cluster address (another CTA's shared memory)
-__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled tile
