@@ -56,6 +56,11 @@ struct BwShared {
     float red[DK / 32][BW_BV];
     float col[BW_BV];
     float scal[DK / 32][2];
+    // the backward walk's per-token reductions, by token parity (a buffer is written again
+    // two tokens later, after both barriers of the token in between)
+    float bred[2][DK / 32][BW_BV];
+    float bcol[2][BW_BV];
+    float bscal[2][DK / 32];
 };
 
 }  // namespace
@@ -212,25 +217,26 @@ backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             }
             atomicAdd(dq + ((size_t)t * H_qk + hq) * DK + r, dq_part);
             // du = dS^T k (over rows)
+            const int pb = i & 1;
             float x[BW_BV];
 #pragma unroll
             for (int j = 0; j < BW_BV; ++j) x[j] = dS[j] * kr;
             {
                 const float part = warp_transpose_sum(x, lane);
-                if (lane < BW_BV) sm.red[warp][lane] = part;
+                if (lane < BW_BV) sm.bred[pb][warp][lane] = part;
             }
             // this row's share of <dS, S_{t-1}>
             float dal_part = 0.f;
 #pragma unroll
             for (int j = 0; j < BW_BV; ++j) dal_part += dS[j] * sp[j];
             dal_part = warp_sum(dal_part);
-            if (lane == 0) sm.scal[warp][0] = dal_part;
+            if (lane == 0) sm.bscal[pb][warp] = dal_part;
             __syncthreads();
             if (r < BW_BV) {
                 float du = 0.f;
 #pragma unroll
-                for (int w = 0; w < NW; ++w) du += sm.red[w][r];
-                sm.col[r] = du;
+                for (int w = 0; w < NW; ++w) du += sm.bred[pb][w][r];
+                sm.bcol[pb][r] = du;
                 dv[((size_t)t * H_v + h) * DV + c0 + r] = bt * du;
             }
             __syncthreads();
@@ -238,20 +244,20 @@ backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             float dk_part = 0.f;
 #pragma unroll
             for (int j = 0; j < BW_BV; ++j) {
-                const float du = sm.col[j];
+                const float du = sm.bcol[pb][j];
                 dk_part += dS[j] * sm.u[i][j] - al * bt * du * sp[j];
             }
             atomicAdd(dk + ((size_t)t * H_qk + hq) * DK + r, dk_part);
             if (warp == 0) {
                 // dbeta (slice share) = <du, v - alpha a>;  -beta <du, a> joins dalpha
                 const bool on = lane < BW_BV;
-                const float du = on ? sm.col[lane] : 0.f, a = on ? sm.a[i][lane] : 0.f;
+                const float du = on ? sm.bcol[pb][lane] : 0.f, a = on ? sm.a[i][lane] : 0.f;
                 const float db = warp_sum(on ? du * (sm.v[i][lane] - al * a) : 0.f);
                 const float da_dot = warp_sum(du * a);
                 if (lane == 0) {
                     float dal = 0.f;
 #pragma unroll
-                    for (int w = 0; w < NW; ++w) dal += sm.scal[w][0];
+                    for (int w = 0; w < NW; ++w) dal += sm.bscal[pb][w];
                     dal -= bt * da_dot;
                     const size_t gi = (size_t)t * H_v + h;
                     atomicAdd(dg + gi, al * dal * sm.dgate_g[i]);
@@ -260,10 +266,9 @@ backward_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn 
             }
             // dS <- alpha dS + k da^T
 #pragma unroll
-            for (int j = 0; j < BW_BV; ++j) dS[j] = al * dS[j] - kr * al * bt * sm.col[j];
+            for (int j = 0; j < BW_BV; ++j) dS[j] = al * dS[j] - kr * al * bt * sm.bcol[pb][j];
 #pragma unroll
             for (int j = 0; j < BW_BV; ++j) s[j] = sp[j];
-            __syncthreads();                     // sm.col, sm.red, sm.scal reused next token
         }
     }
     if (dS0) {
