@@ -67,8 +67,10 @@ typedef enum {
  * error word; they must be zero-filled before first use.  When few (sequence, value
  * head) pairs would leave most SMs idle (long sequences, few heads), the bf16 tensor-core
  * path splits each sequence into segments that run in parallel; the rest of this size
- * then holds each segment's state transfer (two dk x dk / dk x dv fp32 matrices) and
- * start state.  gdn_prefill accepts any workspace of at least 256 bytes: a smaller one
+ * then holds each segment's state transfer and start state (three dk x dv fp32 matrices
+ * per segment and value head) and the transfer chains' per-token outputs Psi
+ * (T_total x H_v x dk bf16: 1.07 GB for 262,144 tokens x 16 heads).  gdn_prefill
+ * accepts any workspace of at least 256 bytes: a smaller one
  * than this size makes it run one unit per sequence (same results, less parallelism).
  * The workspace must stay allocated while work that uses it is in flight, and calls
  * that share one must not overlap on the GPU. */
@@ -208,7 +210,8 @@ gdn_status gdn_prefill_static_scratch(const void *q, const void *k, const void *
  * value columns, and a cluster of four CTAs per (sequence, value head) that splits the
  * value columns and shares each chunk's preparation.
  *    0  automatic (default): a cost model of the device's SM count picks the kernel and,
- *       for the first, whether to segment long sequences;
+ *       for the first, whether to cut long sequences into segments and into how many
+ *       (segments of equal length);
  *   -1  the single-CTA kernel, one unit per sequence;
  *   -2  the four-CTA cluster kernel;
  *   >0  the single-CTA kernel with segments of exactly this many tokens (a multiple of
