@@ -40,10 +40,11 @@
 // Roles (448 threads):
 //   warps 0-3    chain group: E3 and E4; thread 0 issues C1 and C2, thread 32 issues C3
 //   warps 4-7    prep group: A/P epilogue, triangular inverse (in place), T' and -T''
-//   warps 8-11   output group: W rows from W^T, Q~ and K~ in place (finishing a chunk's
-//                preparation), then O^T -> out for the chunk before
-//   warp 12      prep issuer: MMAs P1 ([K;Q] K^T), P2 (W^T = K^T T'^T), P3 (-U~^T = V^T (-T'')^T,
-//                into the -U buffer of the chunk's parity)
+//   warps 8-11   output group: W rows from W^T and Q~ in place (the chunk is then ready for
+//                C1), O^T -> out for the chunk before, then K~ in place (for C2)
+//   warp 12      prep issuer: MMAs P1 ([K;Q] K^T) of the next chunk and P2 (W^T = K^T T'^T),
+//                P3 (-U~^T = V^T (-T'')^T, into the -U buffer of the chunk's parity) of this
+//                one, in whichever order their inputs arrive
 //   warp 13      loader: TMA of K, Q, V; per-chunk vectors (g, beta -> G, gamma, ...)
 // Every wait is bounded: a role whose wait runs out records GDN_ERR_TIMEOUT, raises the
 // CTA's abort flag so the other roles stop at their next wait, and the CTA drains its
