@@ -73,7 +73,11 @@ typedef enum {
  * accepts any workspace of at least 256 bytes: a smaller one
  * than this size makes it run one unit per sequence (same results, less parallelism).
  * The workspace must stay allocated while work that uses it is in flight, and calls
- * that share one must not overlap on the GPU. */
+ * that share one must not overlap on the GPU.
+ * Besides the workspace, the library's module holds 20 MB of static device memory on
+ * every GPU that loads it: the four-CTA cluster kernel's ring of prepared chunks
+ * (64 cluster slots of 320 KB).  A cluster claims one slot for its lifetime; 64 is more
+ * than the clusters one B200 can hold at once, so concurrent calls never share a slot. */
 size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t T_total, int32_t H_v, int32_t dk,
                                   int32_t dv);
 
